@@ -1,0 +1,397 @@
+"""fp64 CPU oracle for the OLMoE mixture-of-experts FFN layer.
+
+TEST INFRASTRUCTURE. Only the tests, the smoke check and the CPU-baseline leg of
+the benchmark may import this module. The product path (the CUDA library and its
+Python binding) never calls it, and this module imports nothing from the product.
+
+Everything here is plain numpy in float64, written to be read against the pages
+it cites, not to be fast. Inputs are taken as already-rounded values (bf16 or
+fp32 tensors converted to float64), so the oracle and the GPU see identical
+numbers. Pages cited:
+
+  [OLMoE-Guide]  "OLMoE Guide: 64-Expert Fine-Grained Open MoE Architecture",
+                 section "Router Mechanics & Loss Formulations" (routing formula,
+                 auxiliary load-balancing loss, router z-loss) and "Hands-On
+                 Implementation" (the PyTorch layer).
+  [MoE-scratch]  "Mixture-of-experts LLMs from scratch with OLMoE",
+                 section 2 "The router and the experts" (softmax_topk, Experts,
+                 dispatch, dense_run) and section 3 "OLMoE in PyTorch" (the config
+                 dump with norm_topk_prob False, RMSNorm, the fp32 residual).
+  [OLMoE-paper]  "OLMoE: Open Mixture-of-Experts Language Models" (summary page),
+                 "Pretraining architecture" (dropless token choice, loss weights
+                 alpha and beta), sections 4.1.6 and 4.1.7.
+
+Readings taken where the pages are silent or disagree (each is also listed in
+the design notes):
+  * Routing: softmax over all E experts, then the k largest probabilities are
+    both the choice and the weights, with no renormalisation ([MoE-scratch] §2
+    and §3, norm_topk_prob False). [OLMoE-Guide]'s top-k-then-softmax formula
+    contradicts this and is not used.
+  * Ties in the top-k: the lower expert index wins; slots are ordered by
+    descending probability.
+  * L_lb is reported unscaled, E * sum_i f_i * P_i with f_i = count_i / (T*k);
+    L_z is reported unscaled, mean_t lse_t^2. alpha and beta weight them only in
+    the backward objective  <dy, y> + alpha * L_lb + beta * L_z.
+  * No gradient flows through the expert choice or through f ([OLMoE-Guide]
+    computes f with bincount, a count).
+
+Parity pins for every function live in tests/test_oracle_pins.py.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "router_logits",
+    "softmax_lse",
+    "topk_no_renorm",
+    "near_tie_tokens",
+    "load_balance_loss",
+    "router_z_loss",
+    "dispatch_order",
+    "silu",
+    "swiglu_expert",
+    "experts_grouped",
+    "experts_dense",
+    "moe_forward",
+    "moe_objective",
+    "moe_backward",
+    "rms_norm",
+    "stack_forward",
+]
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------- router
+
+
+def router_logits(x, w_router, router_bias=None):
+    """Router scores h_t = W_r x_t (+ b), for every token and every expert.
+
+    [OLMoE-Guide] "Top-8 Softmax Routing Formulation": h(x) = W_g x with W_g of
+    shape (E, d). [MoE-scratch] §2: the router is one matrix with a row per
+    expert, s = W_r x; §3 MoE.forward: scores are taken in 32-bit floats and an
+    optional per-expert offset (the keep-mask) is applied before the softmax.
+    `router_bias` is that per-expert additive offset, shape (E,), or None.
+    Returns h of shape (T, E), float64.
+    """
+    h = _f64(x) @ _f64(w_router).T
+    if router_bias is not None:
+        h = h + _f64(router_bias)[None, :]
+    return h
+
+
+def softmax_lse(h):
+    """Softmax over all experts and its log-normaliser.
+
+    p_{t,i} = exp(h_{t,i}) / sum_j exp(h_{t,j}),  lse_t = log sum_j exp(h_{t,j}).
+    [MoE-scratch] §2 softmax_topk takes the softmax over all experts first;
+    [OLMoE-Guide] "Router Z-Loss Regularization" defines the log-sum-exp.
+    The maximum is subtracted first so exp never overflows.
+    """
+    h = _f64(h)
+    m = h.max(axis=1, keepdims=True)
+    e = np.exp(h - m)
+    s = e.sum(axis=1, keepdims=True)
+    return e / s, (m + np.log(s))[:, 0]
+
+
+def topk_no_renorm(p, k):
+    """The k largest probabilities per token, without renormalisation.
+
+    [MoE-scratch] §2 softmax_topk (OLMoE's router) and §3 (norm_topk_prob False):
+    the chosen experts are the k largest softmax probabilities and their weights
+    are those probabilities unchanged, so they sum to less than one.
+    Ties are broken towards the lower expert index (a stable sort of -p).
+    Returns (idx [T,k] int64, w [T,k] float64), slots in descending p.
+    """
+    p = _f64(p)
+    order = np.argsort(-p, axis=1, kind="stable")[:, :k]
+    return order.astype(np.int64), np.take_along_axis(p, order, axis=1)
+
+
+def near_tie_tokens(p, k, rel=1e-6):
+    """Tokens whose selection or slot order is decided by a near-tie.
+
+    A token is flagged when two neighbours among its k+1 largest probabilities
+    differ by less than `rel` relative to the larger one. For such tokens a
+    different rounding order may legitimately pick or order experts
+    differently, so parity on indices is counted separately for them.
+    """
+    p = _f64(p)
+    s = -np.sort(-p, axis=1)[:, : min(k + 1, p.shape[1])]
+    gaps = s[:, :-1] - s[:, 1:]
+    return np.any(gaps < rel * s[:, :-1], axis=1)
+
+
+def load_balance_loss(idx, p, n_experts):
+    """Switch-style load-balancing loss, unscaled: E * sum_i f_i * P_i.
+
+    [OLMoE-Guide] "Auxiliary Load Balancing Loss": f_i is the fraction of the
+    T*k token-slot assignments that went to expert i (a bincount, no gradient),
+    P_i is the mean over tokens of the full softmax probability of expert i.
+    Returns (L_lb, counts [E] int64).
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    counts = np.bincount(idx.reshape(-1), minlength=n_experts)
+    f = counts / float(T * k)
+    P = _f64(p).mean(axis=0)
+    return float(n_experts * np.sum(f * P)), counts
+
+
+def router_z_loss(lse):
+    """Router z-loss, unscaled: (1/T) * sum_t lse_t^2 ([OLMoE-Guide] "Router Z-Loss")."""
+    lse = _f64(lse)
+    return float(np.mean(lse * lse))
+
+
+# --------------------------------------------------------------------------- dispatch
+
+
+def dispatch_order(idx, n_experts):
+    """Grouping of (token, slot) pairs by expert, as in [MoE-scratch] §2 `dispatch`.
+
+    The pairs are the flattened [T, k] choice matrix (pair id = t*k + j). They are
+    sorted stably by expert, so inside one expert the pairs keep token order.
+    Returns
+      perm    [T*k]  pair id at each sorted position,
+      counts  [E]    pairs per expert (bincount),
+      offsets [E+1]  exclusive prefix sum of counts (start of each expert's group).
+    """
+    pairs = np.asarray(idx).reshape(-1)
+    perm = np.argsort(pairs, kind="stable").astype(np.int64)
+    counts = np.bincount(pairs, minlength=n_experts).astype(np.int64)
+    offsets = np.zeros(n_experts + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    return perm, counts, offsets
+
+
+# --------------------------------------------------------------------------- experts
+
+
+def silu(z):
+    """SiLU / Swish: z * sigmoid(z) = z / (1 + exp(-z))."""
+    z = _f64(z)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def swiglu_expert(x_rows, w_gate_up_e, w_down_e):
+    """One SwiGLU expert on a block of rows.
+
+    [OLMoE-Guide] "Top-8 Softmax Routing Formulation": Expert_i(x) =
+    (Swish(x W_gate) * (x W_up)) W_down. [MoE-scratch] §2 `Experts` stores the
+    gate rows first, then the up rows, in one (2f, d) matrix, and the down
+    projection as (d, f).
+    """
+    w_gate_up_e = _f64(w_gate_up_e)
+    f = w_gate_up_e.shape[0] // 2
+    x_rows = _f64(x_rows)
+    a = x_rows @ w_gate_up_e[:f].T
+    b = x_rows @ w_gate_up_e[f:].T
+    return (silu(a) * b) @ _f64(w_down_e).T
+
+
+def experts_grouped(x, idx, w, w_gate_up, w_down):
+    """y_t = sum_j w_tj * Expert_{S_tj}(x_t), computed group by group.
+
+    [MoE-scratch] §2 `dispatch`: sort the pairs by expert, run each expert once on
+    the rows that chose it, add the weighted results back to their tokens.
+    """
+    x = _f64(x)
+    idx = np.asarray(idx)
+    w = _f64(w)
+    T, k = idx.shape
+    n_experts = w_gate_up.shape[0]
+    perm, counts, offsets = dispatch_order(idx, n_experts)
+    y = np.zeros_like(x)
+    for e in range(n_experts):
+        sel = perm[offsets[e] : offsets[e + 1]]
+        if sel.size == 0:
+            continue
+        tok = sel // k
+        out = swiglu_expert(x[tok], w_gate_up[e], w_down[e])
+        # Each token chooses an expert at most once, so `tok` has no repeats.
+        y[tok] += w.reshape(-1)[sel][:, None] * out
+    return y
+
+
+def experts_dense(x, idx, w, w_gate_up, w_down):
+    """The same layer computed the wasteful way: every expert on every token.
+
+    [MoE-scratch] §2 `dense_run`: scatter the k weights into a T x E gate that is
+    zero elsewhere, run all E experts on all tokens and sum gate * output.
+    """
+    x = _f64(x)
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    n_experts = w_gate_up.shape[0]
+    gate = np.zeros((T, n_experts))
+    gate[np.arange(T)[:, None], idx] = _f64(w)
+    y = np.zeros_like(x)
+    for e in range(n_experts):
+        y += gate[:, e : e + 1] * swiglu_expert(x, w_gate_up[e], w_down[e])
+    return y
+
+
+# --------------------------------------------------------------------------- layer
+
+
+def moe_forward(x, w_router, w_gate_up, w_down, k, router_bias=None):
+    """The whole layer: route, dispatch, experts, combine, and the two losses.
+
+    Returns a dict with
+      y [T,d], idx [T,k], w [T,k], p [T,E], lse [T], h [T,E],
+      counts [E], offsets [E+1], perm [T*k], L_lb, L_z, near_tie [T] (bool).
+    """
+    n_experts = _f64(w_router).shape[0]
+    h = router_logits(x, w_router, router_bias)
+    p, lse = softmax_lse(h)
+    idx, w = topk_no_renorm(p, k)
+    y = experts_grouped(x, idx, w, w_gate_up, w_down)
+    L_lb, counts = load_balance_loss(idx, p, n_experts)
+    perm, _, offsets = dispatch_order(idx, n_experts)
+    return {
+        "y": y,
+        "idx": idx,
+        "w": w,
+        "p": p,
+        "lse": lse,
+        "h": h,
+        "counts": counts,
+        "offsets": offsets,
+        "perm": perm,
+        "L_lb": L_lb,
+        "L_z": router_z_loss(lse),
+        "near_tie": near_tie_tokens(p, k),
+    }
+
+
+def moe_objective(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias=None):
+    """The scalar whose gradient the backward returns: <dy, y> + alpha*L_lb + beta*L_z.
+
+    [OLMoE-Guide] "Router Mechanics & Loss Formulations": L = L_LM + alpha*L_balance
+    + beta*L_router_z; [OLMoE-paper] 4.1.6 and 4.1.7 fix alpha = 0.01, beta = 0.001.
+    The upstream gradient dy stands in for dL_LM/dy.
+    """
+    out = moe_forward(x, w_router, w_gate_up, w_down, k, router_bias)
+    return float(np.sum(_f64(dy) * out["y"])) + alpha * out["L_lb"] + beta * out["L_z"]
+
+
+def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias=None,
+                 experts=None):
+    """Gradients of moe_objective with respect to x and the three weights.
+
+    Chain rule through each step of moe_forward (f and the choice carry none):
+      expert rows   o_tj = W_down,e g_tj,  g = silu(a) * b,  [a; b] = W_gate_up,e x_t
+      combine       dw_tj = <dy_t, o_tj>,  do_tj = w_tj dy_t
+      down          dW_down,e = sum_rows do g^T,   dg = W_down,e^T do
+      SwiGLU        da = dg * b * silu'(a),  db = dg * silu(a)
+      gate/up       dW_gate_up,e = sum_rows [da; db] x^T,  dx_t += W_gate_up,e^T [da; db]
+      softmax       dp_ti = sum_j [S_tj = i] dw_tj + alpha * E * f_i / T
+                    dh_t  = p_t * (dp_t - <dp_t, p_t>) + beta * (2 lse_t / T) * p_t
+      router        dW_r = sum_t dh_t x_t^T,   dx_t += W_r^T dh_t
+    `experts` optionally restricts which experts' weight gradients are formed
+    (the rest are left zero); dx and dW_r always use every expert.
+    Returns dict dx [T,d], dw_router [E,d], dw_gate_up [E,2f,d], dw_down [E,d,f],
+    plus the forward dict under "fwd" and dw [T,k].
+    """
+    x = _f64(x)
+    dy = _f64(dy)
+    fwd = moe_forward(x, w_router, w_gate_up, w_down, k, router_bias)
+    idx, w, p, lse = fwd["idx"], fwd["w"], fwd["p"], fwd["lse"]
+    T, d = x.shape
+    n_experts = _f64(w_router).shape[0]
+    f = _f64(w_down[0]).shape[1]
+    want = set(range(n_experts)) if experts is None else set(int(e) for e in experts)
+
+    dx = np.zeros_like(x)
+    dw = np.zeros((T, k))
+    dw_gate_up = np.zeros((n_experts, 2 * f, d))
+    dw_down = np.zeros((n_experts, d, f))
+    perm, counts, offsets = dispatch_order(idx, n_experts)
+    for e in range(n_experts):
+        sel = perm[offsets[e] : offsets[e + 1]]
+        if sel.size == 0:
+            continue
+        tok = sel // k
+        wgu = _f64(w_gate_up[e])
+        wd = _f64(w_down[e])
+        xr = x[tok]
+        a = xr @ wgu[:f].T
+        b = xr @ wgu[f:].T
+        with np.errstate(over="ignore"):
+            sig = 1.0 / (1.0 + np.exp(-a))
+        g = a * sig * b
+        o = g @ wd.T
+        dw.reshape(-1)[sel] = np.sum(dy[tok] * o, axis=1)
+        do = w.reshape(-1)[sel][:, None] * dy[tok]
+        dg = do @ wd
+        da = dg * b * (sig * (1.0 + a * (1.0 - sig)))
+        db = dg * (a * sig)
+        if e in want:
+            dw_down[e] = do.T @ g
+            dw_gate_up[e, :f] = da.T @ xr
+            dw_gate_up[e, f:] = db.T @ xr
+        dx[tok] += da @ wgu[:f] + db @ wgu[f:]
+
+    dp = np.zeros((T, n_experts))
+    np.add.at(dp, (np.arange(T)[:, None].repeat(k, axis=1), idx), dw)
+    frac = counts / float(T * k)
+    dp += alpha * n_experts * frac[None, :] / T
+    dh = p * (dp - np.sum(dp * p, axis=1, keepdims=True))
+    dh += beta * (2.0 * lse / T)[:, None] * p
+    w_r = _f64(w_router)
+    dx += dh @ w_r
+    return {
+        "dx": dx,
+        "dw_router": dh.T @ x,
+        "dw_gate_up": dw_gate_up,
+        "dw_down": dw_down,
+        "dw": dw,
+        "dh": dh,
+        "fwd": fwd,
+    }
+
+
+# --------------------------------------------------------------------------- stack
+
+
+def rms_norm(x, weight=None, eps=1e-5):
+    """RMSNorm: x / sqrt(mean(x^2) + eps) * weight.
+
+    [MoE-scratch] §3 `RMSNorm` (eps 1e-5, the library default noted beside the
+    config; weight initialised to one).
+    """
+    x = _f64(x)
+    y = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return y if weight is None else y * _f64(weight)
+
+
+def stack_forward(x0, layers, k, eps=1e-5, round_input=None):
+    """A stack of MoE blocks with a residual stream: r <- r + MoE_l(RMSNorm(r)).
+
+    [MoE-scratch] §3 `Block.forward`: pre-norm, and the residual stream is kept in
+    32-bit floats between layers. `layers` is a list of dicts with keys
+    w_router, w_gate_up, w_down and optionally router_bias. `round_input`, if
+    given, is applied to the normalised activations before each layer (the
+    GPU feeds the experts bf16 activations, so the oracle can be handed the
+    same rounding). Returns the final residual [T, d] and the per-layer
+    forward dicts.
+    """
+    r = _f64(x0).copy()
+    outs = []
+    for L in layers:
+        xn = rms_norm(r, eps=eps)
+        if round_input is not None:
+            xn = _f64(round_input(xn))
+        out = moe_forward(xn, L["w_router"], L["w_gate_up"], L["w_down"], k,
+                          L.get("router_bias"))
+        r = r + out["y"]
+        outs.append(out)
+    return r, outs
