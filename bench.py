@@ -1,0 +1,420 @@
+#!/usr/bin/env python3
+"""Throughput of the OLMoE-shape MoE layer forward on B200.
+
+Workload: one MoE layer with OLMoE's shapes, T=4096 tokens (one 4096-token
+context), d_model 2048, 64 experts, top-8, SwiGLU width 1024, bf16 activations
+and weights with fp32 accumulation; seeded synthetic inputs (unit-RMS token
+rows, N(0, 0.02^2) weights). A step is one moe_forward: router, dispatch,
+gate/up grouped GEMM with SwiGLU, down grouped GEMM, combine, and both losses.
+Weights and tokens are resident in HBM; the 805 MB of expert weights read by
+every step exceed the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+N > 1 runs as torchrun, one process per GPU, each on its own batch (weak
+scaling, no data-path collective); the device time is the max over ranks and
+`value` counts the tokens of all ranks. `--impl reference` times the fp64 CPU
+oracle on the host cores on a bounded sample of the same workload.
+Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and TFLOP/s (fwd, fwd+bwd) as % of bf16/HBM roofline on 1 B200"
+UNIT = "tokens/s"
+WORKLOAD = "OLMoE MoE layer forward, T=4096 (1x4096 context), d_model=2048, E=64, top-8, d_ff=1024, bf16"
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 6  # router, dispatch rank, dispatch permute, gate/up GEMM, down GEMM, combine
+
+
+# ----------------------------------------------------------------------------- shapes
+
+
+def layer_flops_per_token(d, E, k, f):
+    """Router 2dE plus k experts of (gate/up 4df + down 2fd)."""
+    return 2 * d * E + k * (4 * d * f + 2 * f * d)
+
+
+def gate_up_flops(T, d, k, f):
+    return 2.0 * T * k * d * (2 * f)
+
+
+def layer_bytes(T, d, E, k, f, esize=2):
+    """Algorithmic bytes of one forward: every expert's weights once (all are
+    touched at this T), router weight, tokens in, output out, top-k out."""
+    return E * 3 * d * f * esize + E * d * esize + 2 * T * d * esize + T * k * 8
+
+
+# ----------------------------------------------------------------------------- ranks
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None:
+            dist.barrier(device_ids=[device])
+        else:
+            dist.barrier()
+
+
+def reduce_max(dist, value, device="cpu"):
+    """Max of a float over ranks (the measurement itself is per rank)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def finish_line(rank, line):
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        "gpu_idle": "nvmlClocksEventReasonGpuIdle",
+        "applications_clocks_setting": "nvmlClocksEventReasonApplicationsClocksSetting",
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "sync_boost": "nvmlClocksEventReasonSyncBoost",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+    }
+
+    def __init__(self, device_index, period_s=0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # no NVML: report that, do not guess
+            self.nv = None
+            self.error = str(exc)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, attr in self.REASONS.items():
+                    if mask & getattr(nv, attr, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        return {
+            "sm_mhz": statistics.median(self.samples) if self.samples else None,
+            "sm_max_mhz": self.max_mhz,
+            "reasons": sorted(self.reasons - {"gpu_idle"}),
+            "samples": len(self.samples),
+        }
+
+
+# ----------------------------------------------------------------------------- peaks
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return {k: p[k] for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def committed_traffic(kernel_file, key):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, valid only
+    while the kernel source is unchanged (sha256 recorded beside it)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "sparse_moe_transformer_route_b200", "csrc", kernel_file)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh).get(key)
+    if not rec:
+        return None
+    with open(src, "rb") as fh:
+        digest = hashlib.sha256(fh.read()).hexdigest()
+    return rec.get("bytes_per_launch") if rec.get("source_sha256") == digest else None
+
+
+# ----------------------------------------------------------------------------- oracle leg
+
+
+def oracle_sample(n_tokens_max, budget_s, steps=None, seed=1):
+    """Time the fp64 CPU oracle on contiguous token samples of the workload.
+
+    Returns (tokens/s, tokens per sample, seconds per sample list, threads)."""
+    import numpy as np
+    import torch
+    from oracle import moe_oracle as O
+    from sparse_moe_transformer_route_b200 import synthetic as S
+
+    inp = S.layer_inputs(S.PREFILL_4096, seed=seed)
+    k = inp.shape.top_k
+    x = inp.x.to(torch.float64).numpy()
+    wr = inp.w_router.to(torch.float64).numpy()
+    wgu = inp.w_gate_up.to(torch.float64).numpy()
+    wd = inp.w_down.to(torch.float64).numpy()
+
+    def one(t0, n):
+        xs = x[t0:t0 + n]
+        s = time.perf_counter()
+        O.moe_forward(xs, wr, wgu, wd, k)
+        return time.perf_counter() - s
+
+    probe = 16
+    one(0, probe)  # warm the BLAS threads
+    per_tok = one(probe, probe) / probe
+    n = int(max(probe, min(n_tokens_max, budget_s / max(per_tok, 1e-9))))
+    times = []
+    reps = steps if steps is not None else 1
+    for i in range(reps):
+        t0 = (i * n) % max(1, x.shape[0] - n + 1)
+        times.append(one(t0, n))
+    threads = 0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 0) for i in threadpool_info()), default=0)
+    except Exception:
+        pass
+    threads = threads or (os.cpu_count() or 1)
+    return n / statistics.mean(times), n, times, threads
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return 0
+    per_step_budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+    v, n, times, threads = oracle_sample(4096, per_step_budget, steps=args.steps + args.warmup)
+    timed = times[args.warmup:] or times
+    value = n / statistics.mean(timed)
+    sample = f"{n} contiguous tokens of the T=4096 workload per step (routing, experts, losses), fp64"
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(timed) * 4096 / n,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "T": 4096, "sample_tokens": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    finish_line(rank, line)
+    return 0
+
+
+# ----------------------------------------------------------------------------- B200 leg
+
+
+def run_b200(args, rank, world, local):
+    import torch
+    import sparse_moe_transformer_route_b200 as M
+    from sparse_moe_transformer_route_b200 import synthetic as S
+
+    torch.cuda.set_device(local)
+    dist = init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    sh = S.LayerShape(T=args.tokens)
+    T, d, E, k, f = sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff
+    inp = S.layer_inputs(sh, seed=1 + rank)
+    x = inp.x.to(dev)
+    wr, wgu, wd = inp.w_router.to(dev), inp.w_gate_up.to(dev), inp.w_down.to(dev)
+    cfg = M.config(T, d, E, k, f)
+    ws = M.workspace(cfg, False, dev)
+    y = torch.empty_like(x)
+    losses = torch.empty(2, device=dev)
+
+    def step():
+        M.moe_forward(cfg, x, wr, None, wgu, wd, y, losses, None, None, False, ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    status = M.moe_get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device check failed during warm-up: 0x{status:x}")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(M.binding.STAGE_EVENTS)] for _ in range(K)]
+    for row in ev:
+        for e in row:
+            e.record()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    barrier(dist, local)
+    torch.cuda.synchronize()
+    sampler.start()
+    start.record()
+    for i in range(K):
+        M.moe_set_stage_events(ev[i])
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(dist, local)
+    ms = start.elapsed_time(end) / K
+    stage_ms = {}
+    for s, name in enumerate(M.binding.STAGES):
+        stage_ms[name] = statistics.mean(ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(K))
+    ms_max = reduce_max(dist, ms, dev)
+    gate_up_ms = reduce_max(dist, stage_ms["gate_up"], dev)
+    status = M.moe_get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device check failed in the timed region: 0x{status:x}")
+
+    # end to end through the host-buffer entry point: H2D of x, the layer, D2H of y and losses
+    xh = inp.x.clone().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    lh = torch.empty(2).pin_memory()
+    for _ in range(2):
+        M.moe_forward_host(cfg, xh, wr, None, wgu, wd, yh, lh, ws)
+    barrier(dist, local)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        M.moe_forward_host(cfg, xh, wr, None, wgu, wd, yh, lh, ws)
+    e2e_s = (time.perf_counter() - t0) / K
+    e2e_s = reduce_max(dist, e2e_s, dev)
+
+    peaks, peak_src = measured_peaks()
+    timed_region_s = ms * K / 1000.0
+    burst = timed_region_s < 1.0
+    peak_tf = peaks["bf16_tflops"] if burst else peaks["bf16_tflops_sustained"]
+    gu_flops = gate_up_flops(T, d, k, f)
+    achieved = gu_flops / (gate_up_ms * 1e-3) / 1e12
+    layer_flops = layer_flops_per_token(d, E, k, f) * T
+    layer_tflops = layer_flops / (ms_max * 1e-3) / 1e12
+    lbytes = layer_bytes(T, d, E, k, f)
+    floor_ms_nominal = max(layer_flops / (NOMINAL_BF16_TFLOPS * 1e12), lbytes / (NOMINAL_HBM_GBS * 1e9)) * 1e3
+    floor_ms_measured = max(layer_flops / (peak_tf * 1e12), lbytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+
+    line = {
+        "metric": METRIC,
+        "value": world * T / (ms_max * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD if T == 4096 else WORKLOAD.replace("T=4096 (1x4096 context)", f"T={T}"),
+            "T": T, "d_model": d, "n_experts": E, "top_k": k, "d_ff": f,
+            "global_batch_tokens": world * T, "parallelism": f"replicas{world}",
+            "l2": "no flush: each step reads 805 MB of expert weights, above the 126 MB L2",
+        },
+        "tflops": layer_tflops,
+        "layer_roofline": {
+            "floor_ms_nominal": floor_ms_nominal, "frac_nominal": floor_ms_nominal / ms_max,
+            "floor_ms_measured": floor_ms_measured, "frac_measured": floor_ms_measured / ms_max,
+        },
+        "stage_ms": stage_ms,
+        "roofline": {
+            "kernel": "grouped GEMM gate/up + SwiGLU (tcgen05)",
+            "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+            "frac": achieved / peak_tf, "traffic": committed_traffic("grouped_gemm.cu", "gate_up_T4096"),
+            "peak_source": f"{peak_src} bf16_tflops{'' if burst else '_sustained'}",
+        },
+        "e2e": {
+            "value": world * T / e2e_s, "unit": UNIT,
+            "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2 + 8,
+        },
+        "gpu_launches": KERNELS_PER_STEP * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, times, threads = oracle_sample(4096, args.cpu_budget / 2, steps=2)
+        line["cpu_baseline"] = {
+            "value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} contiguous tokens of the same workload, fp64 numpy, 2 repeats",
+        }
+    finish_line(rank, line)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("b200", "reference"), default="b200")
+    ap.add_argument("--tokens", type=int, default=4096,
+                    help="tokens per layer call (4096 is the benchmarked workload; others are for profiling)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_b200(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

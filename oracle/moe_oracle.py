@@ -51,6 +51,9 @@ __all__ = [
     "router_z_loss",
     "dispatch_order",
     "silu",
+    "gate_up_preact",
+    "swiglu_hidden",
+    "expert_down",
     "swiglu_expert",
     "experts_grouped",
     "experts_dense",
@@ -181,6 +184,33 @@ def silu(z):
         return z / (1.0 + np.exp(-z))
 
 
+def gate_up_preact(x_rows, w_gate_up_e):
+    """The two pre-activations (x W_gate^T, x W_up^T) of one expert, each [n, f]."""
+    w_gate_up_e = _f64(w_gate_up_e)
+    f = w_gate_up_e.shape[0] // 2
+    x_rows = _f64(x_rows)
+    return x_rows @ w_gate_up_e[:f].T, x_rows @ w_gate_up_e[f:].T
+
+
+def swiglu_hidden(x_rows, w_gate_up_e):
+    """The expert's hidden activation Swish(x W_gate) * (x W_up), rows [n, f].
+
+    [MoE-scratch] §2 `Experts.run`: the (2f, d) gate_up matrix holds the gate
+    rows first, then the up rows; the product is split in two halves.
+    """
+    w_gate_up_e = _f64(w_gate_up_e)
+    f = w_gate_up_e.shape[0] // 2
+    x_rows = _f64(x_rows)
+    a = x_rows @ w_gate_up_e[:f].T
+    b = x_rows @ w_gate_up_e[f:].T
+    return silu(a) * b
+
+
+def expert_down(g_rows, w_down_e):
+    """The expert's down projection g W_down^T with W_down of shape (d, f)."""
+    return _f64(g_rows) @ _f64(w_down_e).T
+
+
 def swiglu_expert(x_rows, w_gate_up_e, w_down_e):
     """One SwiGLU expert on a block of rows.
 
@@ -189,12 +219,7 @@ def swiglu_expert(x_rows, w_gate_up_e, w_down_e):
     gate rows first, then the up rows, in one (2f, d) matrix, and the down
     projection as (d, f).
     """
-    w_gate_up_e = _f64(w_gate_up_e)
-    f = w_gate_up_e.shape[0] // 2
-    x_rows = _f64(x_rows)
-    a = x_rows @ w_gate_up_e[:f].T
-    b = x_rows @ w_gate_up_e[f:].T
-    return (silu(a) * b) @ _f64(w_down_e).T
+    return expert_down(swiglu_hidden(x_rows, w_gate_up_e), w_down_e)
 
 
 def experts_grouped(x, idx, w, w_gate_up, w_down):

@@ -1,0 +1,291 @@
+// Backward pieces outside the expert GEMMs, for the objective
+// <dy, y> + alpha * L_lb + beta * L_z ("OLMoE Guide", "Router Mechanics & Loss
+// Formulations"; "OLMoE: Open Mixture-of-Experts Language Models", 4.1.6 and
+// 4.1.7 for alpha and beta). No gradient flows through the choice of experts or
+// through the counts f_i (a bincount).
+//
+//   combine backward  dw_tj = <dy_t, o_tj>;  dO[r] = w_tj dy_t for the row r of
+//                     pair (t, j), zero on padding rows.       (row-parallel gather)
+//   router backward   dp_ti = sum_j [S_tj = i] dw_tj + alpha E f_i / T
+//                     dh_t  = p_t * (dp_t - <dp_t, p_t>) + beta (2 lse_t / T) p_t
+//   dx                dx_t = sum_j dX_perm[row(t, j)] + sum_e dh_t,e W_r[e]
+//   router weights    dW_r[e] = sum_t dh_t,e x_t   (split over tokens, then a
+//                     fixed-order reduction of the partials)
+// Every reduction runs in a fixed order, so the gradients are deterministic.
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+template <typename T_>
+__device__ __forceinline__ void load8(const T_* p, float (&v)[8]) {
+  if constexpr (sizeof(T_) == 4) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0];
+    const float4 b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 q = reinterpret_cast<const uint4*>(p)[0];
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      v[2 * j] = f.x;
+      v[2 * j + 1] = f.y;
+    }
+  }
+}
+
+template <typename T_>
+__device__ __forceinline__ void store8(T_* p, const float (&v)[8]) {
+  if constexpr (sizeof(T_) == 4) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint4 q;
+    q.x = pack_bf16x2(v[0], v[1]);
+    q.y = pack_bf16x2(v[2], v[3]);
+    q.z = pack_bf16x2(v[4], v[5]);
+    q.w = pack_bf16x2(v[6], v[7]);
+    reinterpret_cast<uint4*>(p)[0] = q;
+  }
+}
+
+// One warp per padded row.
+template <typename T_>
+__global__ void __launch_bounds__(256)
+    combine_bwd_kernel(const T_* __restrict__ dy, const T_* __restrict__ o_perm, const int32_t* __restrict__ row_pair,
+                       const int32_t* __restrict__ gs, int E, const float* __restrict__ wts, int d, int k,
+                       float* __restrict__ dw, T_* __restrict__ dout) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+  if (r >= gs[E]) return;
+  const int pair = row_pair[r];
+  const int nv = d / 8;
+  T_* orow = dout + r * d;
+  if (pair < 0) {
+    const float z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int v = lane; v < nv; v += 32) store8<T_>(orow + v * 8, z);
+    return;
+  }
+  const int64_t t = pair / k;
+  const float w = wts[pair];
+  float dot = 0.f;
+  for (int v = lane; v < nv; v += 32) {
+    float g[8], o[8], out[8];
+    load8<T_>(dy + t * d + v * 8, g);
+    load8<T_>(o_perm + r * d + v * 8, o);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      dot = fmaf(g[i], o[i], dot);
+      out[i] = w * g[i];
+    }
+    store8<T_>(orow + v * 8, out);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  if (lane == 0) dw[pair] = dot;
+}
+
+// One warp per token.
+__global__ void __launch_bounds__(256)
+    router_bwd_kernel(const float* __restrict__ dw, const int32_t* __restrict__ idx, const float* __restrict__ probs,
+                      const float* __restrict__ lse, const int32_t* __restrict__ counts, int64_t T, int E, int k,
+                      float alpha, float beta, float* __restrict__ dh) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+  if (t >= T) return;
+  constexpr int Q = kMaxExperts / 32;
+  const float Tf = static_cast<float>(T);
+  float dp[Q], p[Q];
+  float dot = 0.f;
+#pragma unroll
+  for (int q = 0; q < Q; ++q) {
+    const int e = lane + 32 * q;
+    dp[q] = 0.f;
+    p[q] = 0.f;
+    if (e < E) {
+      p[q] = probs[t * E + e];
+      float g = alpha * static_cast<float>(E) * (static_cast<float>(counts[e]) / (Tf * k)) / Tf;
+      for (int j = 0; j < k; ++j)
+        if (idx[t * k + j] == e) g += dw[t * k + j];
+      dp[q] = g;
+      dot = fmaf(g, p[q], dot);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  const float zterm = beta * 2.0f * lse[t] / Tf;
+#pragma unroll
+  for (int q = 0; q < Q; ++q) {
+    const int e = lane + 32 * q;
+    if (e < E) dh[t * E + e] = p[q] * (dp[q] - dot) + zterm * p[q];
+  }
+}
+
+constexpr int kDxTok = 16;
+
+// dx for 16 tokens per CTA: the k expert rows plus the router term dh W_r.
+template <typename T_>
+__global__ void __launch_bounds__(256)
+    dx_kernel(const T_* __restrict__ dx_perm, const int32_t* __restrict__ inv_perm, const float* __restrict__ dh,
+              const T_* __restrict__ w_router, int64_t T, int d, int E, int k, T_* __restrict__ dx) {
+  __shared__ float sdh[kDxTok * kMaxExperts];
+  __shared__ int32_t srow[kDxTok * kMaxTopK];
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kDxTok;
+  const int nt = static_cast<int>((T - t0) < kDxTok ? (T - t0) : kDxTok);
+  for (int i = threadIdx.x; i < nt * E; i += blockDim.x) sdh[i] = dh[t0 * E + i];
+  for (int i = threadIdx.x; i < nt * k; i += blockDim.x) srow[i] = inv_perm[t0 * k + i];
+  __syncthreads();
+  const int nv = d / 8;
+  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+    float acc[kDxTok][8];
+#pragma unroll
+    for (int t = 0; t < kDxTok; ++t)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[t][i] = 0.f;
+    for (int e = 0; e < E; ++e) {
+      float wr[8];
+      load8<T_>(w_router + static_cast<int64_t>(e) * d + v * 8, wr);
+#pragma unroll
+      for (int t = 0; t < kDxTok; ++t) {
+        const float g = (t < nt) ? sdh[t * E + e] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[t][i] = fmaf(g, wr[i], acc[t][i]);
+      }
+    }
+    for (int t = 0; t < nt; ++t) {
+      float out[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[i] = 0.f;
+      for (int j = 0; j < k; ++j) {
+        const int r = srow[t * k + j];
+        if (r < 0) continue;
+        float g[8];
+        load8<T_>(dx_perm + static_cast<int64_t>(r) * d + v * 8, g);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) out[i] += g[i];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[i] += acc[t][i];
+      store8<T_>(dx + (t0 + t) * d + v * 8, out);
+    }
+  }
+}
+
+constexpr int kWrSplit = 32;  // token splits for the router weight gradient
+
+// Partial dW_r over a token range: thread = (8 columns, 8 experts).
+template <typename T_>
+__global__ void __launch_bounds__(256)
+    router_wgrad_partial(const float* __restrict__ dh, const T_* __restrict__ x, int64_t T, int d, int E,
+                         float* __restrict__ part) {
+  const int colblk = blockIdx.x;  // 256 columns
+  const int split = blockIdx.y;
+  const int v = threadIdx.x & 31;   // column vector within the block
+  const int eg = blockIdx.z * 8 + (threadIdx.x >> 5);  // expert group of 8
+  const int col = colblk * 256 + v * 8;
+  const int64_t per = (T + kWrSplit - 1) / kWrSplit;
+  const int64_t ta = split * per;
+  const int64_t tb = (ta + per) < T ? (ta + per) : T;
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+  const bool active = (col < d) && (eg * 8 < E);
+  if (active) {
+    for (int64_t t = ta; t < tb; ++t) {
+      float xv[8];
+      load8<T_>(x + t * d + col, xv);
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        const int e = eg * 8 + a;
+        const float g = (e < E) ? dh[t * E + e] : 0.f;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(g, xv[b], acc[a][b]);
+      }
+    }
+    for (int a = 0; a < 8; ++a) {
+      const int e = eg * 8 + a;
+      if (e >= E) break;
+      float* dst = part + (static_cast<int64_t>(split) * E + e) * d + col;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) dst[b] = acc[a][b];
+    }
+  }
+}
+
+template <typename T_>
+__global__ void router_wgrad_reduce(const float* __restrict__ part, int64_t n, T_* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float s = 0.f;
+  for (int sp = 0; sp < kWrSplit; ++sp) s += part[sp * n + i];
+  out[i] = from_f32<T_>(s);
+}
+
+}  // namespace
+
+size_t router_wgrad_partial_bytes(const Shape& s) {
+  return static_cast<size_t>(kWrSplit) * s.E * s.d * sizeof(float);
+}
+
+cudaError_t launch_combine_backward(const Shape& s, const void* dy, const void* o_perm, const int32_t* gs,
+                                    const int32_t* row_pair, const float* wts, float* dw, void* dout,
+                                    cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((s.P + 7) / 8);
+  if (s.fp32)
+    combine_bwd_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(dy), static_cast<const float*>(o_perm),
+                                                    row_pair, gs, s.E, wts, s.d, s.k, dw, static_cast<float*>(dout));
+  else
+    combine_bwd_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(o_perm), row_pair, gs, s.E, wts, s.d,
+        s.k, dw, static_cast<__nv_bfloat16*>(dout));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_backward(const Shape& s, const float* dw, const int32_t* idx, const float* probs,
+                                   const float* lse, const int32_t* counts, float alpha, float beta, float* dh,
+                                   cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((s.T + 7) / 8);
+  router_bwd_kernel<<<grid, 256, 0, st>>>(dw, idx, probs, lse, counts, s.T, s.E, s.k, alpha, beta, dh);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dx_combine(const Shape& s, const void* dx_perm, const int32_t* inv_perm, const float* dh,
+                              const void* w_router, void* dx, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((s.T + kDxTok - 1) / kDxTok);
+  const int threads = s.d / 8 < 256 ? s.d / 8 : 256;
+  if (s.fp32)
+    dx_kernel<float><<<grid, threads, 0, st>>>(static_cast<const float*>(dx_perm), inv_perm, dh,
+                                               static_cast<const float*>(w_router), s.T, s.d, s.E, s.k,
+                                               static_cast<float*>(dx));
+  else
+    dx_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(static_cast<const __nv_bfloat16*>(dx_perm), inv_perm, dh,
+                                                       static_cast<const __nv_bfloat16*>(w_router), s.T, s.d, s.E, s.k,
+                                                       static_cast<__nv_bfloat16*>(dx));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_weight_grad(const Shape& s, const float* dh, const void* x, void* dw_router, float* part,
+                                      cudaStream_t st) {
+  dim3 grid((s.d + 255) / 256, kWrSplit, (s.E + 63) / 64);
+  if (s.fp32)
+    router_wgrad_partial<float><<<grid, 256, 0, st>>>(dh, static_cast<const float*>(x), s.T, s.d, s.E, part);
+  else
+    router_wgrad_partial<__nv_bfloat16><<<grid, 256, 0, st>>>(dh, static_cast<const __nv_bfloat16*>(x), s.T, s.d,
+                                                              s.E, part);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t n = static_cast<int64_t>(s.E) * s.d;
+  const unsigned g2 = static_cast<unsigned>((n + 255) / 256);
+  if (s.fp32)
+    router_wgrad_reduce<float><<<g2, 256, 0, st>>>(part, n, static_cast<float*>(dw_router));
+  else
+    router_wgrad_reduce<__nv_bfloat16><<<g2, 256, 0, st>>>(part, n, static_cast<__nv_bfloat16*>(dw_router));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,159 @@
+// Combine and RMSNorm.
+//
+// Combine ("OLMoE Guide", "Top-8 Softmax Routing Formulation": y = sum_i P_i
+// Expert_i(x); "Mixture-of-experts LLMs from scratch with OLMoE", section 2,
+// `dispatch` adds each expert's weighted rows back to their tokens): a gather,
+// not a scatter. Token t reads its k expert rows through inv_perm and sums
+// w_tj * o_tj in fp32 in slot order j = 0..k-1, then rounds once, so the result
+// is deterministic (no atomics). The residual variant adds the fp32 sum into
+// an fp32 residual stream instead (section 3, Block: x + mlp(norm(x)).float()).
+//
+// RMSNorm (section 3, RMSNorm, eps 1e-5): y = r / sqrt(mean(r^2) + eps) * w on
+// the fp32 residual, written in the layer's input dtype. The mean of squares is
+// reduced in a fixed order.
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+template <typename T_>
+struct Vec8 {
+  float v[8];
+  __device__ __forceinline__ void load(const T_* p) {
+    if constexpr (sizeof(T_) == 4) {
+      const float4 a = reinterpret_cast<const float4*>(p)[0];
+      const float4 b = reinterpret_cast<const float4*>(p)[1];
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+      const uint4 q = reinterpret_cast<const uint4*>(p)[0];
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+        v[2 * j] = f.x;
+        v[2 * j + 1] = f.y;
+      }
+    }
+  }
+  __device__ __forceinline__ void store(T_* p) const {
+    if constexpr (sizeof(T_) == 4) {
+      reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+      uint4 q;
+      q.x = pack_bf16x2(v[0], v[1]);
+      q.y = pack_bf16x2(v[2], v[3]);
+      q.z = pack_bf16x2(v[4], v[5]);
+      q.w = pack_bf16x2(v[6], v[7]);
+      reinterpret_cast<uint4*>(p)[0] = q;
+    }
+  }
+};
+
+template <typename T_, bool RESID>
+__global__ void __launch_bounds__(256)
+    combine_kernel(const T_* __restrict__ o_perm, const int32_t* __restrict__ inv_perm, const float* __restrict__ wts,
+                   int64_t T, int d, int k, T_* __restrict__ y, float* __restrict__ resid) {
+  __shared__ int32_t rows[kMaxTopK];
+  __shared__ float ws_[kMaxTopK];
+  const int64_t t = blockIdx.x;
+  if (threadIdx.x < k) {
+    rows[threadIdx.x] = inv_perm[t * k + threadIdx.x];
+    ws_[threadIdx.x] = wts[t * k + threadIdx.x];
+  }
+  __syncthreads();
+  const int nv = d / 8;
+  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int r = rows[j];
+      if (r < 0) continue;
+      Vec8<T_> o;
+      o.load(o_perm + static_cast<int64_t>(r) * d + v * 8);
+      const float w = ws_[j];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, o.v[i], acc[i]);
+    }
+    if constexpr (RESID) {
+      float* rp = resid + t * d + v * 8;
+      float4 a = reinterpret_cast<float4*>(rp)[0];
+      float4 b = reinterpret_cast<float4*>(rp)[1];
+      a.x += acc[0]; a.y += acc[1]; a.z += acc[2]; a.w += acc[3];
+      b.x += acc[4]; b.y += acc[5]; b.z += acc[6]; b.w += acc[7];
+      reinterpret_cast<float4*>(rp)[0] = a;
+      reinterpret_cast<float4*>(rp)[1] = b;
+    } else {
+      Vec8<T_> out;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out.v[i] = acc[i];
+      out.store(y + t * d + v * 8);
+    }
+  }
+}
+
+template <typename T_>
+__global__ void __launch_bounds__(256)
+    rmsnorm_kernel(const float* __restrict__ resid, const float* __restrict__ weight, float eps, int d,
+                   T_* __restrict__ out) {
+  __shared__ float red[8];
+  const int64_t t = blockIdx.x;
+  const float* r = resid + t * d;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) ss = fmaf(r[i], r[i], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) s += red[w];
+    red[0] = s;
+  }
+  __syncthreads();
+  const float inv = rsqrtf(red[0] / static_cast<float>(d) + eps);
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    const float v = r[i] * inv * (weight != nullptr ? weight[i] : 1.0f);
+    out[t * d + i] = from_f32<T_>(v);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Shape& s, const void* o_perm, const int32_t* inv_perm, const float* wts, void* y,
+                           float* resid, cudaStream_t st) {
+  const int threads = s.d / 8 < 256 ? s.d / 8 : 256;
+  const unsigned grid = static_cast<unsigned>(s.T);
+  if (s.fp32) {
+    if (resid != nullptr)
+      combine_kernel<float, true><<<grid, threads, 0, st>>>(static_cast<const float*>(o_perm), inv_perm, wts, s.T,
+                                                            s.d, s.k, nullptr, resid);
+    else
+      combine_kernel<float, false><<<grid, threads, 0, st>>>(static_cast<const float*>(o_perm), inv_perm, wts, s.T,
+                                                             s.d, s.k, static_cast<float*>(y), nullptr);
+  } else {
+    if (resid != nullptr)
+      combine_kernel<__nv_bfloat16, true><<<grid, threads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(o_perm), inv_perm, wts, s.T, s.d, s.k, nullptr, resid);
+    else
+      combine_kernel<__nv_bfloat16, false><<<grid, threads, 0, st>>>(static_cast<const __nv_bfloat16*>(o_perm),
+                                                                     inv_perm, wts, s.T, s.d, s.k,
+                                                                     static_cast<__nv_bfloat16*>(y), nullptr);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, float eps, void* out,
+                           cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(s.T);
+  if (s.fp32)
+    rmsnorm_kernel<float><<<grid, 256, 0, st>>>(resid, weight, eps, s.d, static_cast<float*>(out));
+  else
+    rmsnorm_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(resid, weight, eps, s.d, static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

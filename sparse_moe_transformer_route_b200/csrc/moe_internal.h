@@ -1,0 +1,99 @@
+// Internal declarations shared by the host-side entry points and the kernel
+// launchers: the workspace layout and the launcher signatures.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kRowAlign = MOE_ROW_ALIGN;  // expert groups start on multiples of this
+constexpr int kRouterTokensPerCta = 16;   // router kernel token block
+constexpr int kDispatchChunk = 256;       // tokens per dispatch ranking chunk
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 16;
+
+struct Shape {
+  int64_t T;
+  int d, E, k, f;
+  bool fp32;
+  size_t esize;  // bytes per activation / weight element
+  int64_t P;     // padded row capacity
+  int64_t router_ctas() const { return (T + kRouterTokensPerCta - 1) / kRouterTokensPerCta; }
+  int64_t chunks() const { return (T + kDispatchChunk - 1) / kDispatchChunk; }
+};
+
+// Byte offsets of every region inside the caller's workspace.
+struct Workspace {
+  // control words: [0] status, [1] router ticket, [2] dispatch ticket
+  size_t ctrl;
+  size_t counts_part, psum_part, zsum_part;  // router per-CTA partials
+  size_t counts, losses;                     // router totals
+  size_t probs, lse;                         // saved for backward: p [T,E], lse [T]
+  size_t idx, wts;                           // top-k indices and weights
+  size_t local_rank, chunk_count, chunk_base;
+  size_t offsets, group_start, perm, inv_perm, row_pair;
+  size_t x_perm, h, o_perm;
+  size_t preact;                              // [P, 2f] (training)
+  size_t dw, dh, dout, dab, dx_perm, wr_part; // backward scratch
+  size_t x_dev, y_dev;                        // staging for the host-buffer entry point
+  size_t fwd_bytes, bwd_bytes;
+};
+
+bool make_shape(const moe_config* cfg, Shape* s);
+Workspace layout(const Shape& s);
+
+template <typename T>
+inline T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// ---- launchers (each returns cudaSuccess or the launch error)
+cudaError_t launch_router(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
+                          float* wts, int32_t* counts, float* losses, void* ws, const Workspace& L,
+                          cudaStream_t st);
+cudaError_t launch_dispatch(const Shape& s, const int32_t* idx, const void* x, int32_t* offsets, int32_t* perm,
+                            int32_t* inv_perm, int32_t* group_start, void* x_perm, void* ws, const Workspace& L,
+                            cudaStream_t st);
+cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* group_start,
+                           const int32_t* offsets, const void* w_gate_up, void* h, void* preact, int32_t* status,
+                           cudaStream_t st);
+cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_start, const int32_t* offsets,
+                        const void* w_down, void* o_perm, int32_t* status, cudaStream_t st);
+cudaError_t launch_combine(const Shape& s, const void* o_perm, const int32_t* inv_perm, const float* wts,
+                           void* y, float* resid, cudaStream_t st);
+cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, float eps, void* out,
+                           cudaStream_t st);
+
+// backward pieces
+cudaError_t launch_dispatch_impl(const Shape& s, const int32_t* idx, const void* x, int32_t* offsets,
+                                 int32_t* perm, int32_t* inv_perm, int32_t* group_start, void* x_perm, void* ws,
+                                 const Workspace& L, bool zero_pads, cudaStream_t st);
+cudaError_t launch_combine_backward(const Shape& s, const void* dy, const void* o_perm, const int32_t* gs,
+                                    const int32_t* row_pair, const float* wts, float* dw, void* dout,
+                                    cudaStream_t st);
+cudaError_t launch_down_backward_data(const Shape& s, const void* dout, const int32_t* group_start,
+                                      const int32_t* offsets, const void* w_down, const void* preact, void* dab,
+                                      int32_t* status, cudaStream_t st);
+cudaError_t launch_gate_up_backward_data(const Shape& s, const void* dab, const int32_t* group_start,
+                                         const int32_t* offsets, const void* w_gate_up, void* dx_perm,
+                                         int32_t* status, cudaStream_t st);
+cudaError_t launch_weight_grads(const Shape& s, const void* dout, const void* h, const void* dab,
+                                const void* x_perm, const int32_t* group_start, void* dw_down, void* dw_gate_up,
+                                int32_t* status, cudaStream_t st);
+cudaError_t launch_router_backward(const Shape& s, const float* dw, const int32_t* idx, const float* probs,
+                                   const float* lse, const int32_t* counts, float alpha, float beta, float* dh,
+                                   cudaStream_t st);
+cudaError_t launch_dx_combine(const Shape& s, const void* dx_perm, const int32_t* inv_perm, const float* dh,
+                              const void* w_router, void* dx, cudaStream_t st);
+cudaError_t launch_router_weight_grad(const Shape& s, const float* dh, const void* x, void* dw_router,
+                                      float* part, cudaStream_t st);
+size_t router_wgrad_partial_bytes(const Shape& s);
+
+int device_sm_count();
+
+}  // namespace moe

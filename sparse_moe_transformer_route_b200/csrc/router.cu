@@ -1,0 +1,249 @@
+// Router: logits, softmax over all experts, top-k without renormalisation,
+// per-expert counts and the two router losses, in one kernel.
+//
+// "Mixture-of-experts LLMs from scratch with OLMoE", section 2 (softmax_topk:
+// softmax over all experts, then the k largest probabilities, unrenormalised —
+// OLMoE's norm_topk_prob is False, section 3) and section 3 MoE.forward (scores
+// in fp32, an optional per-expert offset before the softmax). "OLMoE Guide",
+// "Router Mechanics & Loss Formulations": f_i = count_i / (T k), P_i = mean_t p,
+// L_lb = E sum_i f_i P_i, L_z = mean_t lse_t^2.
+//
+// Each CTA takes 16 tokens. The dot products h_t,e = <x_t, W_r,e> are formed
+// from exact products of the inputs accumulated in fp64 (a warp per expert,
+// lanes strided over d, then a fixed shuffle tree), so the top-k order is the
+// order of the exact logits except for gaps below ~1e-15 relative; the
+// probabilities and the log-normaliser are then taken in fp32. Ties go to the
+// lower expert index. Per-CTA partial sums (counts, sum_t p_t,e, sum_t lse_t^2)
+// are reduced by the last CTA to finish, in CTA order, so the losses are
+// deterministic.
+#include <cfloat>
+#include <cmath>
+
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTok = kRouterTokensPerCta;
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) router_kernel(
+    const Tin* __restrict__ x, const Tin* __restrict__ w_router, const float* __restrict__ bias, int64_t T, int d,
+    int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out, float* __restrict__ probs,
+    float* __restrict__ lse_out, int32_t* __restrict__ counts_part, float* __restrict__ psum_part,
+    double* __restrict__ zsum_part, int32_t* __restrict__ counts_ws, int32_t* __restrict__ counts_user,
+    float* __restrict__ losses_ws, float* __restrict__ losses_user, int32_t* __restrict__ ticket) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  Tin* xs = reinterpret_cast<Tin*>(smem);                                            // [kTok][d]
+  double* logit = reinterpret_cast<double*>(smem + static_cast<size_t>(kTok) * d * sizeof(Tin));  // [kTok][E]
+  float* ps = reinterpret_cast<float*>(logit + kTok * E);                           // [kTok][E]
+  float* lses = ps + kTok * E;                                                       // [kTok]
+  int* cnt = reinterpret_cast<int*>(lses + kTok);                                    // [E]
+  __shared__ int s_last;
+  __shared__ double s_psum[kMaxExperts];
+
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTok;
+  const int ntok = static_cast<int>((T - t0) < kTok ? (T - t0) : kTok);
+  {
+    constexpr int kVec = 16 / sizeof(Tin);
+    const int nv = ntok * d / kVec;
+    const uint4* src = reinterpret_cast<const uint4*>(x + t0 * d);
+    uint4* dst = reinterpret_cast<uint4*>(xs);
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
+    // rows past the last token read as zero
+    for (int i = ntok * d / kVec + threadIdx.x; i < kTok * d / kVec; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+
+  // ---- logits: a warp per expert, lanes strided over d, fp64 accumulation
+  for (int e = warp; e < E; e += nwarps) {
+    double acc[kTok];
+#pragma unroll
+    for (int t = 0; t < kTok; ++t) acc[t] = 0.0;
+    const Tin* wrow = w_router + static_cast<size_t>(e) * d;
+    for (int i = lane; i < d; i += 32) {
+      const double wv = static_cast<double>(to_f32(wrow[i]));
+#pragma unroll
+      for (int t = 0; t < kTok; ++t) acc[t] = fma(wv, static_cast<double>(to_f32(xs[t * d + i])), acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < kTok; ++t) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+    }
+    if (lane == 0) {
+      const double b = (bias != nullptr) ? static_cast<double>(bias[e]) : 0.0;
+      for (int t = 0; t < ntok; ++t) logit[t * E + e] = acc[t] + b;
+    }
+  }
+  __syncthreads();
+
+  // ---- softmax (fp32) and top-k (on the fp64 logits): a warp per token
+  constexpr int Q = kMaxExperts / 32;
+  for (int t = warp; t < ntok; t += nwarps) {
+    double hv[Q];
+    float m = -FLT_MAX;
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+      const int e = lane + 32 * q;
+      hv[q] = (e < E) ? logit[t * E + e] : -static_cast<double>(INFINITY);
+      if (e < E) m = fmaxf(m, static_cast<float>(hv[q]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float ex[Q];
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+      const int e = lane + 32 * q;
+      ex[q] = (e < E) ? expf(static_cast<float>(hv[q]) - m) : 0.f;
+      s += ex[q];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    float p[Q];
+    const int64_t tg = t0 + t;
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+      const int e = lane + 32 * q;
+      p[q] = ex[q] / s;
+      if (e < E) {
+        ps[t * E + e] = p[q];
+        probs[tg * E + e] = p[q];
+      }
+    }
+    const float lse = m + logf(s);
+
+    uint32_t taken = 0;  // bit q: expert lane+32q already chosen
+    for (int j = 0; j < k; ++j) {
+      double bv = -static_cast<double>(INFINITY);
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        const int e = lane + 32 * q;
+        if (e < E && !((taken >> q) & 1u) && (hv[q] > bv || (hv[q] == bv && e < bi))) {
+          bv = hv[q];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (bi >= E) bi = -1;  // only NaN logits left: recorded as an invalid choice
+      const int qq = bi >> 5;
+      float mine = 0.f;
+#pragma unroll
+      for (int q = 0; q < Q; ++q)
+        if (q == qq) mine = p[q];
+      const float pw = __shfl_sync(0xffffffffu, mine, bi & 31);
+      if (bi >= 0 && lane == (bi & 31)) taken |= 1u << qq;
+      if (lane == 0) {
+        idx_out[tg * k + j] = bi;
+        w_out[tg * k + j] = (bi >= 0) ? pw : 0.f;
+        if (bi >= 0) atomicAdd(&cnt[bi], 1);
+      }
+    }
+    if (lane == 0) {
+      lses[t] = lse;
+      lse_out[tg] = lse;
+    }
+  }
+  __syncthreads();
+
+  // ---- per-CTA partials, fixed order
+  const int cta = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float acc = 0.f;
+    for (int t = 0; t < ntok; ++t) acc += ps[t * E + e];
+    psum_part[static_cast<size_t>(cta) * E + e] = acc;
+    counts_part[static_cast<size_t>(cta) * E + e] = cnt[e];
+  }
+  if (threadIdx.x == 0) {
+    double z = 0.0;
+    for (int t = 0; t < ntok; ++t) z += static_cast<double>(lses[t]) * lses[t];
+    zsum_part[cta] = z;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(ticket, 1) == static_cast<int>(gridDim.x) - 1);
+  __syncthreads();
+  if (!s_last) return;
+
+  // ---- the last CTA reduces the partials in CTA order
+  __threadfence();
+  const int nb = gridDim.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+    double pe = 0.0;
+    for (int b = 0; b < nb; ++b) {
+      c += __ldcg(&counts_part[static_cast<size_t>(b) * E + e]);
+      pe += static_cast<double>(__ldcg(&psum_part[static_cast<size_t>(b) * E + e]));
+    }
+    counts_ws[e] = c;
+    if (counts_user != nullptr) counts_user[e] = c;
+    cnt[e] = c;
+    s_psum[e] = pe;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double z = 0.0;
+    for (int b = 0; b < nb; ++b) z += __ldcg(&zsum_part[b]);
+    const double Td = static_cast<double>(T);
+    double lb = 0.0;
+    for (int e = 0; e < E; ++e) lb += (static_cast<double>(cnt[e]) / (Td * k)) * (s_psum[e] / Td);
+    lb *= E;
+    const float l0 = static_cast<float>(lb), l1 = static_cast<float>(z / Td);
+    losses_ws[0] = l0;
+    losses_ws[1] = l1;
+    if (losses_user != nullptr) {
+      losses_user[0] = l0;
+      losses_user[1] = l1;
+    }
+    *ticket = 0;
+  }
+}
+
+template <typename Tin>
+cudaError_t run(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx, float* wts,
+                int32_t* counts, float* losses, void* ws, const Workspace& L, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(kTok) * s.d * sizeof(Tin) + static_cast<size_t>(kTok) * s.E * 12 +
+                      kTok * 4 + s.E * 4;
+  static size_t configured = 0;
+  if (smem > 48 * 1024 && configured < smem) {
+    cudaError_t e =
+        cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  int32_t* ctrl = at<int32_t>(ws, L.ctrl);
+  cudaError_t e = cudaMemsetAsync(ctrl + 1, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return e;
+  const int grid = static_cast<int>(s.router_ctas());
+  router_kernel<Tin><<<grid, kThreads, smem, st>>>(
+      static_cast<const Tin*>(x), static_cast<const Tin*>(w_router), bias, s.T, s.d, s.E, s.k, idx, wts,
+      at<float>(ws, L.probs), at<float>(ws, L.lse), at<int32_t>(ws, L.counts_part), at<float>(ws, L.psum_part),
+      at<double>(ws, L.zsum_part), at<int32_t>(ws, L.counts), counts, at<float>(ws, L.losses), losses, ctrl + 1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_router(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
+                          float* wts, int32_t* counts, float* losses, void* ws, const Workspace& L,
+                          cudaStream_t st) {
+  if (s.fp32) return run<float>(s, x, w_router, bias, idx, wts, counts, losses, ws, L, st);
+  return run<__nv_bfloat16>(s, x, w_router, bias, idx, wts, counts, losses, ws, L, st);
+}
+
+}  // namespace moe

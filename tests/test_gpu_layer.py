@@ -1,0 +1,214 @@
+"""The whole layer through the C ABI against the oracle, on seeded inputs.
+
+Indices: bit-exact on every token that is not a near-tie (two neighbours among
+the k+1 largest probabilities closer than 1e-6 relative); near-ties are
+counted. Outputs and gradients: max-abs 2e-2 and relative L2 1e-2. Losses:
+1e-4 relative.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import sparse_moe_transformer_route_b200 as M
+from oracle import moe_oracle as O
+from sparse_moe_transformer_route_b200 import synthetic as S
+from tests._parity import (LazyF64, assert_close, assert_loss_close, f64, index_parity,
+                           padded_group_starts, require_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def run_forward(inp, train=False, bias=None):
+    x, wr, wgu, wd = (t.cuda() for t in (inp.x, inp.w_router, inp.w_gate_up, inp.w_down))
+    sh = inp.shape
+    cfg = M.config(sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff, x.dtype)
+    ws = M.workspace(cfg, train)
+    y = torch.empty_like(x)
+    losses = torch.empty(2, device="cuda")
+    idx = torch.empty(sh.T, sh.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(sh.T, sh.top_k, device="cuda")
+    b = bias.cuda() if bias is not None else None
+    M.moe_forward(cfg, x, wr, b, wgu, wd, y, losses, idx, w, train, ws)
+    torch.cuda.synchronize()
+    assert M.moe_get_device_status(ws) == 0
+    return dict(cfg=cfg, ws=ws, y=y, losses=losses, idx=idx, w=w, dev=(x, wr, wgu, wd, b))
+
+
+def check_forward(inp, out, bias=None, sample=None):
+    """Routing for every token; outputs on `sample` tokens (all when None)."""
+    x = f64(inp.x)
+    wr = f64(inp.w_router)
+    k = inp.shape.top_k
+    E = inp.shape.n_experts
+    b = f64(bias) if bias is not None else None
+    h = O.router_logits(x, wr, b)
+    p, lse = O.softmax_lse(h)
+    ref_idx, ref_w = O.topk_no_renorm(p, k)
+    near = O.near_tie_tokens(p, k)
+    gidx = out["idx"].cpu().numpy()
+    bad, n_near, diff = index_parity(gidx, ref_idx, near)
+    assert bad.size == 0, f"{bad.size} non-near-tie tokens routed differently, e.g. {bad[:5]}"
+    same = ~diff
+    assert_close(out["w"].cpu()[torch.from_numpy(same)], ref_w[same], "router weights", max_abs=1e-5, rel_l2=1e-5)
+    L_lb, _ = O.load_balance_loss(ref_idx, p, E)
+    assert_loss_close(out["losses"][0].item(), L_lb, "L_lb")
+    assert_loss_close(out["losses"][1].item(), O.router_z_loss(lse), "L_z")
+    toks = np.arange(inp.shape.T) if sample is None else np.asarray(sample)
+    toks = toks[same[toks]]
+    wgu = LazyF64(inp.w_gate_up)
+    wd = LazyF64(inp.w_down)
+    y_ref = O.experts_grouped(x[toks], ref_idx[toks], ref_w[toks], wgu, wd)
+    assert_close(out["y"].cpu()[torch.from_numpy(toks)], y_ref, "y")
+    return n_near
+
+
+def test_small_fp32_layer():
+    """T=128, d=512, E=64, k=8, f=256 in fp32, seed 0, x ~ N(0, 1)."""
+    inp = S.layer_inputs(S.SMALL_FP32, seed=0, dtype=torch.float32, normalised=False)
+    out = run_forward(inp)
+    check_forward(inp, out)
+
+
+@pytest.mark.parametrize("T,d,E,k,f", [(300, 256, 16, 4, 256), (1000, 512, 64, 8, 256), (1, 2048, 64, 8, 1024),
+                                       (77, 384, 32, 3, 128)])
+def test_bf16_layers_with_ragged_groups(T, d, E, k, f):
+    inp = S.layer_inputs(S.LayerShape(T, d, E, k, f), seed=T + d)
+    out = run_forward(inp)
+    check_forward(inp, out)
+
+
+def test_eight_experts_take_every_token():
+    """A large router offset on experts 0..7: they receive all T rows (several
+    tiles each) and the other 56 experts none."""
+    sh = S.LayerShape(600, 256, 64, 8, 256)
+    inp = S.layer_inputs(sh, seed=4)
+    bias = torch.zeros(64)
+    bias[:8] = 30.0
+    out = run_forward(inp, bias=bias)
+    assert set(np.unique(out["idx"].cpu().numpy())) == set(range(8))
+    check_forward(inp, out, bias=bias)
+
+
+def test_olmoe_prefill_4096():
+    """The OLMoE-shape layer: T=4096, d=2048, E=64, k=8, f=1024, bf16. Routing of
+    every token; outputs on a sample of tokens (the first, the last, and 46 drawn)."""
+    inp = S.layer_inputs(S.PREFILL_4096, seed=1)
+    out = run_forward(inp)
+    r = np.random.default_rng(0)
+    sample = np.unique(np.concatenate([[0, 4095], r.choice(4096, 46, replace=False)]))
+    check_forward(inp, out, sample=sample)
+
+
+def test_forward_is_deterministic_and_stages_compose():
+    sh = S.LayerShape(700, 512, 64, 8, 256)
+    inp = S.layer_inputs(sh, seed=12)
+    a = run_forward(inp)
+    b = run_forward(inp)
+    assert torch.equal(a["y"], b["y"]) and torch.equal(a["losses"], b["losses"])
+    # the stage entry points reproduce moe_forward bit for bit
+    x, wr, wgu, wd, _ = a["dev"]
+    cfg = a["cfg"]
+    T, E, k = sh.T, sh.n_experts, sh.top_k
+    P = M.moe_padded_rows(cfg)
+    ws = M.workspace(cfg)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    losses = torch.empty(2, device="cuda")
+    M.moe_route(cfg, x, wr, None, idx, w, counts, losses, ws)
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    gs = torch.empty_like(off)
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty_like(perm)
+    xp = torch.empty(P, sh.d_model, dtype=x.dtype, device="cuda")
+    M.moe_dispatch(cfg, idx, x, off, perm, inv, gs, xp, ws)
+    h = torch.empty(P, sh.d_ff, dtype=x.dtype, device="cuda")
+    op = torch.empty(P, sh.d_model, dtype=x.dtype, device="cuda")
+    M.moe_expert_ffn(cfg, xp, gs, off, wgu, wd, h, op, ws)
+    y = torch.empty_like(x)
+    M.moe_combine(cfg, op, inv, w, y)
+    torch.cuda.synchronize()
+    assert torch.equal(y, a["y"]) and torch.equal(losses, a["losses"]) and torch.equal(idx, a["idx"])
+    assert int(counts.sum()) == T * k
+    assert np.array_equal(counts.cpu().numpy(), np.bincount(idx.cpu().numpy().reshape(-1), minlength=E))
+
+
+def test_host_buffer_entry_point_matches_device():
+    sh = S.LayerShape(256, 512, 64, 8, 256)
+    inp = S.layer_inputs(sh, seed=13)
+    a = run_forward(inp)
+    x, wr, wgu, wd, _ = a["dev"]
+    cfg = a["cfg"]
+    ws = M.workspace(cfg)
+    xh = inp.x.clone().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    lh = torch.empty(2).pin_memory()
+    M.moe_forward_host(cfg, xh, wr, None, wgu, wd, yh, lh, ws)
+    assert torch.equal(yh, a["y"].cpu()) and torch.equal(lh, a["losses"].cpu())
+
+
+def check_backward(inp, alpha=0.01, beta=0.001, experts=None, tol_scale=1.0):
+    sh = inp.shape
+    x, wr, wgu, wd, dy = (t.cuda() for t in (inp.x, inp.w_router, inp.w_gate_up, inp.w_down, inp.dy))
+    cfg = M.config(sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff, x.dtype, alpha, beta)
+    ws = M.workspace(cfg, True)
+    y = torch.empty_like(x)
+    losses = torch.empty(2, device="cuda")
+    idx = torch.empty(sh.T, sh.top_k, dtype=torch.int32, device="cuda")
+    M.moe_forward(cfg, x, wr, None, wgu, wd, y, losses, idx, None, True, ws)
+    g = dict(dx=torch.empty_like(x), dw_router=torch.empty_like(wr), dw_gate_up=torch.empty_like(wgu),
+             dw_down=torch.empty_like(wd))
+    M.moe_backward(cfg, dy, x, wr, wgu, wd, g["dx"], g["dw_router"], g["dw_gate_up"], g["dw_down"], ws)
+    torch.cuda.synchronize()
+    assert M.moe_get_device_status(ws) == 0
+    ref = O.moe_backward(f64(inp.x), f64(inp.w_router), LazyF64(inp.w_gate_up), LazyF64(inp.w_down), sh.top_k,
+                         f64(inp.dy), alpha, beta, experts=experts)
+    # gradients sum over tokens, so the routing must agree on every token (near-ties
+    # included: the router decides on logits accumulated in fp64 from exact products)
+    assert np.array_equal(idx.cpu().numpy(), ref["fwd"]["idx"]), "routing differs from the oracle"
+    assert_close(g["dx"], ref["dx"], "dx")
+    assert_close(g["dw_router"], ref["dw_router"], "dW_router")
+    es = range(sh.n_experts) if experts is None else experts
+    for e in es:
+        assert_close(g["dw_gate_up"][e], ref["dw_gate_up"][e], f"dW_gate_up[{e}]")
+        assert_close(g["dw_down"][e], ref["dw_down"][e], f"dW_down[{e}]")
+    return g
+
+
+def test_backward_small_layer_bf16():
+    """The small layer's shapes (T=128, d=512, E=64, k=8, f=256) in bf16."""
+    inp = S.layer_inputs(S.SMALL_FP32, seed=0, dtype=torch.bfloat16, normalised=False, with_grad=True)
+    check_backward(inp)
+
+
+def test_backward_rejects_fp32():
+    sh = S.SMALL_FP32
+    cfg = M.config(sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff, torch.float32)
+    ws = M.workspace(cfg, True)
+    t = torch.zeros(sh.T, sh.d_model, device="cuda")
+    wr = torch.zeros(sh.n_experts, sh.d_model, device="cuda")
+    wgu = torch.zeros(sh.n_experts, 2 * sh.d_ff, sh.d_model, device="cuda")
+    wd = torch.zeros(sh.n_experts, sh.d_model, sh.d_ff, device="cuda")
+    with pytest.raises(M.MoeError) as ei:
+        M.moe_backward(cfg, t, t, wr, wgu, wd, t.clone(), wr.clone(), wgu.clone(), wd.clone(), ws)
+    assert ei.value.status == 2
+
+
+@pytest.mark.parametrize("T,d,E,k,f", [(512, 256, 16, 4, 256), (300, 384, 8, 2, 128)])
+def test_backward_bf16(T, d, E, k, f):
+    inp = S.layer_inputs(S.LayerShape(T, d, E, k, f), seed=T, with_grad=True)
+    check_backward(inp)
+
+
+def test_backward_loss_terms_alone():
+    """dy = 0: only alpha * L_lb + beta * L_z drive the router gradient."""
+    sh = S.LayerShape(256, 256, 16, 4, 128)
+    inp = S.layer_inputs(sh, seed=21, dtype=torch.bfloat16, with_grad=True)
+    inp.dy = torch.zeros_like(inp.dy)
+    check_backward(inp, alpha=0.5, beta=0.25)
