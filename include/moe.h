@@ -121,6 +121,29 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
                      int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,
                      size_t ws_bytes, cudaStream_t stream);
 
+/* moe_route without a workspace: the same router, results and output buffers,
+ * but its scratch is a fixed MOE_ROUTE_STATIC_SCRATCH_BYTES array inside the
+ * library, so the call allocates nothing and needs no `ws`. The pages have no
+ * counterpart: this is for callers that cannot provide device memory of their
+ * own, such as code whose device memory is planned and owned by a host
+ * framework or serving runtime, or a loop that must not call cudaMalloc because
+ * it synchronises the device.
+ *   - Limit: the scratch holds T * (4.5 * E + 4.5) bytes plus under 2 KB of
+ *     alignment, so at E = 64 up to 7,167 tokens (the 4,096-token OLMoE layer
+ *     fits); larger calls return MOE_ERR_WORKSPACE_TOO_SMALL before
+ *     launching anything.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (it must be the current device); make that first call before any
+ *     stream capture.
+ *   - Every device that loads the library keeps the array until the process
+ *     exits. All calls share it and find the last call's contents in it; the
+ *     part that must start at zero is cleared on `stream` before each launch.
+ *     Calls that overlap on the GPU (different streams or host threads) race on
+ *     the array and must be serialised by the caller. */
+#define MOE_ROUTE_STATIC_SCRATCH_BYTES (2u << 20)
+moe_status moe_route_static(const moe_config* cfg, const void* x, const void* w_router, const float* router_bias,
+                            int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, cudaStream_t stream);
+
 /* Dispatch: group the T*k (token, slot) pairs by expert, dropless and stable in
  * token order, and gather the token rows into expert-contiguous order
  * ("Mixture-of-experts LLMs from scratch with OLMoE", section 2, `dispatch`:

@@ -28,6 +28,7 @@ from .binding import (  # noqa: F401
     moe_padded_rows,
     moe_rmsnorm,
     moe_route,
+    moe_route_static,
     moe_set_stage_events,
     moe_stack_forward,
     moe_workspace_bytes,

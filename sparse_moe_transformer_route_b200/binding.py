@@ -34,7 +34,7 @@ STATUS_NAMES = {
 # Every symbol the header declares, in declaration order.
 EXPORTS = (
     "moe_status_string", "moe_abi_version", "moe_check_config", "moe_padded_rows",
-    "moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_dispatch",
+    "moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_route_static", "moe_dispatch",
     "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_forward",
     "moe_forward_host", "moe_backward", "moe_rmsnorm", "moe_combine_residual",
     "moe_stack_forward", "moe_set_stage_events", "moe_get_device_status",
@@ -73,6 +73,7 @@ _SIGS = {
     "moe_workspace_bytes": (ctypes.c_size_t, [_CFG, ctypes.c_int32]),
     "moe_workspace_init": (ctypes.c_int, [_P, _P]),
     "moe_route": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_route_static": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_expert_gate_up": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_expert_down": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -201,6 +202,21 @@ def moe_route(cfg, x, w_router, router_bias, topk_idx, topk_w, counts, losses, w
         _ptr(losses, torch.float32, (2,), "losses", allow_none=True),
         _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
     _check(st, "moe_route")
+
+
+def moe_route_static(cfg, x, w_router, router_bias, topk_idx, topk_w, counts, losses, stream=None):
+    """moe_route on the library's own fixed scratch: no workspace, no allocation.
+    For callers that cannot provide device memory; see include/moe.h for the
+    size limit and the sharing rules (one array per device, calls must not overlap)."""
+    dt = torch_dtype(cfg)
+    T, d, E, k = cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k
+    st = lib().moe_route_static(
+        _cfgp(cfg), _ptr(x, dt, (T, d), "x"), _ptr(w_router, dt, (E, d), "w_router"),
+        _ptr(router_bias, torch.float32, (E,), "router_bias", allow_none=True),
+        _ptr(topk_idx, torch.int32, (T, k), "topk_idx"), _ptr(topk_w, torch.float32, (T, k), "topk_w"),
+        _ptr(counts, torch.int32, (E,), "counts", allow_none=True),
+        _ptr(losses, torch.float32, (2,), "losses", allow_none=True), _stream(stream))
+    _check(st, "moe_route_static")
 
 
 def moe_dispatch(cfg, topk_idx, x, offsets, perm, inv_perm, group_start, x_perm, ws, stream=None):

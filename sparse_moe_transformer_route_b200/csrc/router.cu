@@ -247,3 +247,131 @@ cudaError_t launch_router(const Shape& s, const void* x, const void* w_router, c
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// The router on library-owned scratch: moe_route_static.
+//
+// For callers that cannot hand the library a workspace: code whose device
+// memory is owned and planned by a host framework or serving runtime (it may
+// not call cudaMalloc itself, and has no arena slot for an extra buffer), or a
+// latency-critical loop that must not allocate because cudaMalloc synchronises
+// the device. The router's scratch (per-CTA partial sums, the completion
+// counter, the saved probabilities) then lives in one file-scope device array
+// that every device loading this library holds until the process exits.
+//
+// Host code must not pass the array's name to a kernel: on the host it is only
+// a stand-in symbol, not a device address. Its device address is looked up
+// once per device, with that device current, on the first call made on that
+// device; make that first call before any stream capture. Every call uses the
+// same array and finds the previous call's contents in it: the completion
+// counter is cleared on the stream before each launch, and everything else is
+// overwritten before it is read. Calls whose executions overlap on the GPU
+// (other streams, other host threads) race on the array.
+#include <mutex>
+
+namespace moe {
+namespace {
+
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(MOE_ROUTE_STATIC_SCRATCH_BYTES);
+static __device__ __align__(256) unsigned char g_route_scratch[kStaticScratchBytes];
+
+struct StaticLayout {
+  size_t ticket, counts_part, psum_part, zsum_part, counts, losses, probs, lse, total;
+};
+
+StaticLayout static_layout(const Shape& s) {
+  StaticLayout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at_ = o;
+    o = (o + bytes + 255) / 256 * 256;
+    return at_;
+  };
+  const size_t ctas = static_cast<size_t>(s.router_ctas());
+  const size_t T = static_cast<size_t>(s.T), E = static_cast<size_t>(s.E);
+  L.ticket = take(sizeof(int32_t));
+  L.counts_part = take(ctas * E * sizeof(int32_t));
+  L.psum_part = take(ctas * E * sizeof(float));
+  L.zsum_part = take(ctas * sizeof(double));
+  L.counts = take(E * sizeof(int32_t));
+  L.losses = take(2 * sizeof(float));
+  L.probs = take(T * E * sizeof(float));
+  L.lse = take(T * sizeof(float));
+  L.total = o;
+  return L;
+}
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+unsigned char* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_route_scratch on the current device (looked up once per device).
+cudaError_t static_scratch(unsigned char** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+template <typename Tin>
+cudaError_t run_static(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
+                       float* wts, int32_t* counts, float* losses, unsigned char* scratch, const StaticLayout& L,
+                       cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(kTok) * s.d * sizeof(Tin) + static_cast<size_t>(kTok) * s.E * 12 +
+                      kTok * 4 + s.E * 4;
+  if (smem > 48 * 1024) {
+    cudaError_t e =
+        cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  int32_t* ticket = reinterpret_cast<int32_t*>(scratch + L.ticket);
+  cudaError_t e = cudaMemsetAsync(ticket, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return e;
+  const int grid = static_cast<int>(s.router_ctas());
+  router_kernel<Tin><<<grid, kThreads, smem, st>>>(
+      static_cast<const Tin*>(x), static_cast<const Tin*>(w_router), bias, s.T, s.d, s.E, s.k, idx, wts,
+      reinterpret_cast<float*>(scratch + L.probs), reinterpret_cast<float*>(scratch + L.lse),
+      reinterpret_cast<int32_t*>(scratch + L.counts_part), reinterpret_cast<float*>(scratch + L.psum_part),
+      reinterpret_cast<double*>(scratch + L.zsum_part), reinterpret_cast<int32_t*>(scratch + L.counts), counts,
+      reinterpret_cast<float*>(scratch + L.losses), losses, ticket);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_route_static(const moe_config* cfg, const void* x, const void* w_router,
+                                       const float* router_bias, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                       float* losses, cudaStream_t stream) {
+  using namespace moe;
+  if (cfg == nullptr) return MOE_ERR_INVALID_ARG;
+  Shape s;
+  if (!make_shape(cfg, &s)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (x == nullptr || w_router == nullptr || topk_idx == nullptr || topk_w == nullptr ||
+      (reinterpret_cast<uintptr_t>(x) & 15u) != 0 || (reinterpret_cast<uintptr_t>(w_router) & 15u) != 0)
+    return MOE_ERR_INVALID_ARG;
+  const StaticLayout L = static_layout(s);
+  if (L.total > kStaticScratchBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int dev = -1, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess || major != 10 ||
+      minor != 0)
+    return MOE_ERR_NO_DEVICE;
+  unsigned char* scratch = nullptr;
+  if (static_scratch(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  const cudaError_t e =
+      s.fp32 ? run_static<float>(s, x, w_router, router_bias, topk_idx, topk_w, counts, losses, scratch, L, stream)
+             : run_static<__nv_bfloat16>(s, x, w_router, router_bias, topk_idx, topk_w, counts, losses, scratch, L,
+                                         stream);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
