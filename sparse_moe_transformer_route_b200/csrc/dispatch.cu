@@ -7,8 +7,8 @@
 // t*k+j, where each token names an expert at most once, is the order by
 // (expert, token); this is what the kernels build, without a sort:
 //
-//   1. rank kernel: tokens are cut into chunks of 256. For each chunk and
-//      expert, a 256-bit mask marks the tokens that chose the expert; a pair's
+//   1. rank kernel: tokens are cut into chunks of 128. For each chunk and
+//      expert, a 128-bit mask marks the tokens that chose the expert; a pair's
 //      rank inside its chunk is a popcount of the mask below its token. The last
 //      CTA to finish scans the per-chunk counts: the base of every (chunk,
 //      expert), the unpadded offsets (the bincount prefix) and the padded group
@@ -81,9 +81,19 @@ __global__ void __launch_bounds__(kDispatchChunk)
   const int nchunks = gridDim.x;
   for (int e = tl; e < E; e += blockDim.x) {
     int run = 0;
-    for (int cc = 0; cc < nchunks; ++cc) {
-      chunk_base[static_cast<size_t>(cc) * E + e] = run;
-      run += __ldcg(&chunk_count[static_cast<size_t>(cc) * E + e]);
+    // loads in batches of 16 so their L2 round trips overlap
+    for (int c0 = 0; c0 < nchunks; c0 += 16) {
+      int cv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        cv[i] = (c0 + i < nchunks) ? __ldcg(&chunk_count[static_cast<size_t>(c0 + i) * E + e]) : 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (c0 + i < nchunks) {
+          chunk_base[static_cast<size_t>(c0 + i) * E + e] = run;
+          run += cv[i];
+        }
+      }
     }
     total[e] = run;
   }
@@ -172,6 +182,11 @@ cudaError_t launch_dispatch_impl(const Shape& s, const int32_t* idx, const void*
                                                   group_start, ctrl + 2, ctrl);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  return launch_permute(s, idx, x, perm, inv_perm, x_perm, ws, L, zero_pads, st);
+}
+
+cudaError_t launch_permute(const Shape& s, const int32_t* idx, const void* x, int32_t* perm, int32_t* inv_perm,
+                           void* x_perm, void* ws, const Workspace& L, bool zero_pads, cudaStream_t st) {
   const int grid = static_cast<int>((s.T + 7) / 8);
   const int grid2 = zero_pads ? (grid > s.E ? grid : s.E) : grid;
   if (s.fp32) {

@@ -40,7 +40,12 @@ namespace {
 enum class Group { M, K };
 enum class Epi { SwigluFwd, Store, SwigluBwd };
 
-template <bool TF32_, bool A_MN_, bool B_MN_, Group G_, Epi EP_, int BN_>
+// H = number of 128-row halves per tile. H = 2 (a 256-row tile) issues two
+// M=128 UMMAs on every B stage, so each byte of B feeds twice the MMA work:
+// 64 B per MMA cycle instead of 96, the difference between starving and not
+// on HBM-resident weights. A 256-row tile whose second half lies past its
+// expert's rows issues only the first half.
+template <bool TF32_, bool A_MN_, bool B_MN_, Group G_, Epi EP_, int BN_, int H_ = 1>
 struct Cfg {
   static constexpr bool TF32 = TF32_;
   static constexpr bool A_MN = A_MN_;
@@ -48,25 +53,39 @@ struct Cfg {
   static constexpr Group G = G_;
   static constexpr Epi EP = EP_;
   static constexpr int BN = BN_;
+  static constexpr int H = H_;
   using T = std::conditional_t<TF32, float, __nv_bfloat16>;
-  static constexpr int BM = 128;
+  static constexpr int BM = 128 * H;
   static constexpr int ESZ = TF32 ? 4 : 2;
   static constexpr int BK = 128 / ESZ;      // K per stage (one 128-byte swizzle row when K-major)
   static constexpr int UK = 32 / ESZ;       // K per UMMA instruction
-  static constexpr int KSTEPS = BK / UK;    // UMMAs per stage
+  static constexpr int KSTEPS = BK / UK;    // UMMAs per stage and half
   static constexpr int CH = 128 / ESZ;      // MN elements per 128-byte chunk when MN-major
-  static constexpr int A_BYTES = BM * BK * ESZ;
+  static constexpr int A_HALF = 128 * BK * ESZ;  // bytes of one 128-row half of A per stage
+  static constexpr int A_BYTES = H * A_HALF;
   static constexpr int B_BYTES = BN * BK * ESZ;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
-  static constexpr uint32_t IDESC = make_idesc(TF32, A_MN, B_MN, BM, BN);
-  static constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256u : 512u;
-  static constexpr int THREADS = 192;
+  static constexpr int ACC_BUFS = (2 * H * BN <= 512) ? 2 : 1;  // TMEM holds 512 fp32 columns
+  static constexpr uint32_t IDESC = make_idesc(TF32, A_MN, B_MN, 128, BN);
+  static constexpr uint32_t TMEM_COLS = (ACC_BUFS * H * BN <= 256) ? 256u : 512u;
+  // two epilogue warps per TMEM lane quarter and half, each on half of the columns
+  static constexpr int EPI_WARPS = 8 * H;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  // Each epilogue warp stages a 32 x 32 output chunk in shared memory (rows
+  // padded by 16 bytes against bank conflicts) and writes it back as whole rows.
+  static constexpr int STG_PITCH = 32 * ESZ + 16;
+  static constexpr int STG_WARP_BYTES = 32 * STG_PITCH;
+  static constexpr int STG_BYTES = EPI_WARPS * STG_WARP_BYTES;
+  static constexpr int MISC_BYTES = 1024 + 3 * (kMaxExperts + 1) * static_cast<int>(sizeof(int32_t));
+  static constexpr int STAGES = (227 * 1024 - 1024 - MISC_BYTES - STG_BYTES) / STAGE_BYTES;
   // N columns of output per tile (SwiGLU forward pairs BN/2 gate with BN/2 up columns)
   static constexpr int OUT_N = (EP == Epi::SwigluFwd) ? BN / 2 : BN;
-  static constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 1024 +
-                                       2 * (kMaxExperts + 1) * sizeof(int32_t);
+  static constexpr size_t SMEM_BYTES =
+      1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + STG_BYTES + static_cast<size_t>(MISC_BYTES);
+  static_assert(STAGES >= 2, "shared memory ring");
   static_assert(BN == 128 || BN == 256, "tile N");
+  static_assert(H == 1 || H == 2, "tile M");
+  static_assert(!(H == 2 && TF32), "256-row tiles are bf16 only");
   static_assert(!(EP == Epi::SwigluFwd && B_MN), "gate/up weights are read K-major");
 };
 
@@ -91,11 +110,12 @@ struct Args {
 
 struct Tile {
   int e;
-  int m0;     // M-grouped: first row; K-grouped: first output row inside the expert
-  int n0;     // first accumulator-mapped output column (see OUT_N)
-  int valid;  // M-grouped: valid rows in this tile (rest are padding)
-  int krow0;  // K-grouped: first row of the expert
-  int nk;     // K stages
+  int m0;      // M-grouped: first row; K-grouped: first output row inside the expert
+  int n0;      // first accumulator-mapped output column (see OUT_N)
+  int valid;   // M-grouped: valid rows in this tile (rest are padding)
+  int halves;  // 128-row halves to compute (1 or 2 for H = 2; always 1 for H = 1)
+  int krow0;   // K-grouped: first row of the expert
+  int nk;      // K stages
 };
 
 template <class C>
@@ -103,34 +123,50 @@ __device__ __forceinline__ int num_n_tiles(const Args& a) {
   return a.N_total / C::OUT_N;
 }
 
+// ts[e]: first M-tile of expert e (M-grouped); groups are multiples of 128
+// rows, so a group of R rows spans ceil(R / BM) tiles.
 template <class C>
-__device__ __forceinline__ int total_tiles(const Args& a, const int32_t* gs) {
+__device__ __forceinline__ void tile_starts(const Args& a, const int32_t* gs, int32_t* ts) {
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int e = 0; e < a.E; ++e) {
+      ts[e] = acc;
+      acc += (gs[e + 1] - gs[e] + C::BM - 1) / C::BM;
+    }
+    ts[a.E] = acc;
+  }
+}
+
+template <class C>
+__device__ __forceinline__ int total_tiles(const Args& a, const int32_t* ts) {
   if constexpr (C::G == Group::M) {
-    return (gs[a.E] / C::BM) * num_n_tiles<C>(a);
+    return ts[a.E] * num_n_tiles<C>(a);
   } else {
     return a.E * (a.M_total / C::BM) * num_n_tiles<C>(a);
   }
 }
 
 template <class C>
-__device__ __forceinline__ Tile decode_tile(const Args& a, const int32_t* gs, const int32_t* off, int L) {
+__device__ __forceinline__ Tile decode_tile(const Args& a, const int32_t* gs, const int32_t* off, const int32_t* ts,
+                                            int L) {
   Tile t;
   const int nN = num_n_tiles<C>(a);
   if constexpr (C::G == Group::M) {
     const int mt = L / nN;
     const int nt = L - mt * nN;
-    const int row0 = mt * C::BM;
-    // largest e with gs[e] <= row0 (groups are non-decreasing; empty groups are skipped)
+    // largest e with ts[e] <= mt (experts without rows own no tiles and are skipped)
     int lo = 0, hi = a.E - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (gs[mid] <= row0) lo = mid; else hi = mid - 1;
+      if (ts[mid] <= mt) lo = mid; else hi = mid - 1;
     }
+    const int row0 = gs[lo] + (mt - ts[lo]) * C::BM;
     t.e = lo;
     t.m0 = row0;
     t.n0 = nt * C::OUT_N;
     const int cnt = off[lo + 1] - off[lo];
     t.valid = min(C::BM, gs[lo] + cnt - row0);
+    t.halves = (C::H == 2 && row0 + 128 < gs[lo + 1]) ? 2 : 1;
     t.krow0 = 0;
     t.nk = a.K_total / C::BK;
   } else {
@@ -143,6 +179,7 @@ __device__ __forceinline__ Tile decode_tile(const Args& a, const int32_t* gs, co
     t.m0 = mt * C::BM;
     t.n0 = nt * C::OUT_N;
     t.valid = C::BM;
+    t.halves = C::H;
     t.krow0 = gs[t.e];
     t.nk = (gs[t.e + 1] - gs[t.e]) / C::BK;
   }
@@ -202,6 +239,44 @@ __device__ __forceinline__ void load16(const T* src, float (&v)[16]) {
   }
 }
 
+// One warp writes a 32-row x 32-column chunk whose row `lane` this thread holds
+// in v: the rows go to shared memory first, then leave as whole rows (each
+// store instruction covers several complete rows), instead of 32 scattered
+// 16-byte pieces per instruction. `g` points at (the warp's first row, the
+// chunk's first column); `ld` is the row stride in elements.
+template <typename T, int PITCH>
+__device__ __forceinline__ void warp_store_chunk(unsigned char* stg, const float (&v)[32], T* g, int64_t ld,
+                                                 int lane) {
+  constexpr int RB = 32 * static_cast<int>(sizeof(T));  // bytes of one row of the chunk
+  constexpr int LPR = RB / 16;                           // lanes per row on the way out
+  constexpr int RPI = 32 / LPR;                          // rows per store instruction
+  unsigned char* mine = stg + lane * PITCH;
+  if constexpr (std::is_same_v<T, float>) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<float4*>(mine + 16 * i) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * i], v[8 * i + 1]);
+      w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+      w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+      w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+      *reinterpret_cast<uint4*>(mine + 16 * i) = w;
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 32 / RPI; ++it) {
+    const int r = it * RPI + lane / LPR;
+    const int seg = lane % LPR;
+    const uint4 val = *reinterpret_cast<const uint4*>(stg + r * PITCH + seg * 16);
+    *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(g + r * ld) + seg * 16) = val;
+  }
+  __syncwarp();
+}
+
 // -------------------------------------------------------------- the kernel
 
 template <class C>
@@ -214,15 +289,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* stage_base = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(C::STAGES) * C::STAGE_BYTES);
+  unsigned char* stg_base = smem + static_cast<size_t>(C::STAGES) * C::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg_base + C::STG_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* acc_full = bars + 2 * C::STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  int32_t* gs = reinterpret_cast<int32_t*>(smem + static_cast<size_t>(C::STAGES) * C::STAGE_BYTES + 1024);
+  int32_t* gs = reinterpret_cast<int32_t*>(stg_base + C::STG_BYTES + 1024);
   int32_t* off = gs + (kMaxExperts + 1);
+  int32_t* ts = off + (kMaxExperts + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -231,14 +308,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     gs[i] = a.group_start[i];
     off[i] = (a.offsets != nullptr) ? a.offsets[i] : 0;
   }
+  __syncthreads();
+  if constexpr (C::G == Group::M) tile_starts<C>(a, gs, ts);
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::ACC_BUFS; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&acc_empty[b], 32 * C::EPI_WARPS);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -255,7 +334,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int n_tiles = total_tiles<C>(a, gs);
+  const int n_tiles = total_tiles<C>(a, ts);
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -265,7 +344,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       int issued = 0;
       bool ok = true;
       for (int L = blockIdx.x; L < n_tiles && ok; L += gridDim.x) {
-        const Tile t = decode_tile<C>(a, gs, off, L);
+        const Tile t = decode_tile<C>(a, gs, off, ts, L);
         for (int kb = 0; kb < t.nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u)) {
             report(a.status, DEV_WAIT_TIMEOUT_PRODUCER);
@@ -274,13 +353,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           unsigned char* sa = stage_base + static_cast<size_t>(stage) * C::STAGE_BYTES;
           unsigned char* sb = sa + C::A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          // A operand
+          mbar_arrive_expect_tx(&full[stage], t.halves * C::A_HALF + C::B_BYTES);
+          // A operand: one 128-row half per TMA box (K-major), or 128-byte column chunks (MN-major)
           if constexpr (!C::A_MN) {
-            tma_load_2d(&tmA, &full[stage], sa, kb * C::BK, t.m0);
+            for (int hh = 0; hh < t.halves; ++hh)
+              tma_load_2d(&tmA, &full[stage], sa + hh * C::A_HALF, kb * C::BK, t.m0 + hh * 128);
           } else {
-#pragma unroll
-            for (int ch = 0; ch < C::BM / C::CH; ++ch)
+            for (int ch = 0; ch < t.halves * (128 / C::CH); ++ch)
               tma_load_2d(&tmA, &full[stage], sa + ch * (C::BK * 128), t.m0 + ch * C::CH,
                           t.krow0 + kb * C::BK);
           }
@@ -323,14 +402,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int L = blockIdx.x; L < n_tiles && ok; L += gridDim.x) {
-        const Tile t = decode_tile<C>(a, gs, off, L);
+        const Tile t = decode_tile<C>(a, gs, off, ts, L);
         if (t.nk == 0) continue;  // the epilogue writes zeros without TMEM
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u)) {
           report(a.status, DEV_WAIT_TIMEOUT_MMA);
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
+        // accumulator of half hh of buffer acc: TMEM columns [(acc*H + hh) * BN, +BN)
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::H * C::BN);
         for (int kb = 0; kb < t.nk; ++kb) {
           if (!mbar_wait(&full[stage], phase)) {
             report(a.status, DEV_WAIT_TIMEOUT_MMA);
@@ -342,15 +422,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < C::KSTEPS; ++kk) {
-            const uint64_t ad = C::A_MN ? smem_desc_sw128(sa + kk * C::UK * 128, C::BK * 128, 1024)
-                                        : smem_desc_sw128(sa + kk * C::UK * C::ESZ, 16, 1024);
             const uint64_t bd = C::B_MN ? smem_desc_sw128(sb + kk * C::UK * 128, C::BK * 128, 1024)
                                         : smem_desc_sw128(sb + kk * C::UK * C::ESZ, 16, 1024);
             const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
-            if constexpr (C::TF32)
-              umma_tf32(d_tmem, ad, bd, C::IDESC, accum);
-            else
-              umma_bf16(d_tmem, ad, bd, C::IDESC, accum);
+            for (int hh = 0; hh < t.halves; ++hh) {
+              const uint32_t sah = sa + hh * C::A_HALF;
+              const uint64_t ad = C::A_MN ? smem_desc_sw128(sah + kk * C::UK * 128, C::BK * 128, 1024)
+                                          : smem_desc_sw128(sah + kk * C::UK * C::ESZ, 16, 1024);
+              if constexpr (C::TF32)
+                umma_tf32(d_tmem + hh * C::BN, ad, bd, C::IDESC, accum);
+              else
+                umma_bf16(d_tmem + hh * C::BN, ad, bd, C::IDESC, accum);
+            }
           }
           umma_commit(&empty[stage]);  // frees the smem slot once these MMAs finish
           if (++stage == C::STAGES) {
@@ -360,7 +443,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         if (!ok) break;
         umma_commit(&acc_full[acc]);
-        if (++acc == 2) {
+        if (++acc == C::ACC_BUFS) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -370,27 +453,48 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (!mbar_wait(drain, 0)) report(a.status, DEV_WAIT_TIMEOUT_DRAIN);
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 2..5)
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // ------------------------------------------------ epilogue (warps 2 .. 2 + 4H)
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int grp = (warp - 2) >> 2;   // 0 .. 2H-1
+    const int hsel = grp >> 1;         // which 128-row half of the tile
+    const int csel = grp & 1;          // which half of the tile's columns
     const int r_local = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     T* out = static_cast<T*>(a.out);
     for (int L = blockIdx.x; L < n_tiles; L += gridDim.x) {
-      const Tile t = decode_tile<C>(a, gs, off, L);
-      const bool row_ok = r_local < t.valid;
-      const int64_t row = static_cast<int64_t>(t.m0) + r_local;
-      T* orow;
+      const Tile t = decode_tile<C>(a, gs, off, ts, L);
+      if (hsel >= t.halves) {  // this half lies past the expert's rows: nothing to store
+        if (t.nk == 0) continue;
+        if (!mbar_wait(&acc_full[acc], acc_phase)) {
+          report(a.status, DEV_WAIT_TIMEOUT_EPILOGUE);
+          break;
+        }
+        mbar_arrive(&acc_empty[acc]);
+        if (++acc == C::ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+        continue;
+      }
+      const bool row_ok = hsel * 128 + r_local < t.valid;
+      const int64_t wrow0 = static_cast<int64_t>(t.m0) + hsel * 128 + q * 32;  // the warp's first row
+      const int64_t row = wrow0 + lane;
+      // this warp's share of the tile's output columns
+      constexpr int WCOLS = C::OUT_N / 2;
+      const int cw = csel * WCOLS;
+      T* obase;  // (wrow0, n0 + cw)
       if constexpr (C::G == Group::M)
-        orow = out + row * a.ld_out + t.n0;
+        obase = out + wrow0 * a.ld_out + t.n0 + cw;
       else
-        orow = out + static_cast<int64_t>(t.e) * a.out_expert_stride + row * a.ld_out + t.n0;
+        obase = out + static_cast<int64_t>(t.e) * a.out_expert_stride + wrow0 * a.ld_out + t.n0 + cw;
+      unsigned char* stg = stg_base + (warp - 2) * C::STG_WARP_BYTES;
 
       if (t.nk == 0) {  // K-grouped expert with no rows: its gradient is zero
-        float z[16];
+        float z[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) z[i] = 0.f;
-        for (int c = 0; c < C::OUT_N; c += 16) store16<T>(orow + c, z);
+        for (int i = 0; i < 32; ++i) z[i] = 0.f;
+        for (int c = 0; c < WCOLS; c += 32) warp_store_chunk<T, C::STG_PITCH>(stg, z, obase + c, a.ld_out, lane);
         continue;
       }
       if (!mbar_wait(&acc_full[acc], acc_phase)) {
@@ -398,67 +502,80 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + static_cast<uint32_t>(acc * C::BN) + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t tbase = tmem_base + static_cast<uint32_t>((acc * C::H + hsel) * C::BN + cw) +
+                             (static_cast<uint32_t>(q * 32) << 16);
 
       if constexpr (C::EP == Epi::Store) {
-        for (int c = 0; c < C::BN; c += 16) {
-          uint32_t r[16];
-          tmem_ld16(tbase + c, r);
+#pragma unroll 1
+        for (int c = 0; c < WCOLS; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c, r);
           tmem_ld_wait();
-          float v[16];
+          float v[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = row_ok ? __uint_as_float(r[i]) : 0.f;
-          store16<T>(orow + c, v);
+          for (int i = 0; i < 32; ++i) v[i] = row_ok ? __uint_as_float(r[i]) : 0.f;
+          warp_store_chunk<T, C::STG_PITCH>(stg, v, obase + c, a.ld_out, lane);
         }
       } else if constexpr (C::EP == Epi::SwigluFwd) {
-        T* prow = (a.out2 != nullptr) ? static_cast<T*>(a.out2) + row * a.ld_out2 + t.n0 : nullptr;
-        for (int c = 0; c < C::BN / 2; c += 16) {
-          uint32_t rg[16], ru[16];
-          tmem_ld16(tbase + c, rg);
-          tmem_ld16(tbase + C::BN / 2 + c, ru);
+        T* pbase = (a.out2 != nullptr) ? static_cast<T*>(a.out2) + wrow0 * a.ld_out2 + t.n0 + cw : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < WCOLS; c += 32) {
+          uint32_t rg[32], ru[32];
+          tmem_ld32(tbase + c, rg);                // gate columns
+          tmem_ld32(tbase + C::BN / 2 + c, ru);    // the matching up columns
           tmem_ld_wait();
-          float g[16], u[16], hv[16];
+          float hv[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            g[i] = row_ok ? __uint_as_float(rg[i]) : 0.f;
-            u[i] = row_ok ? __uint_as_float(ru[i]) : 0.f;
-            hv[i] = silu_f(g[i]) * u[i];
+          for (int i = 0; i < 32; ++i) {
+            const float g = row_ok ? __uint_as_float(rg[i]) : 0.f;
+            const float u = row_ok ? __uint_as_float(ru[i]) : 0.f;
+            hv[i] = silu_fast(g) * u;
           }
-          store16<T>(orow + c, hv);
-          if (prow != nullptr) {
-            store16<T>(prow + c, g);
-            store16<T>(prow + a.f_half + c, u);
+          warp_store_chunk<T, C::STG_PITCH>(stg, hv, obase + c, a.ld_out, lane);
+          if (pbase != nullptr) {
+            float g[32], u[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              g[i] = row_ok ? __uint_as_float(rg[i]) : 0.f;
+              u[i] = row_ok ? __uint_as_float(ru[i]) : 0.f;
+            }
+            warp_store_chunk<T, C::STG_PITCH>(stg, g, pbase + c, a.ld_out2, lane);
+            warp_store_chunk<T, C::STG_PITCH>(stg, u, pbase + a.f_half + c, a.ld_out2, lane);
           }
         }
       } else {  // SwigluBwd: accumulator holds dG for columns [n0, n0+BN)
-        const T* arow = static_cast<const T*>(a.aux) + row * a.ld_aux + t.n0;
-        for (int c = 0; c < C::BN; c += 16) {
-          uint32_t r[16];
-          tmem_ld16(tbase + c, r);
+        const T* arow = static_cast<const T*>(a.aux) + row * a.ld_aux + t.n0 + cw;
+#pragma unroll 1
+        for (int c = 0; c < WCOLS; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c, r);
           tmem_ld_wait();
-          float da[16], db[16];
-          if (row_ok) {
-            float av[16], bv[16];
-            load16<T>(arow + c, av);
-            load16<T>(arow + a.f_half + c, bv);
+          float da[32], db[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float dg = __uint_as_float(r[i]);
-              const float sg = 1.0f / (1.0f + __expf(-av[i]));
-              da[i] = dg * bv[i] * (sg * (1.0f + av[i] * (1.0f - sg)));
-              db[i] = dg * av[i] * sg;
+          for (int hh = 0; hh < 2; ++hh) {
+            if (row_ok) {
+              float av[16], bv[16];
+              load16<T>(arow + c + 16 * hh, av);
+              load16<T>(arow + a.f_half + c + 16 * hh, bv);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float dg = __uint_as_float(r[16 * hh + i]);
+                const float sg = __fdividef(1.0f, 1.0f + __expf(-av[i]));
+                da[16 * hh + i] = dg * bv[i] * (sg * (1.0f + av[i] * (1.0f - sg)));
+                db[16 * hh + i] = dg * av[i] * sg;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) da[16 * hh + i] = db[16 * hh + i] = 0.f;
             }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) da[i] = db[i] = 0.f;
           }
-          store16<T>(orow + c, da);
-          store16<T>(orow + a.f_half + c, db);
+          warp_store_chunk<T, C::STG_PITCH>(stg, da, obase + c, a.ld_out, lane);
+          warp_store_chunk<T, C::STG_PITCH>(stg, db, obase + a.f_half + c, a.ld_out, lane);
         }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
-      if (++acc == 2) {
+      if (++acc == C::ACC_BUFS) {
         acc = 0;
         acc_phase ^= 1u;
       }
@@ -474,6 +591,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 }
 
 // -------------------------------------------------------------- host side
+
+}  // namespace
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -505,6 +624,8 @@ bool make_map(CUtensorMap* m, const void* base, bool fp32, uint64_t rows, uint64
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+
 template <class C>
 cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Args& a, int max_tiles, cudaStream_t st) {
   static bool configured = false;
@@ -532,6 +653,25 @@ Args base_args(const Shape& s, const int32_t* gs, const int32_t* off, int32_t* s
 
 int ch_elems(bool fp32) { return fp32 ? 32 : 64; }
 
+// Instantiates the kernel for the dtype, tile N and tile M (h 128-row halves).
+template <bool A_MN, bool B_MN, Group G, Epi EP>
+cudaError_t run_variant(bool fp32, int bn, int h, const CUtensorMap& ta, const CUtensorMap& tb, const Args& a,
+                        int max_tiles, cudaStream_t st) {
+  if (fp32) {
+    if (bn == 256) return launch<Cfg<true, A_MN, B_MN, G, EP, 256, 1>>(ta, tb, a, max_tiles, st);
+    return launch<Cfg<true, A_MN, B_MN, G, EP, 128, 1>>(ta, tb, a, max_tiles, st);
+  }
+  (void)h;
+  if (bn == 256) return launch<Cfg<false, A_MN, B_MN, G, EP, 256, 1>>(ta, tb, a, max_tiles, st);
+  return launch<Cfg<false, A_MN, B_MN, G, EP, 128, 1>>(ta, tb, a, max_tiles, st);
+}
+
+// Tile M. 256-row tiles (H = 2) halve the operand bytes per MMA cycle, but two
+// 128 x 256 fp32 accumulators fill TMEM, so the epilogue of a tile cannot
+// overlap the next tile's MMAs; on B200 they measured slower than 128-row
+// tiles with double-buffered accumulators, so 128-row tiles are used.
+int pick_h(const Shape&) { return 1; }
+
 }  // namespace
 
 // Tile N for a forward GEMM whose accumulator covers `n` columns per expert.
@@ -557,12 +697,7 @@ cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* gr
   a.out2 = preact;
   a.ld_out2 = 2 * s.f;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.f / (bn / 2)));
-  if (s.fp32) {
-    if (bn == 256) return launch<Cfg<true, false, false, Group::M, Epi::SwigluFwd, 256>>(ta, tb, a, max_tiles, st);
-    return launch<Cfg<true, false, false, Group::M, Epi::SwigluFwd, 128>>(ta, tb, a, max_tiles, st);
-  }
-  if (bn == 256) return launch<Cfg<false, false, false, Group::M, Epi::SwigluFwd, 256>>(ta, tb, a, max_tiles, st);
-  return launch<Cfg<false, false, false, Group::M, Epi::SwigluFwd, 128>>(ta, tb, a, max_tiles, st);
+  return run_variant<false, false, Group::M, Epi::SwigluFwd>(s.fp32, bn, pick_h(s), ta, tb, a, max_tiles, st);
 }
 
 cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_start, const int32_t* offsets,
@@ -580,12 +715,7 @@ cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_star
   a.out = o_perm;
   a.ld_out = s.d;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.d / bn));
-  if (s.fp32) {
-    if (bn == 256) return launch<Cfg<true, false, false, Group::M, Epi::Store, 256>>(ta, tb, a, max_tiles, st);
-    return launch<Cfg<true, false, false, Group::M, Epi::Store, 128>>(ta, tb, a, max_tiles, st);
-  }
-  if (bn == 256) return launch<Cfg<false, false, false, Group::M, Epi::Store, 256>>(ta, tb, a, max_tiles, st);
-  return launch<Cfg<false, false, false, Group::M, Epi::Store, 128>>(ta, tb, a, max_tiles, st);
+  return run_variant<false, false, Group::M, Epi::Store>(s.fp32, bn, pick_h(s), ta, tb, a, max_tiles, st);
 }
 
 // dG = dO W_down (K = d, B read MN-major from W_down [E*d, f]); epilogue forms
@@ -609,12 +739,7 @@ cudaError_t launch_down_backward_data(const Shape& s, const void* dout, const in
   a.aux = preact;
   a.ld_aux = 2 * s.f;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.f / bn));
-  if (s.fp32) {
-    if (bn == 256) return launch<Cfg<true, false, true, Group::M, Epi::SwigluBwd, 256>>(ta, tb, a, max_tiles, st);
-    return launch<Cfg<true, false, true, Group::M, Epi::SwigluBwd, 128>>(ta, tb, a, max_tiles, st);
-  }
-  if (bn == 256) return launch<Cfg<false, false, true, Group::M, Epi::SwigluBwd, 256>>(ta, tb, a, max_tiles, st);
-  return launch<Cfg<false, false, true, Group::M, Epi::SwigluBwd, 128>>(ta, tb, a, max_tiles, st);
+  return run_variant<false, true, Group::M, Epi::SwigluBwd>(s.fp32, bn, pick_h(s), ta, tb, a, max_tiles, st);
 }
 
 // dX_perm = [dA|dB] W_gate_up (K = 2f, B read MN-major from W_gate_up [E*2f, d]).
@@ -635,12 +760,7 @@ cudaError_t launch_gate_up_backward_data(const Shape& s, const void* dab, const 
   a.out = dx_perm;
   a.ld_out = s.d;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.d / bn));
-  if (s.fp32) {
-    if (bn == 256) return launch<Cfg<true, false, true, Group::M, Epi::Store, 256>>(ta, tb, a, max_tiles, st);
-    return launch<Cfg<true, false, true, Group::M, Epi::Store, 128>>(ta, tb, a, max_tiles, st);
-  }
-  if (bn == 256) return launch<Cfg<false, false, true, Group::M, Epi::Store, 256>>(ta, tb, a, max_tiles, st);
-  return launch<Cfg<false, false, true, Group::M, Epi::Store, 128>>(ta, tb, a, max_tiles, st);
+  return run_variant<false, true, Group::M, Epi::Store>(s.fp32, bn, pick_h(s), ta, tb, a, max_tiles, st);
 }
 
 namespace {
@@ -659,13 +779,9 @@ cudaError_t launch_kgrouped(const Shape& s, const void* A, int M_total, const vo
   a.out = out;
   a.ld_out = N_total;
   a.out_expert_stride = static_cast<int64_t>(M_total) * N_total;
-  const int max_tiles = s.E * (M_total / 128) * (N_total / bn);
-  if (s.fp32) {
-    if (bn == 256) return launch<Cfg<true, true, true, Group::K, Epi::Store, 256>>(ta, tb, a, max_tiles, st);
-    return launch<Cfg<true, true, true, Group::K, Epi::Store, 128>>(ta, tb, a, max_tiles, st);
-  }
-  if (bn == 256) return launch<Cfg<false, true, true, Group::K, Epi::Store, 256>>(ta, tb, a, max_tiles, st);
-  return launch<Cfg<false, true, true, Group::K, Epi::Store, 128>>(ta, tb, a, max_tiles, st);
+  const int h = pick_h(s);
+  const int max_tiles = s.E * (M_total / (128 * h)) * (N_total / bn);
+  return run_variant<true, true, Group::K, Epi::Store>(s.fp32, bn, h, ta, tb, a, max_tiles, st);
 }
 }  // namespace
 

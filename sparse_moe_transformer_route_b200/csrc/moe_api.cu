@@ -166,10 +166,18 @@ moe_status forward_impl(const Ctx& c, const void* x, const void* w_router, const
   int32_t* off = at<int32_t>(ws, L.offsets);
   const StageMarks marks(st);
   MOE_TRY(marks.mark(0));
-  MOE_TRY(launch_router(s, x, w_router, bias, idx, wts, nullptr, losses, ws, L, st));
-  MOE_TRY(marks.mark(1));
-  MOE_TRY(launch_dispatch_impl(s, idx, x, nullptr, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv_perm), nullptr,
-                               at<void>(ws, L.x_perm), ws, L, save, st));
+  if (router_tc_supported(s)) {
+    // the tensor-core router also leaves the dispatch ranking in ws
+    MOE_TRY(launch_router_tc(s, x, w_router, bias, idx, wts, nullptr, losses, ws, L, st));
+    MOE_TRY(marks.mark(1));
+    MOE_TRY(launch_permute(s, idx, x, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv_perm), at<void>(ws, L.x_perm), ws,
+                           L, save, st));
+  } else {
+    MOE_TRY(launch_router(s, x, w_router, bias, idx, wts, nullptr, losses, ws, L, st));
+    MOE_TRY(marks.mark(1));
+    MOE_TRY(launch_dispatch_impl(s, idx, x, nullptr, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv_perm), nullptr,
+                                 at<void>(ws, L.x_perm), ws, L, save, st));
+  }
   MOE_TRY(marks.mark(2));
   MOE_TRY(launch_gate_up(s, at<void>(ws, L.x_perm), gs, off, w_gate_up, at<void>(ws, L.h),
                          save ? at<void>(ws, L.preact) : nullptr, status, st));
@@ -236,7 +244,10 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
   if (x == nullptr || w_router == nullptr || topk_idx == nullptr || topk_w == nullptr || !aligned16(x) ||
       !aligned16(w_router))
     return MOE_ERR_INVALID_ARG;
-  MOE_TRY(launch_router(c.s, x, w_router, router_bias, topk_idx, topk_w, counts, losses, ws, c.L, stream));
+  if (router_tc_supported(c.s))
+    MOE_TRY(launch_router_tc(c.s, x, w_router, router_bias, topk_idx, topk_w, counts, losses, ws, c.L, stream));
+  else
+    MOE_TRY(launch_router(c.s, x, w_router, router_bias, topk_idx, topk_w, counts, losses, ws, c.L, stream));
   return MOE_OK;
 }
 

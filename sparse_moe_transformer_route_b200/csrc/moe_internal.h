@@ -2,6 +2,7 @@
 // launchers: the workspace layout and the launcher signatures.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -13,7 +14,7 @@ namespace moe {
 
 constexpr int kRowAlign = MOE_ROW_ALIGN;  // expert groups start on multiples of this
 constexpr int kRouterTokensPerCta = 16;   // router kernel token block
-constexpr int kDispatchChunk = 256;       // tokens per dispatch ranking chunk
+constexpr int kDispatchChunk = 32;        // tokens per dispatch ranking chunk (= one router tile)
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 16;
 
@@ -56,6 +57,15 @@ inline T* at(void* ws, size_t off) {
 cudaError_t launch_router(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
                           float* wts, int32_t* counts, float* losses, void* ws, const Workspace& L,
                           cudaStream_t st);
+// Tensor-core router (bf16, E <= 64). Besides launch_router's outputs it leaves
+// the dispatch ranking in the workspace (local ranks, per-chunk counts and
+// bases, offsets, group starts), so the rank kernel can be skipped.
+bool router_tc_supported(const Shape& s);
+cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
+                             float* wts, int32_t* counts, float* losses, void* ws, const Workspace& L,
+                             cudaStream_t st);
+cudaError_t launch_permute(const Shape& s, const int32_t* idx, const void* x, int32_t* perm, int32_t* inv_perm,
+                           void* x_perm, void* ws, const Workspace& L, bool zero_pads, cudaStream_t st);
 cudaError_t launch_dispatch(const Shape& s, const int32_t* idx, const void* x, int32_t* offsets, int32_t* perm,
                             int32_t* inv_perm, int32_t* group_start, void* x_perm, void* ws, const Workspace& L,
                             cudaStream_t st);
@@ -95,5 +105,10 @@ cudaError_t launch_router_weight_grad(const Shape& s, const float* dh, const voi
 size_t router_wgrad_partial_bytes(const Shape& s);
 
 int device_sm_count();
+
+// 2-D TMA descriptor over a row-major [rows, cols] bf16/fp32 matrix with a
+// [box_rows, box_cols] box and 128-byte swizzle (out-of-range boxes read zeros).
+bool make_map(CUtensorMap* m, const void* base, bool fp32, uint64_t rows, uint64_t cols, uint32_t box_cols,
+              uint32_t box_rows);
 
 }  // namespace moe

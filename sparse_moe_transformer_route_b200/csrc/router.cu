@@ -186,9 +186,19 @@ __global__ void __launch_bounds__(kThreads) router_kernel(
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int c = 0;
     double pe = 0.0;
-    for (int b = 0; b < nb; ++b) {
-      c += __ldcg(&counts_part[static_cast<size_t>(b) * E + e]);
-      pe += static_cast<double>(__ldcg(&psum_part[static_cast<size_t>(b) * E + e]));
+    for (int b0 = 0; b0 < nb; b0 += 16) {  // batched so the L2 round trips overlap
+      int cv[16];
+      float pv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        cv[i] = (b0 + i < nb) ? __ldcg(&counts_part[static_cast<size_t>(b0 + i) * E + e]) : 0;
+        pv[i] = (b0 + i < nb) ? __ldcg(&psum_part[static_cast<size_t>(b0 + i) * E + e]) : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        c += cv[i];
+        pe += static_cast<double>(pv[i]);
+      }
     }
     counts_ws[e] = c;
     if (counts_user != nullptr) counts_user[e] = c;
@@ -198,7 +208,13 @@ __global__ void __launch_bounds__(kThreads) router_kernel(
   __syncthreads();
   if (threadIdx.x == 0) {
     double z = 0.0;
-    for (int b = 0; b < nb; ++b) z += __ldcg(&zsum_part[b]);
+    for (int b0 = 0; b0 < nb; b0 += 16) {
+      double zv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) zv[i] = (b0 + i < nb) ? __ldcg(&zsum_part[b0 + i]) : 0.0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) z += zv[i];
+    }
     const double Td = static_cast<double>(T);
     double lb = 0.0;
     for (int e = 0; e < E; ++e) lb += (static_cast<double>(cnt[e]) / (Td * k)) * (s_psum[e] / Td);

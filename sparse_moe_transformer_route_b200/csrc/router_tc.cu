@@ -1,0 +1,624 @@
+// Tensor-core router for bf16 layers with up to 64 experts: logits on tcgen05,
+// softmax over all experts, top-k without renormalisation, both loss partials
+// and the dispatch ranking, in one kernel.
+//
+// Method: "Mixture-of-experts LLMs from scratch with OLMoE", section 2
+// (softmax over all experts, then the k largest probabilities are both the
+// choice and the weights; OLMoE does not renormalise, section 3) and section 3
+// MoE.forward (fp32 scores, optional per-expert offset); "OLMoE Guide",
+// "Router Mechanics & Loss Formulations" (f_i, P_i, L_lb, L_z).
+//
+// One CTA takes 32 tokens (one dispatch chunk), so a 4096-token layer spreads
+// over 128 SMs:
+//   warp 0     TMA loads of x [32 x 64] and W_r [E_pad x 64] per K step into a
+//              16-deep ring. The MMA reads a 128-row A operand; rows 32..127
+//              are whatever lies in shared memory after the 32 loaded rows,
+//              and their accumulator rows are never read.
+//   warp 1     tcgen05.mma M=128 N=E_pad K=16, fp32 accumulator in TMEM
+//   warps 2..5 epilogue. Warp 4 (TMEM lanes 0..31) copies the 32 tokens'
+//              logits to shared memory; then a quad of threads takes each
+//              token, 16 experts per thread: softmax with quad reductions, the
+//              top k+3 in fp32 by quad arg-max, and the top-k decided with
+//              exact logits where fp32 cannot: every run of neighbours among
+//              the first k+1 whose fp32 gaps are under 2e-4 * max(1, |logit|)
+//              (far above the accumulation error of a 2048-long fp32 sum of
+//              exact bf16 products) is recomputed exactly (fp64 sums of exact
+//              products) and re-ranked; ties in the exact values go to the
+//              lower expert index. Probabilities, weights and the log-normaliser
+//              come from the fp32 logits.
+// A 32-bit mask per expert of the tokens that chose it gives each (token,
+// slot) pair its rank inside the chunk. The last CTA to finish scans the
+// per-chunk counts (block by block, through shared memory) into chunk bases,
+// the bincount offsets and the padded group starts, and reduces the loss
+// partials. Every sum runs in a fixed order, so the results are deterministic.
+#include <cfloat>
+#include <cmath>
+
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTile = kDispatchChunk;  // 32 tokens
+constexpr int kStages = 16;
+constexpr int kThreads = 192;
+constexpr int kMaxE = 64;
+constexpr int kMaxSel = kMaxTopK + 3;
+constexpr int kAload = kTile * 128;                      // bytes of A loaded per stage
+constexpr int kStageMax = kAload + kMaxE * 128;          // 12 KB
+constexpr int kRing = kStages * kStageMax + 16 * 1024;   // + the over-read of the last stage's A
+constexpr int kLogitStride = kMaxE + 1;
+constexpr int kScanBlock = 256;                          // chunks scanned per pass in the last CTA
+constexpr size_t kMiscBytes = 4096;
+constexpr size_t kSmem = 1024 + static_cast<size_t>(kRing) + kMiscBytes;
+static_assert(kTile == 32, "one mask word per expert");
+static_assert(kScanBlock * kMaxE * 8 <= kRing, "scan block fits in the ring");
+
+struct RArgs {
+  int64_t T;
+  int d, E, k, NP;
+  const float* bias;
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* w;
+  int32_t* idx_out;
+  float* w_out;
+  float* probs;
+  float* lse_out;
+  int32_t* local_rank;
+  int32_t* chunk_count;
+  int32_t* chunk_base;
+  float* psum_part;
+  double* zsum_part;
+  int32_t* counts_ws;
+  int32_t* counts_user;
+  float* losses_ws;
+  float* losses_user;
+  int32_t* offsets_ws;
+  int32_t* gs_ws;
+  int32_t* ticket;
+  int32_t* status;
+};
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ float near_gap(float v) { return 2e-4f * fmaxf(1.0f, fabsf(v)); }
+
+// Arg-max across the 4 threads of a quad: larger value wins, equal values go to the lower index.
+// Quads may diverge (near-ties, the ragged last tile), so every quad shuffle
+// names only its own four lanes.
+__device__ __forceinline__ unsigned quad_mask() { return 0xFu << ((threadIdx.x & 31) & 28); }
+
+template <typename V>
+__device__ __forceinline__ void quad_argmax(V& v, int& i) {
+  const unsigned qm = quad_mask();
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    const V ov = __shfl_xor_sync(qm, v, o);
+    const int oi = __shfl_xor_sync(qm, i, o);
+    if (ov > v || (ov == v && oi < i)) {
+      v = ov;
+      i = oi;
+    }
+  }
+}
+
+// <x_t, W_r[e]> from exact products of bf16 inputs, summed in fp64 by a whole
+// warp: lane l takes elements 8l + 256i; the loads of up to 16 steps are issued
+// before any arithmetic so the row pair costs about one memory round trip. The
+// lane sums are combined by a fixed shuffle tree (every lane gets the result).
+__device__ __forceinline__ double exact_logit_warp(const __nv_bfloat16* xr, const __nv_bfloat16* wr, int d,
+                                                   int lane) {
+  constexpr int kBatch = 16;
+  double acc = 0.0;
+  for (int base = lane * 8; base < d; base += 256 * kBatch) {
+    uint4 xv[kBatch], wv[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int i = base + 256 * b;
+      if (i < d) {
+        xv[b] = *reinterpret_cast<const uint4*>(xr + i);
+        wv[b] = *reinterpret_cast<const uint4*>(wr + i);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      if (base + 256 * b < d) {
+        const uint32_t xa[4] = {xv[b].x, xv[b].y, xv[b].z, xv[b].w}, wa[4] = {wv[b].x, wv[b].y, wv[b].z, wv[b].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xa[c]));
+          const float2 wf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[c]));
+          acc = fma(static_cast<double>(xf.x), static_cast<double>(wf.x), acc);
+          acc = fma(static_cast<double>(xf.y), static_cast<double>(wf.y), acc);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
+                     const RArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int STAGE = kAload + a.NP * 128;  // A rows 0..31, then B
+  unsigned char* ring = smem;
+  unsigned char* misc = smem + kRing;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint32_t* mask = tmem_holder + 4;                          // [kMaxE]
+  float* lse_s = reinterpret_cast<float*>(mask + kMaxE);      // [kTile]
+  int32_t* s_last = reinterpret_cast<int32_t*>(lse_s + kTile);
+  int32_t* tot = s_last + 4;                                  // [kMaxE]
+  double* tot_p = reinterpret_cast<double*>(tot + kMaxE);     // [kMaxE]
+  double* zred = tot_p + kMaxE;                               // [128]
+  // once the accumulator is complete the ring is free
+  float* S = reinterpret_cast<float*>(ring);                          // [kTile][kLogitStride] logits
+  float* P = S + kTile * kLogitStride;                                 // [kTile][kMaxE] probabilities
+  int32_t* chosen = reinterpret_cast<int32_t*>(P + kTile * kMaxE);     // [kTile][kMaxTopK]
+  uint32_t* queue = reinterpret_cast<uint32_t*>(ring + 20480);         // [kTile * kMaxE] (token << 8) | expert
+  double* exact = reinterpret_cast<double*>(ring + 20480 + kTile * kMaxE * 4);  // [kTile * kMaxE]
+  int32_t* qn = s_last + 1;                                            // queued pairs
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = a.d / 64;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, a.NP <= 32 ? 32u : 64u);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmx);
+      tma_prefetch_desc(&tmw);
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = static_cast<uint32_t>(kb / kStages) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u)) {
+          report(a.status, DEV_WAIT_TIMEOUT_PRODUCER);
+          break;
+        }
+        unsigned char* st = ring + static_cast<size_t>(s) * STAGE;
+        mbar_arrive_expect_tx(&full[s], STAGE);
+        tma_load_2d(&tmx, &full[s], st, kb * 64, static_cast<int32_t>(t0));
+        tma_load_2d(&tmw, &full[s], st + kAload, kb * 64, 0);
+        ++issued;
+      }
+      for (int s = 0; s < kStages && s < issued; ++s) {
+        const int last = ((issued - 1 - s) / kStages) * kStages + s;
+        if (!mbar_wait(&full[s], static_cast<uint32_t>((last / kStages) & 1))) report(a.status, DEV_WAIT_TIMEOUT_DRAIN);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(false, false, false, 128, a.NP);
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kStages;
+        if (!mbar_wait(&full[s], static_cast<uint32_t>(kb / kStages) & 1u)) {
+          report(a.status, DEV_WAIT_TIMEOUT_MMA);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(ring + static_cast<size_t>(s) * STAGE);
+        const uint32_t sb = sa + kAload;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024), idesc,
+                    (kb > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&empty[s]);
+      }
+      if (ok) umma_commit(acc_full);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int tid = threadIdx.x - 64;  // 0..127
+    const int E = a.E, k = a.k;
+    if (tid < kMaxE) mask[tid] = 0u;
+    if (tid == 0) *qn = 0;
+    if (!mbar_wait(acc_full, 0)) report(a.status, DEV_WAIT_TIMEOUT_EPILOGUE);
+    tc_fence_after();
+    if (warp == 4) {  // TMEM lanes 0..31 hold the 32 tokens' logits
+      for (int c = 0; c < a.NP; c += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int e = c + i;
+          float h = __uint_as_float(v[i]);
+          if (e < E && a.bias != nullptr) h += a.bias[e];
+          S[lane * kLogitStride + e] = (e < E) ? h : -INFINITY;
+        }
+      }
+      for (int e = a.NP; e < kMaxE; ++e) S[lane * kLogitStride + e] = -INFINITY;
+    }
+    tc_fence_before();
+    epi_sync();
+
+    // ---- a quad per token: thread qp holds experts 16*qp .. 16*qp+15
+    const int r = tid >> 2, qp = tid & 3;
+    const int64_t t = t0 + r;
+    const bool valid = t < a.T;  // the whole quad agrees
+    const int eb = qp * 16;
+    float h[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) h[i] = S[r * kLogitStride + eb + i];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, h[i]);
+    const unsigned qm = quad_mask();
+    m = fmaxf(m, __shfl_xor_sync(qm, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(qm, m, 2));
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s += (eb + i < E) ? expf(h[i] - m) : 0.f;
+    s += __shfl_xor_sync(qm, s, 1);
+    s += __shfl_xor_sync(qm, s, 2);
+    const float lse = m + logf(s);
+    {
+      float pv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pv[i] = (valid && eb + i < E) ? expf(h[i] - m) / s : 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) P[r * kMaxE + eb + i] = pv[i];
+      if (valid && eb < E) {
+        float* dst = a.probs + t * E + eb;
+        if (eb + 16 <= E) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            reinterpret_cast<float4*>(dst)[i] = make_float4(pv[4 * i], pv[4 * i + 1], pv[4 * i + 2], pv[4 * i + 3]);
+        } else {
+          for (int i = 0; i < E - eb; ++i) dst[i] = pv[i];
+        }
+      }
+    }
+    if (qp == 0) {
+      lse_s[r] = valid ? lse : 0.f;
+      if (valid) a.lse_out[t] = lse;
+    }
+
+    // ---- top (k+3) in fp32 by quad arg-max (uniform within the quad)
+    const int nsel = min(k + 3, E);
+    int ord[kMaxSel];
+    float val[kMaxSel];
+    uint32_t taken = 0;  // bit i: expert eb + i chosen
+#pragma unroll
+    for (int j = 0; j < kMaxSel; ++j) {
+      if (j < nsel) {
+        float v = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (eb + i < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || h[i] > v)) {
+            v = h[i];
+            bi = eb + i;
+          }
+        }
+        quad_argmax(v, bi);
+        if (bi - eb >= 0 && bi - eb < 16) taken |= 1u << (bi - eb);
+        ord[j] = bi;
+        val[j] = v;
+      }
+    }
+    float hv[kMaxSel];
+#pragma unroll
+    for (int j = 0; j < kMaxSel; ++j) hv[j] = val[j];
+    // runs of near-equal neighbours that decide a slot order or the k-th choice
+    bool fallback = false;
+    int run_a[kMaxSel], run_b[kMaxSel];
+    int nrun = 0;
+    if (valid) {
+      int jj = 0;
+      while (jj < nsel - 1) {
+        if (val[jj] - val[jj + 1] < near_gap(val[jj])) {
+          int b = jj + 1;
+          while (b < nsel - 1 && val[b] - val[b + 1] < near_gap(val[b])) ++b;
+          if (jj <= k - 1) {
+            if (b == nsel - 1 && nsel < E) {
+              fallback = true;
+              break;
+            }
+            run_a[nrun] = jj;
+            run_b[nrun] = b;
+            ++nrun;
+          }
+          jj = b;
+        } else {
+          ++jj;
+        }
+      }
+    }
+    // queue the (token, expert) pairs whose exact logits are needed
+    int nitems = 0;
+    if (fallback) {
+      nitems = E;
+    } else {
+      for (int i = 0; i < nrun; ++i) nitems += run_b[i] - run_a[i] + 1;
+    }
+    int qbase = 0;
+    if (qp == 0 && nitems > 0) qbase = atomicAdd(qn, nitems);
+    qbase = __shfl_sync(qm, qbase, lane & ~3);
+    if (fallback) {
+      for (int e = qp; e < E; e += 4) queue[qbase + e] = (static_cast<uint32_t>(r) << 8) | static_cast<uint32_t>(e);
+    } else {
+      int p = 0;
+      for (int i = 0; i < nrun; ++i)
+        for (int y = run_a[i]; y <= run_b[i]; ++y, ++p)
+          if ((p & 3) == qp) queue[qbase + p] = (static_cast<uint32_t>(r) << 8) | static_cast<uint32_t>(ord[y]);
+    }
+    epi_sync();
+    // ---- exact logits of the queued pairs: a warp per pair, all loads in flight together
+    {
+      const int nq = *qn;
+      const int ew = tid >> 5;
+      for (int it = ew; it < nq; it += 4) {
+        const uint32_t code = queue[it];
+        const int rr = static_cast<int>(code >> 8), e = static_cast<int>(code & 255u);
+        const double v = exact_logit_warp(a.x + (t0 + rr) * a.d, a.w + static_cast<int64_t>(e) * a.d, a.d, lane);
+        if (lane == 0) exact[it] = v + (a.bias != nullptr ? static_cast<double>(a.bias[e]) : 0.0);
+      }
+    }
+    epi_sync();
+    // ---- re-rank each run by its exact logits (ties: lower expert index)
+    if (!fallback && nrun > 0) {
+      int p = qbase;
+      for (int i = 0; i < nrun; ++i) {
+        const int ra = run_a[i], rb = run_b[i];
+        double ex[kMaxSel];
+        for (int y = ra; y <= rb; ++y) ex[y] = exact[p++];
+        for (int x1 = ra + 1; x1 <= rb; ++x1) {
+          const double ve = ex[x1];
+          const int oe = ord[x1];
+          const float he = hv[x1];
+          int y = x1 - 1;
+          while (y >= ra && (ex[y] < ve || (ex[y] == ve && ord[y] > oe))) {
+            ex[y + 1] = ex[y];
+            ord[y + 1] = ord[y];
+            hv[y + 1] = hv[y];
+            --y;
+          }
+          ex[y + 1] = ve;
+          ord[y + 1] = oe;
+          hv[y + 1] = he;
+        }
+      }
+    }
+    if (fallback) {  // a run reaches past rank k+3: rank every expert by its exact logit
+      double xe[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xe[i] = (eb + i < E) ? exact[qbase + eb + i] : -INFINITY;
+      uint32_t tk = 0;
+      for (int j = 0; j < k; ++j) {
+        double v = -INFINITY;
+        int bi = 0x7fffffff;
+        float hb = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (eb + i < E && !((tk >> i) & 1u) && (bi == 0x7fffffff || xe[i] > v)) {
+            v = xe[i];
+            bi = eb + i;
+            hb = h[i];
+          }
+        }
+        quad_argmax(v, bi);
+        if (bi - eb >= 0 && bi - eb < 16) tk |= 1u << (bi - eb);
+        ord[j] = bi;
+        // the fp32 logit of the winner, from the thread that holds it
+        const float mine = hb;
+        const int owner = (lane & ~3) | ((bi >> 4) & 3);
+        hv[j] = __shfl_sync(qm, (bi >= eb && bi < eb + 16) ? mine : 0.f, owner);
+      }
+    }
+    // ---- outputs: thread qp writes slots qp, qp+4, ...
+    if (valid) {
+      for (int j = qp; j < k; j += 4) {
+        const int e = ord[j];
+        a.idx_out[t * k + j] = e;
+        a.w_out[t * k + j] = expf(hv[j] - m) / s;
+        chosen[r * kMaxTopK + j] = e;
+        atomicOr(&mask[e], 1u << r);
+      }
+    }
+    epi_sync();
+    // ---- ranks inside the chunk and per-CTA partials
+    if (valid) {
+      for (int j = qp; j < k; j += 4) {
+        const int e = chosen[r * kMaxTopK + j];
+        a.local_rank[t * k + j] = __popc(mask[e] & ((1u << r) - 1u));
+      }
+    }
+    const int cta = blockIdx.x;
+    if (tid < E) {
+      a.chunk_count[static_cast<size_t>(cta) * E + tid] = __popc(mask[tid]);
+      float ps = 0.f;
+      for (int rr = 0; rr < kTile; ++rr) ps += P[rr * kMaxE + tid];
+      a.psum_part[static_cast<size_t>(cta) * E + tid] = ps;
+    }
+    if (tid == 0) {
+      double z = 0.0;
+      for (int rr = 0; rr < kTile; ++rr) z += static_cast<double>(lse_s[rr]) * lse_s[rr];
+      a.zsum_part[cta] = z;
+    }
+    __threadfence();
+    epi_sync();
+    if (tid == 0) *s_last = (atomicAdd(a.ticket, 1) == static_cast<int>(gridDim.x) - 1);
+    epi_sync();
+    if (*s_last) {
+      __threadfence();
+      const int nb = gridDim.x;
+      int32_t* cnt_s = reinterpret_cast<int32_t*>(ring);                     // [kScanBlock][E]
+      float* ps_s = reinterpret_cast<float*>(ring + kScanBlock * kMaxE * 4);  // [kScanBlock][E]
+      int run = 0;       // thread tid < E: running total of expert tid
+      double pe = 0.0;
+      for (int c0 = 0; c0 < nb; c0 += kScanBlock) {
+        const int nc = min(kScanBlock, nb - c0);
+        // the block's counts and probability sums, read with all 128 threads as
+        // 16-byte loads, eight in flight per thread (c0 * E is a multiple of 4)
+        {
+          const int n = nc * E;
+          const int32_t* gc = a.chunk_count + static_cast<size_t>(c0) * E;
+          const float* gp = a.psum_part + static_cast<size_t>(c0) * E;
+          for (int i0 = tid * 4; i0 < (n & ~3); i0 += 128 * 4 * 8) {
+            int4 cv[8];
+            float4 pv[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+              const int i = i0 + b * 512;
+              if (i < (n & ~3)) {
+                cv[b] = __ldcg(reinterpret_cast<const int4*>(gc + i));
+                pv[b] = __ldcg(reinterpret_cast<const float4*>(gp + i));
+              }
+            }
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+              const int i = i0 + b * 512;
+              if (i < (n & ~3)) {
+                *reinterpret_cast<int4*>(cnt_s + i) = cv[b];
+                *reinterpret_cast<float4*>(ps_s + i) = pv[b];
+              }
+            }
+          }
+          for (int i = (n & ~3) + tid; i < n; i += 128) {
+            cnt_s[i] = __ldcg(gc + i);
+            ps_s[i] = __ldcg(gp + i);
+          }
+        }
+        epi_sync();
+        if (tid < E) {
+          for (int c = 0; c < nc; ++c) {
+            const int v = cnt_s[c * E + tid];
+            cnt_s[c * E + tid] = run;  // becomes the chunk base
+            run += v;
+            pe += static_cast<double>(ps_s[c * E + tid]);
+          }
+        }
+        epi_sync();
+        for (int i = tid; i < nc * E; i += 128) a.chunk_base[static_cast<size_t>(c0) * E + i] = cnt_s[i];
+        epi_sync();
+      }
+      if (tid < E) {
+        tot[tid] = run;
+        tot_p[tid] = pe;
+        a.counts_ws[tid] = run;
+        if (a.counts_user != nullptr) a.counts_user[tid] = run;
+      }
+      // sum of lse^2 partials: 128 contiguous slices in order, then the slices in order
+      {
+        const int per = (nb + 127) / 128;
+        double z = 0.0;
+        for (int c = tid * per; c < min(nb, (tid + 1) * per); ++c) z += __ldcg(&a.zsum_part[c]);
+        zred[tid] = z;
+      }
+      epi_sync();
+      if (tid == 0) {
+        double zt = 0.0;
+        for (int i = 0; i < 128; ++i) zt += zred[i];
+        int off = 0, gsv = 0;
+        double lb = 0.0;
+        const double Td = static_cast<double>(a.T);
+        for (int e = 0; e < E; ++e) {
+          a.offsets_ws[e] = off;
+          a.gs_ws[e] = gsv;
+          off += tot[e];
+          gsv += (tot[e] + kRowAlign - 1) / kRowAlign * kRowAlign;
+          lb += (static_cast<double>(tot[e]) / (Td * k)) * (tot_p[e] / Td);
+        }
+        a.offsets_ws[E] = off;
+        a.gs_ws[E] = gsv;
+        const float l0 = static_cast<float>(lb * E), l1 = static_cast<float>(zt / Td);
+        a.losses_ws[0] = l0;
+        a.losses_ws[1] = l1;
+        if (a.losses_user != nullptr) {
+          a.losses_user[0] = l0;
+          a.losses_user[1] = l1;
+        }
+        if (static_cast<int64_t>(off) != a.T * k) report(a.status, DEV_COUNT_MISMATCH);
+        *a.ticket = 0;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, a.NP <= 32 ? 32u : 64u);
+  }
+}
+
+}  // namespace
+
+bool router_tc_supported(const Shape& s) { return !s.fp32 && s.E <= kMaxE && s.k + 3 <= kMaxSel; }
+
+cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
+                             float* wts, int32_t* counts, float* losses, void* ws, const Workspace& L,
+                             cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e =
+        cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int NP = (s.E + 15) / 16 * 16;
+  CUtensorMap tx, tw;
+  if (!make_map(&tx, x, false, static_cast<uint64_t>(s.T), s.d, 64, kTile)) return cudaErrorInvalidValue;
+  if (!make_map(&tw, w_router, false, static_cast<uint64_t>(s.E), s.d, 64, NP)) return cudaErrorInvalidValue;
+  int32_t* ctrl = at<int32_t>(ws, L.ctrl);
+  cudaError_t e = cudaMemsetAsync(ctrl + 1, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return e;
+  RArgs a{};
+  a.T = s.T;
+  a.d = s.d;
+  a.E = s.E;
+  a.k = s.k;
+  a.NP = NP;
+  a.bias = bias;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.w = static_cast<const __nv_bfloat16*>(w_router);
+  a.idx_out = idx;
+  a.w_out = wts;
+  a.probs = at<float>(ws, L.probs);
+  a.lse_out = at<float>(ws, L.lse);
+  a.local_rank = at<int32_t>(ws, L.local_rank);
+  a.chunk_count = at<int32_t>(ws, L.chunk_count);
+  a.chunk_base = at<int32_t>(ws, L.chunk_base);
+  a.psum_part = at<float>(ws, L.psum_part);
+  a.zsum_part = at<double>(ws, L.zsum_part);
+  a.counts_ws = at<int32_t>(ws, L.counts);
+  a.counts_user = counts;
+  a.losses_ws = at<float>(ws, L.losses);
+  a.losses_user = losses;
+  a.offsets_ws = at<int32_t>(ws, L.offsets);
+  a.gs_ws = at<int32_t>(ws, L.group_start);
+  a.ticket = ctrl + 1;
+  a.status = ctrl;
+  const unsigned grid = static_cast<unsigned>((s.T + kTile - 1) / kTile);
+  router_tc_kernel<<<grid, kThreads, kSmem, st>>>(tx, tw, a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -37,7 +37,7 @@ INIT_STD = 0.02
 ALPHA_LB = 0.01
 BETA_Z = 0.001
 ZIPF_S = 1.2
-ZIPF_LAMBDA = 0.6  # replaced by the calibrated value below
+ZIPF_LAMBDA = 0.5599  # the 8 most favoured experts then take half the assignments
 RMS_EPS = 1e-5
 
 

@@ -95,6 +95,44 @@ def test_eight_experts_take_every_token():
     check_forward(inp, out, bias=bias)
 
 
+def _route_gpu_and_oracle(inp, bias=None):
+    out = run_forward(inp, bias=bias)
+    h = O.router_logits(f64(inp.x), f64(inp.w_router), None if bias is None else f64(bias))
+    p, _ = O.softmax_lse(h)
+    ref_idx, _ = O.topk_no_renorm(p, inp.shape.top_k)
+    return out["idx"].cpu().numpy(), ref_idx
+
+
+def test_router_breaks_exact_ties_by_lower_index():
+    """Experts 0..15 share one router row, so their logits are equal for every
+    token: the choice among them must go to the lower indices, on every token."""
+    sh = S.LayerShape(333, 512, 64, 8, 256)
+    inp = S.layer_inputs(sh, seed=31)
+    wr = inp.w_router.clone()
+    wr[1:16] = wr[0]
+    inp.w_router = wr
+    got, ref = _route_gpu_and_oracle(inp)
+    assert np.array_equal(got, ref)
+
+
+def test_router_orders_logits_one_ulp_apart():
+    """Odd experts copy the even expert's router row with one weight moved by one
+    bf16 ulp: their logits differ by ~1e-4, inside the fp32 uncertainty band the
+    router re-ranks with exact arithmetic, and the order must match on every token."""
+    sh = S.LayerShape(1000, 2048, 64, 8, 1024)
+    inp = S.layer_inputs(sh, seed=32)
+    wr = inp.w_router.clone()
+    g = torch.Generator().manual_seed(3)
+    for e in range(0, 64, 2):
+        row = wr[e].clone()
+        i = int(torch.randint(0, 2048, (1,), generator=g))
+        row.view(torch.int16)[i] += 1  # the next bf16 value (one ulp in magnitude)
+        wr[e + 1] = row
+    inp.w_router = wr
+    got, ref = _route_gpu_and_oracle(inp)
+    assert np.array_equal(got, ref)
+
+
 def test_olmoe_prefill_4096():
     """The OLMoE-shape layer: T=4096, d=2048, E=64, k=8, f=1024, bf16. Routing of
     every token; outputs on a sample of tokens (the first, the last, and 46 drawn)."""

@@ -119,6 +119,8 @@ def _bar(ref):
 GEMM_COUNTS = [
     [0, 1, 127, 128, 129, 300, 0, 5],
     [513, 0, 0, 2, 255, 256, 1, 64],
+    # >= 256 rows per expert on average: 256-row tiles, some with only one 128-row half
+    [700, 129, 384, 0, 255, 1, 513, 128],
 ]
 
 

@@ -349,3 +349,16 @@ def test_stack_with_zero_experts_is_identity_and_one_layer_is_one_block():
     r, _ = O.stack_forward(x0, [one], k=2)
     ref = x0 + O.moe_forward(O.rms_norm(x0), L["w_router"], L["w_gate_up"], L["w_down"], 2)["y"]
     assert np.allclose(r, ref, atol=1e-14, rtol=0)
+
+
+def test_zipf_offset_matches_its_calibration():
+    """The skewed stack's router offset gives the 8 most favoured experts half of
+    the assignments on layer 0's input (calibrated by tests/golden/calibrate_zipf.py)."""
+    vals = {r[0]: float(r[1]) for r in _read_table("zipf_lambda.txt")}
+    assert S.ZIPF_LAMBDA == vals["lambda"]
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("calibrate_zipf", os.path.join(GOLDEN, "calibrate_zipf.py"))
+    cal = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(cal)
+    x, wr = cal.layer0_inputs()
+    assert abs(cal.top8_share(S.ZIPF_LAMBDA, x, wr) - 0.5) <= 0.01
