@@ -193,6 +193,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmx);
       tma_prefetch_desc(&tmw);
       int issued = 0;
+      // CTAs walk K from different starting points so they do not all read the
+      // same router-weight tile of L2 at the same moment
+      const int k0 = static_cast<int>(blockIdx.x % static_cast<unsigned>(nk));
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % kStages;
         const uint32_t ph = static_cast<uint32_t>(kb / kStages) & 1u;
@@ -200,10 +203,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           report(a.status, DEV_WAIT_TIMEOUT_PRODUCER);
           break;
         }
+        const int kc = (kb + k0) % nk;
         unsigned char* st = ring + static_cast<size_t>(s) * STAGE;
         mbar_arrive_expect_tx(&full[s], STAGE);
-        tma_load_2d(&tmx, &full[s], st, kb * 64, static_cast<int32_t>(t0));
-        tma_load_2d(&tmw, &full[s], st + kAload, kb * 64, 0);
+        tma_load_2d(&tmx, &full[s], st, kc * 64, static_cast<int32_t>(t0));
+        tma_load_2d(&tmw, &full[s], st + kAload, kc * 64, 0);
         ++issued;
       }
       for (int s = 0; s < kStages && s < issued; ++s) {
@@ -301,11 +305,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (valid) a.lse_out[t] = lse;
     }
 
-    // ---- top (k+3) in fp32 by quad arg-max (uniform within the quad)
+    // ---- top (k+3) in fp32 by quad arg-max (uniform within the quad); nearm bit j
+    //      marks ranks j and j+1 as closer than the fp32 uncertainty
     const int nsel = min(k + 3, E);
     int ord[kMaxSel];
     float val[kMaxSel];
     uint32_t taken = 0;  // bit i: expert eb + i chosen
+    uint32_t nearm = 0;
 #pragma unroll
     for (int j = 0; j < kMaxSel; ++j) {
       if (j < nsel) {
@@ -322,21 +328,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (bi - eb >= 0 && bi - eb < 16) taken |= 1u << (bi - eb);
         ord[j] = bi;
         val[j] = v;
+        if (j > 0 && val[j - 1] - v < near_gap(val[j - 1])) nearm |= 1u << (j - 1);
       }
     }
-    float hv[kMaxSel];
+    float hv[kMaxSel];  // fp32 logit of ord[j], kept for the weights
 #pragma unroll
     for (int j = 0; j < kMaxSel; ++j) hv[j] = val[j];
-    // runs of near-equal neighbours that decide a slot order or the k-th choice
+    // Slow path (rare): some run of near-equal neighbours decides a slot order or
+    // the k-th choice. It works on local copies so the common path stays in registers.
+    const bool slow = valid && (nearm & ((1u << k) - 1u)) != 0;
     bool fallback = false;
     int run_a[kMaxSel], run_b[kMaxSel];
     int nrun = 0;
-    if (valid) {
+    int oloc[kMaxSel];
+    float hloc[kMaxSel];
+    if (slow) {
+#pragma unroll
+      for (int j = 0; j < kMaxSel; ++j) {
+        oloc[j] = ord[j];
+        hloc[j] = hv[j];
+      }
       int jj = 0;
       while (jj < nsel - 1) {
-        if (val[jj] - val[jj + 1] < near_gap(val[jj])) {
+        if ((nearm >> jj) & 1u) {
           int b = jj + 1;
-          while (b < nsel - 1 && val[b] - val[b + 1] < near_gap(val[b])) ++b;
+          while (b < nsel - 1 && ((nearm >> b) & 1u)) ++b;
           if (jj <= k - 1) {
             if (b == nsel - 1 && nsel < E) {
               fallback = true;
@@ -364,11 +380,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     qbase = __shfl_sync(qm, qbase, lane & ~3);
     if (fallback) {
       for (int e = qp; e < E; e += 4) queue[qbase + e] = (static_cast<uint32_t>(r) << 8) | static_cast<uint32_t>(e);
-    } else {
+    } else if (nrun > 0) {
       int p = 0;
       for (int i = 0; i < nrun; ++i)
         for (int y = run_a[i]; y <= run_b[i]; ++y, ++p)
-          if ((p & 3) == qp) queue[qbase + p] = (static_cast<uint32_t>(r) << 8) | static_cast<uint32_t>(ord[y]);
+          if ((p & 3) == qp) queue[qbase + p] = (static_cast<uint32_t>(r) << 8) | static_cast<uint32_t>(oloc[y]);
     }
     epi_sync();
     // ---- exact logits of the queued pairs: a warp per pair, all loads in flight together
@@ -383,72 +399,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     epi_sync();
-    // ---- re-rank each run by its exact logits (ties: lower expert index)
-    if (!fallback && nrun > 0) {
-      int p = qbase;
-      for (int i = 0; i < nrun; ++i) {
-        const int ra = run_a[i], rb = run_b[i];
-        double ex[kMaxSel];
-        for (int y = ra; y <= rb; ++y) ex[y] = exact[p++];
-        for (int x1 = ra + 1; x1 <= rb; ++x1) {
-          const double ve = ex[x1];
-          const int oe = ord[x1];
-          const float he = hv[x1];
-          int y = x1 - 1;
-          while (y >= ra && (ex[y] < ve || (ex[y] == ve && ord[y] > oe))) {
-            ex[y + 1] = ex[y];
-            ord[y + 1] = ord[y];
-            hv[y + 1] = hv[y];
-            --y;
+    if (slow) {
+      if (!fallback) {  // re-rank each run by its exact logits (ties: lower expert index)
+        int p = qbase;
+        for (int i = 0; i < nrun; ++i) {
+          const int ra = run_a[i], rb = run_b[i];
+          double ex[kMaxSel];
+          for (int y = ra; y <= rb; ++y) ex[y] = exact[p++];
+          for (int x1 = ra + 1; x1 <= rb; ++x1) {
+            const double ve = ex[x1];
+            const int oe = oloc[x1];
+            const float he = hloc[x1];
+            int y = x1 - 1;
+            while (y >= ra && (ex[y] < ve || (ex[y] == ve && oloc[y] > oe))) {
+              ex[y + 1] = ex[y];
+              oloc[y + 1] = oloc[y];
+              hloc[y + 1] = hloc[y];
+              --y;
+            }
+            ex[y + 1] = ve;
+            oloc[y + 1] = oe;
+            hloc[y + 1] = he;
           }
-          ex[y + 1] = ve;
-          ord[y + 1] = oe;
-          hv[y + 1] = he;
+        }
+      } else {  // a run reaches past rank k+3: rank every expert by its exact logit
+        double xe[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xe[i] = (eb + i < E) ? exact[qbase + eb + i] : -INFINITY;
+        uint32_t tk = 0;
+        for (int j = 0; j < k; ++j) {
+          double v = -INFINITY;
+          int bi = 0x7fffffff;
+          float hb = 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (eb + i < E && !((tk >> i) & 1u) && (bi == 0x7fffffff || xe[i] > v)) {
+              v = xe[i];
+              bi = eb + i;
+              hb = h[i];
+            }
+          }
+          quad_argmax(v, bi);
+          if (bi - eb >= 0 && bi - eb < 16) tk |= 1u << (bi - eb);
+          oloc[j] = bi;
+          // the fp32 logit of the winner, from the thread that holds it
+          const int owner = (lane & ~3) | ((bi >> 4) & 3);
+          hloc[j] = __shfl_sync(qm, (bi >= eb && bi < eb + 16) ? hb : 0.f, owner);
         }
       }
-    }
-    if (fallback) {  // a run reaches past rank k+3: rank every expert by its exact logit
-      double xe[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) xe[i] = (eb + i < E) ? exact[qbase + eb + i] : -INFINITY;
-      uint32_t tk = 0;
-      for (int j = 0; j < k; ++j) {
-        double v = -INFINITY;
-        int bi = 0x7fffffff;
-        float hb = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (eb + i < E && !((tk >> i) & 1u) && (bi == 0x7fffffff || xe[i] > v)) {
-            v = xe[i];
-            bi = eb + i;
-            hb = h[i];
-          }
-        }
-        quad_argmax(v, bi);
-        if (bi - eb >= 0 && bi - eb < 16) tk |= 1u << (bi - eb);
-        ord[j] = bi;
-        // the fp32 logit of the winner, from the thread that holds it
-        const float mine = hb;
-        const int owner = (lane & ~3) | ((bi >> 4) & 3);
-        hv[j] = __shfl_sync(qm, (bi >= eb && bi < eb + 16) ? mine : 0.f, owner);
+      for (int j = 0; j < kMaxSel; ++j) {
+        ord[j] = oloc[j];
+        hv[j] = hloc[j];
       }
     }
     // ---- outputs: thread qp writes slots qp, qp+4, ...
     if (valid) {
-      for (int j = qp; j < k; j += 4) {
-        const int e = ord[j];
-        a.idx_out[t * k + j] = e;
-        a.w_out[t * k + j] = expf(hv[j] - m) / s;
-        chosen[r * kMaxTopK + j] = e;
-        atomicOr(&mask[e], 1u << r);
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        if (j < k && (j & 3) == qp) {
+          const int e = ord[j];
+          a.idx_out[t * k + j] = e;
+          a.w_out[t * k + j] = expf(hv[j] - m) / s;
+          chosen[r * kMaxTopK + j] = e;
+          atomicOr(&mask[e], 1u << r);
+        }
       }
     }
     epi_sync();
     // ---- ranks inside the chunk and per-CTA partials
     if (valid) {
-      for (int j = qp; j < k; j += 4) {
-        const int e = chosen[r * kMaxTopK + j];
-        a.local_rank[t * k + j] = __popc(mask[e] & ((1u << r) - 1u));
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        if (j < k && (j & 3) == qp) {
+          const int e = ord[j];
+          a.local_rank[t * k + j] = __popc(mask[e] & ((1u << r) - 1u));
+        }
       }
     }
     const int cta = blockIdx.x;
@@ -508,10 +534,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         epi_sync();
-        if (tid < E) {
-          for (int c = 0; c < nc; ++c) {
+        if (tid < E) {  // eight chunks' loads in flight, then the running sums in order
+          int c = 0;
+          for (; c + 8 <= nc; c += 8) {
+            int v[8];
+            float q[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+              v[b] = cnt_s[(c + b) * E + tid];
+              q[b] = ps_s[(c + b) * E + tid];
+            }
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+              cnt_s[(c + b) * E + tid] = run;  // becomes the chunk base
+              run += v[b];
+              pe += static_cast<double>(q[b]);
+            }
+          }
+          for (; c < nc; ++c) {
             const int v = cnt_s[c * E + tid];
-            cnt_s[c * E + tid] = run;  // becomes the chunk base
+            cnt_s[c * E + tid] = run;
             run += v;
             pe += static_cast<double>(ps_s[c * E + tid]);
           }
@@ -534,30 +576,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         zred[tid] = z;
       }
       epi_sync();
-      if (tid == 0) {
-        double zt = 0.0;
-        for (int i = 0; i < 128; ++i) zt += zred[i];
-        int off = 0, gsv = 0;
-        double lb = 0.0;
-        const double Td = static_cast<double>(a.T);
-        for (int e = 0; e < E; ++e) {
-          a.offsets_ws[e] = off;
-          a.gs_ws[e] = gsv;
-          off += tot[e];
-          gsv += (tot[e] + kRowAlign - 1) / kRowAlign * kRowAlign;
-          lb += (static_cast<double>(tot[e]) / (Td * k)) * (tot_p[e] / Td);
+      if (warp == 2) {
+        // warp-wide finalisation (E <= 64): lane holds experts lane and lane + 32.
+        // Group starts and offsets are exclusive prefix sums; the two loss sums use a
+        // fixed butterfly order, so every lane ends with the same bits on every run.
+        const int e0 = lane, e1 = lane + 32;
+        const int c0v = e0 < E ? tot[e0] : 0, c1v = e1 < E ? tot[e1] : 0;
+        const int g0v = (c0v + kRowAlign - 1) / kRowAlign * kRowAlign;
+        const int g1v = (c1v + kRowAlign - 1) / kRowAlign * kRowAlign;
+        int ic0 = c0v, ig0 = g0v, ic1 = c1v, ig1 = g1v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u0 = __shfl_up_sync(0xffffffffu, ic0, o), w0 = __shfl_up_sync(0xffffffffu, ig0, o);
+          const int u1 = __shfl_up_sync(0xffffffffu, ic1, o), w1 = __shfl_up_sync(0xffffffffu, ig1, o);
+          if (lane >= o) {
+            ic0 += u0;
+            ig0 += w0;
+            ic1 += u1;
+            ig1 += w1;
+          }
         }
-        a.offsets_ws[E] = off;
-        a.gs_ws[E] = gsv;
-        const float l0 = static_cast<float>(lb * E), l1 = static_cast<float>(zt / Td);
-        a.losses_ws[0] = l0;
-        a.losses_ws[1] = l1;
-        if (a.losses_user != nullptr) {
-          a.losses_user[0] = l0;
-          a.losses_user[1] = l1;
+        const int tc0 = __shfl_sync(0xffffffffu, ic0, 31), tg0 = __shfl_sync(0xffffffffu, ig0, 31);
+        const int tc1 = __shfl_sync(0xffffffffu, ic1, 31), tg1 = __shfl_sync(0xffffffffu, ig1, 31);
+        if (e0 < E) {
+          a.offsets_ws[e0] = ic0 - c0v;
+          a.gs_ws[e0] = ig0 - g0v;
         }
-        if (static_cast<int64_t>(off) != a.T * k) report(a.status, DEV_COUNT_MISMATCH);
-        *a.ticket = 0;
+        if (e1 < E) {
+          a.offsets_ws[e1] = tc0 + ic1 - c1v;
+          a.gs_ws[e1] = tg0 + ig1 - g1v;
+        }
+        // load balance: E * sum_e (c_e / (T k)) (P_e / T) = E * sum_e c_e P_e / (T^2 k)
+        double lb = (e0 < E ? static_cast<double>(c0v) * tot_p[e0] : 0.0) +
+                    (e1 < E ? static_cast<double>(c1v) * tot_p[e1] : 0.0);
+        double zt = ((zred[4 * lane] + zred[4 * lane + 1]) + zred[4 * lane + 2]) + zred[4 * lane + 3];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          lb += __shfl_xor_sync(0xffffffffu, lb, o);
+          zt += __shfl_xor_sync(0xffffffffu, zt, o);
+        }
+        if (lane == 0) {
+          const int off = tc0 + tc1;
+          a.offsets_ws[E] = off;
+          a.gs_ws[E] = tg0 + tg1;
+          const double Td = static_cast<double>(a.T);
+          const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(zt / Td);
+          a.losses_ws[0] = l0;
+          a.losses_ws[1] = l1;
+          if (a.losses_user != nullptr) {
+            a.losses_user[0] = l0;
+            a.losses_user[1] = l1;
+          }
+          if (static_cast<int64_t>(off) != a.T * k) report(a.status, DEV_COUNT_MISMATCH);
+          *a.ticket = 0;
+        }
       }
     }
   }
