@@ -60,6 +60,8 @@ __all__ = [
     "moe_forward",
     "moe_objective",
     "moe_backward",
+    "token_input_grads",
+    "expert_weight_grad_slices",
     "rms_norm",
     "stack_forward",
 ]
@@ -382,6 +384,89 @@ def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias
         "dh": dh,
         "fwd": fwd,
     }
+
+
+def token_input_grads(x_rows, w_router, w_gate_up, w_down, k, dy_rows, alpha, beta, counts, n_tokens,
+                      router_bias=None):
+    """dx for some of the tokens of a batch, one token at a time.
+
+    Every step of the chain rule in moe_backward acts on one token alone except
+    the load-balance term, whose derivative with respect to p_ti is
+    alpha * E * f_i / T: it needs only the batch's counts (f_i = count_i / (T k))
+    and its size T = `n_tokens`. Given those, the rows `x_rows` (any subset of
+    the batch, with their upstream gradients `dy_rows`) get exactly the dx rows
+    moe_backward gives them. Returns dx [n, d].
+    """
+    x = _f64(x_rows)
+    dy = _f64(dy_rows)
+    w_r = _f64(w_router)
+    n_experts = w_r.shape[0]
+    f = _f64(w_down[0]).shape[1]
+    h = router_logits(x, w_r, router_bias)
+    p, lse = softmax_lse(h)
+    idx, w = topk_no_renorm(p, k)
+    n = x.shape[0]
+    dx = np.zeros_like(x)
+    dp = np.zeros((n, n_experts))
+    for t in range(n):
+        for j in range(k):
+            e = int(idx[t, j])
+            wgu = _f64(w_gate_up[e])
+            wd = _f64(w_down[e])
+            a = wgu[:f] @ x[t]
+            b = wgu[f:] @ x[t]
+            sig = 1.0 / (1.0 + np.exp(-a))
+            g = a * sig * b
+            dp[t, e] += dy[t] @ (wd @ g)        # dw_tj = <dy_t, o_tj>
+            dg = wd.T @ (w[t, j] * dy[t])       # do_tj = w_tj dy_t
+            da = dg * b * (sig * (1.0 + a * (1.0 - sig)))
+            db = dg * (a * sig)
+            dx[t] += wgu[:f].T @ da + wgu[f:].T @ db
+    frac = np.asarray(counts, dtype=np.float64) / float(n_tokens * k)
+    dp += alpha * n_experts * frac[None, :] / n_tokens
+    dh = p * (dp - np.sum(dp * p, axis=1, keepdims=True))
+    dh += beta * (2.0 * lse / n_tokens)[:, None] * p
+    return dx + dh @ w_r
+
+
+def expert_weight_grad_slices(x, idx, w, dy, w_gate_up_e, w_down_e, e, gate_up_rows, down_cols):
+    """Chosen rows of dW_gate_up,e and chosen columns of dW_down,e.
+
+    Same formulas as moe_backward (dW_gate_up,e = sum over e's rows of [da; db] x^T,
+    dW_down,e = sum over e's rows of do g^T), restricted so that only the named
+    hidden units are evaluated: row j < f of dW_gate_up needs a_j, b_j and dg_j of
+    every row routed to e; row f + j the same; column c of dW_down needs g_c.
+    `x`, `idx`, `w`, `dy` are the whole batch's. Returns (rows [len, d], cols [d, len]).
+    """
+    x = _f64(x)
+    dy = _f64(dy)
+    idx = np.asarray(idx)
+    w = _f64(w)
+    wgu = _f64(w_gate_up_e)
+    wd = _f64(w_down_e)
+    f = wd.shape[1]
+    tok, slot = np.nonzero(idx == e)
+    xr = x[tok]
+    do = w[tok, slot][:, None] * dy[tok]
+
+    def unit(j):
+        a = xr @ wgu[j]
+        b = xr @ wgu[f + j]
+        sig = 1.0 / (1.0 + np.exp(-a))
+        return a, b, sig
+
+    rows = []
+    for r in gate_up_rows:
+        j = int(r) % f
+        a, b, sig = unit(j)
+        dg = do @ wd[:, j]
+        coef = dg * b * (sig * (1.0 + a * (1.0 - sig))) if int(r) < f else dg * (a * sig)
+        rows.append(coef @ xr)
+    cols = []
+    for c in down_cols:
+        a, b, sig = unit(int(c))
+        cols.append(do.T @ (a * sig * b))
+    return np.array(rows).reshape(len(rows), x.shape[1]), np.array(cols).T.reshape(wd.shape[0], len(cols))
 
 
 # --------------------------------------------------------------------------- stack

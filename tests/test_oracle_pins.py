@@ -326,6 +326,31 @@ def test_backward_expert_subset_matches_full():
     assert np.array_equal(part["dx"], full["dx"])
 
 
+def test_token_subset_input_grads_match_the_batch():
+    """dx of a few tokens, given only the batch's counts and size, equals those
+    rows of the batch backward (itself pinned by finite differences above); a
+    dropped load-balance or z term, or the wrong T, would show here."""
+    L = _small_layer(20, T=14, d=16, E=8, k=3, f=6, std=0.4)
+    dy = _rng(21).standard_normal((14, 16))
+    full = O.moe_backward(dy=dy, alpha=0.7, beta=0.3, **L)
+    rows = [0, 5, 13]
+    dx = O.token_input_grads(L["x"][rows], L["w_router"], L["w_gate_up"], L["w_down"], L["k"], dy[rows],
+                             0.7, 0.3, full["fwd"]["counts"], 14)
+    assert np.abs(dx - full["dx"][rows]).max() < 1e-12
+
+
+def test_expert_weight_grad_slices_match_the_batch():
+    L = _small_layer(22, T=20, d=16, E=8, k=3, f=6)
+    dy = _rng(23).standard_normal((20, 16))
+    full = O.moe_backward(dy=dy, alpha=0.01, beta=0.001, **L)
+    fw = full["fwd"]
+    for e in (0, 3):
+        rows, cols = O.expert_weight_grad_slices(L["x"], fw["idx"], fw["w"], dy, L["w_gate_up"][e],
+                                                 L["w_down"][e], e, gate_up_rows=[0, 4, 6, 11], down_cols=[1, 5])
+        assert np.abs(rows - full["dw_gate_up"][e][[0, 4, 6, 11]]).max() < 1e-12
+        assert np.abs(cols - full["dw_down"][e][:, [1, 5]]).max() < 1e-12
+
+
 # ------------------------------------------------------------------ stack
 
 
