@@ -34,6 +34,15 @@ the design notes):
     the backward objective  <dy, y> + alpha * L_lb + beta * L_z.
   * No gradient flows through the expert choice or through f ([OLMoE-Guide]
     computes f with bincount, a count).
+  * Storage precision (optional `store` argument of the expert functions,
+    moe_forward and moe_backward): the pages fix no precision for the expert
+    activations. By default nothing is rounded. Given a rounding function,
+    every activation a bf16 implementation keeps between two contractions is
+    passed through it (the SwiGLU output h, the expert output o, and in the
+    backward the saved pre-activations a and b, do = w dy and [da; db]); all
+    arithmetic stays fp64. This states what an implementation with bf16
+    storage computes, so a gradient that sums many such rounded terms can be
+    compared at the bar it should meet.
 
 Parity pins for every function live in tests/test_oracle_pins.py.
 """
@@ -213,18 +222,23 @@ def expert_down(g_rows, w_down_e):
     return _f64(g_rows) @ _f64(w_down_e).T
 
 
-def swiglu_expert(x_rows, w_gate_up_e, w_down_e):
+def _store(store):
+    return (lambda v: v) if store is None else (lambda v: _f64(store(v)))
+
+
+def swiglu_expert(x_rows, w_gate_up_e, w_down_e, store=None):
     """One SwiGLU expert on a block of rows.
 
     [OLMoE-Guide] "Top-8 Softmax Routing Formulation": Expert_i(x) =
     (Swish(x W_gate) * (x W_up)) W_down. [MoE-scratch] §2 `Experts` stores the
     gate rows first, then the up rows, in one (2f, d) matrix, and the down
-    projection as (d, f).
+    projection as (d, f). `store` (see the module notes) rounds h and o.
     """
-    return expert_down(swiglu_hidden(x_rows, w_gate_up_e), w_down_e)
+    S = _store(store)
+    return S(expert_down(S(swiglu_hidden(x_rows, w_gate_up_e)), w_down_e))
 
 
-def experts_grouped(x, idx, w, w_gate_up, w_down):
+def experts_grouped(x, idx, w, w_gate_up, w_down, store=None):
     """y_t = sum_j w_tj * Expert_{S_tj}(x_t), computed group by group.
 
     [MoE-scratch] §2 `dispatch`: sort the pairs by expert, run each expert once on
@@ -242,7 +256,7 @@ def experts_grouped(x, idx, w, w_gate_up, w_down):
         if sel.size == 0:
             continue
         tok = sel // k
-        out = swiglu_expert(x[tok], w_gate_up[e], w_down[e])
+        out = swiglu_expert(x[tok], w_gate_up[e], w_down[e], store)
         # Each token chooses an expert at most once, so `tok` has no repeats.
         y[tok] += w.reshape(-1)[sel][:, None] * out
     return y
@@ -269,7 +283,7 @@ def experts_dense(x, idx, w, w_gate_up, w_down):
 # --------------------------------------------------------------------------- layer
 
 
-def moe_forward(x, w_router, w_gate_up, w_down, k, router_bias=None):
+def moe_forward(x, w_router, w_gate_up, w_down, k, router_bias=None, store=None):
     """The whole layer: route, dispatch, experts, combine, and the two losses.
 
     Returns a dict with
@@ -280,7 +294,7 @@ def moe_forward(x, w_router, w_gate_up, w_down, k, router_bias=None):
     h = router_logits(x, w_router, router_bias)
     p, lse = softmax_lse(h)
     idx, w = topk_no_renorm(p, k)
-    y = experts_grouped(x, idx, w, w_gate_up, w_down)
+    y = experts_grouped(x, idx, w, w_gate_up, w_down, store)
     L_lb, counts = load_balance_loss(idx, p, n_experts)
     perm, _, offsets = dispatch_order(idx, n_experts)
     return {
@@ -311,7 +325,7 @@ def moe_objective(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bia
 
 
 def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias=None,
-                 experts=None):
+                 experts=None, store=None):
     """Gradients of moe_objective with respect to x and the three weights.
 
     Chain rule through each step of moe_forward (f and the choice carry none):
@@ -324,13 +338,15 @@ def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias
                     dh_t  = p_t * (dp_t - <dp_t, p_t>) + beta * (2 lse_t / T) * p_t
       router        dW_r = sum_t dh_t x_t^T,   dx_t += W_r^T dh_t
     `experts` optionally restricts which experts' weight gradients are formed
-    (the rest are left zero); dx and dW_r always use every expert.
+    (the rest are left zero); dx and dW_r always use every expert. `store`
+    (see the module notes) rounds h, o, the saved a and b, do and [da; db].
     Returns dict dx [T,d], dw_router [E,d], dw_gate_up [E,2f,d], dw_down [E,d,f],
     plus the forward dict under "fwd" and dw [T,k].
     """
     x = _f64(x)
     dy = _f64(dy)
-    fwd = moe_forward(x, w_router, w_gate_up, w_down, k, router_bias)
+    S = _store(store)
+    fwd = moe_forward(x, w_router, w_gate_up, w_down, k, router_bias, store)
     idx, w, p, lse = fwd["idx"], fwd["w"], fwd["p"], fwd["lse"]
     T, d = x.shape
     n_experts = _f64(w_router).shape[0]
@@ -354,13 +370,17 @@ def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias
         b = xr @ wgu[f:].T
         with np.errstate(over="ignore"):
             sig = 1.0 / (1.0 + np.exp(-a))
-        g = a * sig * b
-        o = g @ wd.T
+        g = S(a * sig * b)
+        o = S(g @ wd.T)
         dw.reshape(-1)[sel] = np.sum(dy[tok] * o, axis=1)
-        do = w.reshape(-1)[sel][:, None] * dy[tok]
+        do = S(w.reshape(-1)[sel][:, None] * dy[tok])
         dg = do @ wd
-        da = dg * b * (sig * (1.0 + a * (1.0 - sig)))
-        db = dg * (a * sig)
+        if store is not None:  # the derivative reads the stored pre-activations
+            a, b = S(a), S(b)
+            with np.errstate(over="ignore"):
+                sig = 1.0 / (1.0 + np.exp(-a))
+        da = S(dg * b * (sig * (1.0 + a * (1.0 - sig))))
+        db = S(dg * (a * sig))
         if e in want:
             dw_down[e] = do.T @ g
             dw_gate_up[e, :f] = da.T @ xr

@@ -351,6 +351,49 @@ def test_expert_weight_grad_slices_match_the_batch():
         assert np.abs(cols - full["dw_down"][e][:, [1, 5]]).max() < 1e-12
 
 
+# ------------------------------------------------------------------ storage rounding
+
+
+def test_store_identity_changes_nothing_and_zero_store_removes_the_experts():
+    L = _small_layer(24, T=12, d=16, E=8, k=3, f=6, std=0.4)
+    dy = _rng(25).standard_normal((12, 16))
+    plain = O.moe_backward(dy=dy, alpha=0.3, beta=0.2, **L)
+    ident = O.moe_backward(dy=dy, alpha=0.3, beta=0.2, store=lambda v: v, **L)
+    for key in ("dx", "dw_router", "dw_gate_up", "dw_down"):
+        assert np.array_equal(plain[key], ident[key]), key
+    assert np.array_equal(plain["fwd"]["y"], ident["fwd"]["y"])
+    # a store that zeroes every activation silences the experts: y = 0, and the
+    # gradient is that of the two losses alone (the same as dy = 0)
+    zero = O.moe_backward(dy=dy, alpha=0.3, beta=0.2, store=lambda v: 0.0 * v, **L)
+    loss_only = O.moe_backward(dy=np.zeros_like(dy), alpha=0.3, beta=0.2, **L)
+    assert np.all(zero["fwd"]["y"] == 0)
+    assert np.allclose(zero["dx"], loss_only["dx"], atol=1e-15, rtol=0)
+    assert np.allclose(zero["dw_router"], loss_only["dw_router"], atol=1e-15, rtol=0)
+    assert np.all(zero["dw_gate_up"] == 0) and np.all(zero["dw_down"] == 0)
+
+
+def test_store_rounding_on_a_two_expert_scalar_layer():
+    """d = f = 1, two experts, k = 1, rounding to multiples of 1/8. By hand:
+    h = [0.3, -0.2] so expert 0 wins with p0 = 1 / (1 + e^-0.5); its hidden
+    silu(0.7) * 1.3 = 0.608 is stored as 0.625, its output 0.8 * 0.625 = 0.5 is
+    exact; y = p0 * 0.5. With dy = 1 and no loss terms, dw = <dy, o> = 0.5, so
+    dh = [0.5 p0 p1, -0.5 p0 p1] and dW_r = dh x with x = 1; do = p0 is stored
+    as 0.625, so dW_down = 0.625 * 0.625."""
+    R = lambda v: np.round(np.asarray(v) * 8.0) / 8.0
+    x = np.array([[1.0]])
+    w_router = np.array([[0.3], [-0.2]])
+    w_gate_up = np.array([[[0.7], [1.3]], [[0.5], [0.5]]])
+    w_down = np.array([[[0.8]], [[0.5]]])
+    g = O.moe_backward(x, w_router, w_gate_up, w_down, 1, np.array([[1.0]]), 0.0, 0.0, store=R)
+    p0 = 1.0 / (1.0 + math.exp(-0.5))
+    p1 = 1.0 - p0
+    assert g["fwd"]["idx"][0, 0] == 0
+    assert abs(g["fwd"]["y"][0, 0] - p0 * 0.5) < 1e-15
+    assert abs(g["dw"][0, 0] - 0.5) < 1e-15
+    assert np.allclose(g["dw_router"][:, 0], [0.5 * p0 * p1, -0.5 * p0 * p1], atol=1e-15, rtol=0)
+    assert abs(g["dw_down"][0, 0, 0] - 0.625 * 0.625) < 1e-15
+
+
 # ------------------------------------------------------------------ stack
 
 
