@@ -11,6 +11,11 @@ every step exceed the 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
 
+At N=1 the line also carries the other OLMoE-shape workloads, each timed on
+the device: "decode" (T = 1, 8, 32, 64; CUDA-graph replays with the L2 flushed
+before each, HBM GB/s of the touched experts' weights), "train" (T = 16384
+forward + backward) and "stack" (16 layers, T = 8192, Zipf-skewed routing).
+
 N > 1 runs as torchrun, one process per GPU, each on its own batch (weak
 scaling, no data-path collective); the device time is the max over ranks and
 `value` counts the tokens of all ranks. `--impl reference` times the fp64 CPU
@@ -41,7 +46,9 @@ WORKLOAD = "OLMoE MoE layer forward, T=4096 (1x4096 context), d_model=2048, E=64
 NOMINAL_BF16_TFLOPS = 2250.0
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 6  # router, dispatch rank, dispatch permute, gate/up GEMM, down GEMM, combine
+# router (which also ranks the dispatch), dispatch permute, gate/up GEMM, down GEMM,
+# combine; plus one memset of the router's ticket word (not a kernel)
+KERNELS_PER_STEP = 5
 
 
 # ----------------------------------------------------------------------------- shapes
@@ -267,6 +274,163 @@ def run_reference(args, rank, world):
 # ----------------------------------------------------------------------------- B200 leg
 
 
+def _percentiles(xs):
+    xs = sorted(xs)
+    q = lambda f: xs[min(len(xs) - 1, int(f * (len(xs) - 1) + 0.5))]
+    return statistics.median(xs), q(0.1), q(0.9)
+
+
+def bench_decode(M, S, dev, weights, reps, peaks):
+    """Decode-shaped layers (T = 1, 8, 32, 64): the forward captured in a CUDA
+    graph and replayed, the L2 flushed before every replay so the touched
+    experts' weights come from HBM. Algorithmic bytes: the touched experts'
+    weights, the router weight, x, y and the top-k outputs."""
+    import torch
+    wr, wgu, wd = weights
+    E, d = wr.shape
+    f = wd.shape[2]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = {}
+    for T in S.DECODE_TOKENS:
+        k = S.OLMOE_TOP_K
+        x = S.make_tokens(S.LayerShape(T=T), seed=700 + T).to(dev)
+        cfg = M.config(T, d, E, k, f)
+        ws = M.workspace(cfg, False, dev)
+        y = torch.empty_like(x)
+        losses = torch.empty(2, device=dev)
+        idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        wts = torch.empty(T, k, device=dev)
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            M.moe_forward(cfg, x, wr, None, wgu, wd, y, losses, idx, wts, False, ws)
+            torch.cuda.synchronize(dev)
+            with torch.cuda.graph(graph, stream=side):
+                M.moe_forward(cfg, x, wr, None, wgu, wd, y, losses, idx, wts, False, ws)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        for _ in range(5):
+            flush.zero_()
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record()
+            graph.replay()
+            b.record()
+        torch.cuda.synchronize(dev)
+        us = [a.elapsed_time(b) * 1e3 for a, b in evs]
+        med, p10, p90 = _percentiles(us)
+        touched = int(torch.unique(idx).numel())
+        nbytes = touched * 3 * d * f * 2 + E * d * 2 + 2 * T * d * 2 + T * k * 8
+        gbs = nbytes / (med * 1e-6) / 1e9
+        status = M.moe_get_device_status(ws)
+        if status != 0:
+            raise RuntimeError(f"device check failed in the decode runs: 0x{status:x}")
+        del graph
+        out[f"T{T}"] = {
+            "us_median": med, "us_p10": p10, "us_p90": p90, "replays": reps, "experts_touched": touched,
+            "bytes": nbytes, "GB_per_s": gbs, "frac_of_8TBs": gbs / NOMINAL_HBM_GBS,
+            "frac_of_measured_hbm": gbs / peaks["hbm_gbs"], "tokens_per_s": T / (med * 1e-6),
+        }
+    out["timing"] = "CUDA-graph replay of moe_forward, L2 flushed (256 MB write) before each replay"
+    return out
+
+
+def bench_train(M, S, dev, steps, peaks):
+    """One training step at T = 16384: moe_forward (saving for backward) and
+    moe_backward, with the OLMoE loss weights, an N(0, 1) upstream gradient and
+    fp32 weight gradients."""
+    import torch
+    sh = S.TRAIN_16384
+    inp = S.layer_inputs(sh, seed=3, with_grad=True)
+    T, d, E, k, f = sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff
+    x, wr, wgu, wd, dy = (t.to(dev) for t in (inp.x, inp.w_router, inp.w_gate_up, inp.w_down, inp.dy))
+    del inp
+    cfg = M.config(T, d, E, k, f, alpha_lb=S.ALPHA_LB, beta_z=S.BETA_Z, grad_dtype=torch.float32)
+    ws = M.workspace(cfg, True, dev)
+    y = torch.empty_like(x)
+    losses = torch.empty(2, device=dev)
+    dx = torch.empty_like(x)
+    dwr, dwgu, dwd = (torch.empty_like(t, dtype=torch.float32) for t in (wr, wgu, wd))
+
+    def fwd():
+        M.moe_forward(cfg, x, wr, None, wgu, wd, y, losses, None, None, True, ws)
+
+    def bwd():
+        M.moe_backward(cfg, dy, x, wr, wgu, wd, dx, dwr, dwgu, dwd, ws)
+
+    for _ in range(3):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e0, e1, e2 in evs:
+        e0.record()
+        fwd()
+        e1.record()
+        bwd()
+        e2.record()
+    torch.cuda.synchronize(dev)
+    status = M.moe_get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device check failed in the training step: 0x{status:x}")
+    f_ms = statistics.median(a.elapsed_time(b) for a, b, _ in evs)
+    b_ms = statistics.median(b.elapsed_time(c) for _, b, c in evs)
+    s_ms = statistics.median(a.elapsed_time(c) for a, _, c in evs)
+    fl_fwd = layer_flops_per_token(d, E, k, f) * T
+    # backward: twice the expert forward (data and weight gradients) plus the
+    # router's two products (dx += dh W_r and dW_r = dh^T x)
+    fl_bwd = 2.0 * k * (6 * d * f) * T + 4.0 * T * d * E
+    peak = peaks["bf16_tflops"]
+    return {
+        "T": T, "ms_forward": f_ms, "ms_backward": b_ms, "ms_step": s_ms, "steps": steps,
+        "tokens_per_s": T / (s_ms * 1e-3),
+        "tflops_step": (fl_fwd + fl_bwd) / (s_ms * 1e-3) / 1e12,
+        "tflops_forward": fl_fwd / (f_ms * 1e-3) / 1e12, "tflops_backward": fl_bwd / (b_ms * 1e-3) / 1e12,
+        "frac_of_2250TF": (fl_fwd + fl_bwd) / (s_ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS,
+        "frac_of_measured_bf16": (fl_fwd + fl_bwd) / (s_ms * 1e-3) / 1e12 / peak,
+        "flops_step": fl_fwd + fl_bwd, "weight_grads": "fp32",
+    }
+
+
+def bench_stack(M, S, dev, steps, peaks):
+    """The 16-layer skewed stack at T = 8192 (pre-RMSNorm, fp32 residual, Zipf
+    router offset), each step from the same input residual."""
+    import torch
+    sh = S.STACK_8192
+    T, d, E, k, f = sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff
+    x0, layers = S.stack_inputs(sh, S.STACK_LAYERS, seed=8)
+    x0 = x0.to(dev)
+    layers = [{n: (v.to(dev) if v is not None else None) for n, v in L.items()} for L in layers]
+    cfg = M.config(T, d, E, k, f)
+    ws = M.workspace(cfg, False, dev)
+    resid = torch.empty_like(x0)
+    for _ in range(3):
+        resid.copy_(x0)
+        M.moe_stack_forward(cfg, layers, resid, ws)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        resid.copy_(x0)
+        a.record()
+        M.moe_stack_forward(cfg, layers, resid, ws)
+        b.record()
+    torch.cuda.synchronize(dev)
+    status = M.moe_get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device check failed in the stack: 0x{status:x}")
+    ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    flops = S.STACK_LAYERS * layer_flops_per_token(d, E, k, f) * T
+    return {
+        "T": T, "layers": S.STACK_LAYERS, "ms": ms, "steps": steps, "tokens_per_s": T / (ms * 1e-3),
+        "tflops": flops / (ms * 1e-3) / 1e12, "frac_of_2250TF": flops / (ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS,
+        "frac_of_measured_bf16": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "flops": flops,
+    }
+
+
 def run_b200(args, rank, world, local):
     import torch
     import sparse_moe_transformer_route_b200 as M
@@ -387,6 +551,14 @@ def run_b200(args, rank, world, local):
         "gpu_launches": KERNELS_PER_STEP * K,
         "clocks": clocks,
     }
+    if world == 1 and not args.no_extras:
+        # the other OLMoE-shape workloads on this GPU, each reported beside the headline
+        line["decode"] = bench_decode(M, S, dev, (wr, wgu, wd), 200, peaks)
+        del x, wr, wgu, wd, ws, y
+        torch.cuda.empty_cache()
+        line["train"] = bench_train(M, S, dev, 10, peaks)
+        torch.cuda.empty_cache()
+        line["stack"] = bench_stack(M, S, dev, 5, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, n, times, threads = oracle_sample(4096, args.cpu_budget / 2, steps=2)
         line["cpu_baseline"] = {
@@ -408,6 +580,8 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=4096,
                     help="tokens per layer call (4096 is the benchmarked workload; others are for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the decode, training-step and 16-layer stack workloads (run at N=1 only)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args(argv)
     rank, world, local = dist_env()

@@ -50,7 +50,7 @@ extern "C" {
 struct CUstream_st;
 typedef struct CUstream_st* cudaStream_t;
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 #define MOE_ROW_ALIGN 128
 
 typedef enum moe_status {
@@ -69,7 +69,12 @@ typedef enum moe_dtype { MOE_BF16 = 0, MOE_FP32 = 1 } moe_dtype;
  * d_model a multiple of 128 in [128, 4096] (bf16) or [128, 2048] (fp32);
  * d_ff a multiple of 128 in [128, 4096]; 1 <= top_k <= min(16, E);
  * 1 <= n_experts <= 256. alpha_lb and beta_z weight L_lb and L_z in the backward
- * objective <dy, y> + alpha_lb * L_lb + beta_z * L_z (OLMoE: 0.01 and 0.001). */
+ * objective <dy, y> + alpha_lb * L_lb + beta_z * L_z (OLMoE: 0.01 and 0.001).
+ * grad_dtype is the type moe_backward writes the three weight gradients in:
+ * MOE_BF16 (0, the zero-initialised default: the same type as bf16 weights) or
+ * MOE_FP32 (fp32 gradients for an fp32 optimizer state; the accumulation is fp32
+ * either way, so the bf16 result is the fp32 one rounded once). Ignored by the
+ * forward entry points; an fp32 cfg always gets fp32 gradients. */
 typedef struct moe_config {
   int64_t T;
   int32_t d_model;
@@ -79,6 +84,7 @@ typedef struct moe_config {
   int32_t dtype; /* moe_dtype */
   float alpha_lb;
   float beta_z;
+  int32_t grad_dtype; /* moe_dtype of dw_router, dw_gate_up, dw_down */
 } moe_config;
 
 /* Human-readable name of a status code. Never NULL. */
@@ -218,6 +224,7 @@ moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const voi
  * or through the counts f_i.
  *   dy [device] [T, d];  dx [device] [T, d] out;  dw_router [device] [E, d] out;
  *   dw_gate_up [device] [E, 2f, d] out;  dw_down [device] [E, d, f] out.
+ * dx has the input dtype; the weight gradients have cfg->grad_dtype.
  * Weight gradients are overwritten, not accumulated. bf16 only: an fp32 cfg
  * returns MOE_ERR_UNSUPPORTED_SHAPE (its GEMMs would need MN-major tf32 operands). */
 moe_status moe_backward(const moe_config* cfg, const void* dy, const void* x, const void* w_router,

@@ -13,6 +13,7 @@ from .binding import (  # noqa: F401
     MoeError,
     MoELayer,
     config,
+    grad_torch_dtype,
     lib,
     moe_backward,
     moe_check_config,

@@ -59,6 +59,7 @@ class moe_config(ctypes.Structure):
         ("dtype", ctypes.c_int32),
         ("alpha_lb", ctypes.c_float),
         ("beta_z", ctypes.c_float),
+        ("grad_dtype", ctypes.c_int32),
     ]
 
 
@@ -118,16 +119,26 @@ def _check(status, where):
         raise MoeError(status, where)
 
 
-def config(T, d_model, n_experts, top_k, d_ff, dtype=torch.bfloat16, alpha_lb=0.01, beta_z=0.001):
-    """A moe_config. `dtype` is torch.bfloat16 or torch.float32."""
-    if dtype not in (torch.bfloat16, torch.float32):
-        raise ValueError("dtype must be torch.bfloat16 or torch.float32")
-    return moe_config(int(T), int(d_model), int(n_experts), int(top_k), int(d_ff),
-                      MOE_BF16 if dtype == torch.bfloat16 else MOE_FP32, float(alpha_lb), float(beta_z))
+def config(T, d_model, n_experts, top_k, d_ff, dtype=torch.bfloat16, alpha_lb=0.01, beta_z=0.001,
+           grad_dtype=None):
+    """A moe_config. `dtype` is torch.bfloat16 or torch.float32; `grad_dtype`, the
+    type of the weight gradients moe_backward writes, defaults to `dtype`."""
+    grad_dtype = dtype if grad_dtype is None else grad_dtype
+    for t in (dtype, grad_dtype):
+        if t not in (torch.bfloat16, torch.float32):
+            raise ValueError("dtypes must be torch.bfloat16 or torch.float32")
+    code = lambda t: MOE_BF16 if t == torch.bfloat16 else MOE_FP32
+    return moe_config(int(T), int(d_model), int(n_experts), int(top_k), int(d_ff), code(dtype), float(alpha_lb),
+                      float(beta_z), code(grad_dtype))
 
 
 def torch_dtype(cfg) -> torch.dtype:
     return torch.bfloat16 if cfg.dtype == MOE_BF16 else torch.float32
+
+
+def grad_torch_dtype(cfg) -> torch.dtype:
+    """The dtype of the weight gradients moe_backward writes for `cfg`."""
+    return torch.float32 if (cfg.dtype == MOE_FP32 or cfg.grad_dtype == MOE_FP32) else torch.bfloat16
 
 
 def _stream(stream=None):
@@ -333,12 +344,13 @@ def moe_forward_host(cfg, x_host, w_router, router_bias, w_gate_up, w_down, y_ho
 def moe_backward(cfg, dy, x, w_router, w_gate_up, w_down, dx, dw_router, dw_gate_up, dw_down, ws,
                  stream=None):
     dt = torch_dtype(cfg)
+    gt = grad_torch_dtype(cfg)
     T, d, E, f = cfg.T, cfg.d_model, cfg.n_experts, cfg.d_ff
     st = lib().moe_backward(
         _cfgp(cfg), _ptr(dy, dt, (T, d), "dy"), _ptr(x, dt, (T, d), "x"), _ptr(w_router, dt, (E, d), "w_router"),
         _ptr(w_gate_up, dt, (E, 2 * f, d), "w_gate_up"), _ptr(w_down, dt, (E, d, f), "w_down"),
-        _ptr(dx, dt, (T, d), "dx"), _ptr(dw_router, dt, (E, d), "dw_router"),
-        _ptr(dw_gate_up, dt, (E, 2 * f, d), "dw_gate_up"), _ptr(dw_down, dt, (E, d, f), "dw_down"),
+        _ptr(dx, dt, (T, d), "dx"), _ptr(dw_router, gt, (E, d), "dw_router"),
+        _ptr(dw_gate_up, gt, (E, 2 * f, d), "dw_gate_up"), _ptr(dw_down, gt, (E, d, f), "dw_down"),
         _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
     _check(st, "moe_backward")
 
@@ -392,17 +404,18 @@ class MoELayer:
     """
 
     def __init__(self, w_router, w_gate_up, w_down, router_bias=None, top_k=8, alpha_lb=0.01,
-                 beta_z=0.001):
+                 beta_z=0.001, grad_dtype=None):
         self.w_router, self.w_gate_up, self.w_down = w_router, w_gate_up, w_down
         self.router_bias = router_bias
         self.top_k = top_k
         self.alpha_lb, self.beta_z = alpha_lb, beta_z
+        self.grad_dtype = grad_dtype
         self._ws = {}
 
     def cfg(self, T):
         E, d = self.w_router.shape
         f = self.w_down.shape[2]
-        return config(T, d, E, self.top_k, f, self.w_router.dtype, self.alpha_lb, self.beta_z)
+        return config(T, d, E, self.top_k, f, self.w_router.dtype, self.alpha_lb, self.beta_z, self.grad_dtype)
 
     def ws(self, T, train):
         key = (T, bool(train))
@@ -426,11 +439,12 @@ class MoELayer:
         x = self._x
         T = x.shape[0]
         cfg = self.cfg(T)
+        gt = grad_torch_dtype(cfg)
         g = {
             "dx": torch.empty_like(x),
-            "dw_router": torch.empty_like(self.w_router),
-            "dw_gate_up": torch.empty_like(self.w_gate_up),
-            "dw_down": torch.empty_like(self.w_down),
+            "dw_router": torch.empty_like(self.w_router, dtype=gt),
+            "dw_gate_up": torch.empty_like(self.w_gate_up, dtype=gt),
+            "dw_down": torch.empty_like(self.w_down, dtype=gt),
         }
         moe_backward(cfg, dy, x, self.w_router, self.w_gate_up, self.w_down, g["dx"], g["dw_router"],
                      g["dw_gate_up"], g["dw_down"], self.ws(T, True))

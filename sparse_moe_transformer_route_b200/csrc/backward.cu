@@ -281,7 +281,7 @@ cudaError_t launch_router_weight_grad(const Shape& s, const float* dh, const voi
   if (e != cudaSuccess) return e;
   const int64_t n = static_cast<int64_t>(s.E) * s.d;
   const unsigned g2 = static_cast<unsigned>((n + 255) / 256);
-  if (s.fp32)
+  if (s.fp32 || s.grad32)
     router_wgrad_reduce<float><<<g2, 256, 0, st>>>(part, n, static_cast<float*>(dw_router));
   else
     router_wgrad_reduce<__nv_bfloat16><<<g2, 256, 0, st>>>(part, n, static_cast<__nv_bfloat16*>(dw_router));

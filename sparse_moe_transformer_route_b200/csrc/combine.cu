@@ -52,6 +52,30 @@ struct Vec8 {
   }
 };
 
+// Eight elements as loaded (16 bytes of bf16 or 32 of fp32), unpacked later.
+template <typename T_>
+struct Raw8 {
+  uint4 a, b;
+  __device__ __forceinline__ void load(const T_* p) {
+    a = __ldg(reinterpret_cast<const uint4*>(p));
+    if constexpr (sizeof(T_) == 4) b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+  }
+  __device__ __forceinline__ void unpack(float (&v)[8]) const {
+    if constexpr (sizeof(T_) == 4) {
+      v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y); v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
+      v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y); v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
+    } else {
+      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+        v[2 * j] = f.x;
+        v[2 * j + 1] = f.y;
+      }
+    }
+  }
+};
+
 template <typename T_, bool RESID>
 __global__ void __launch_bounds__(256)
     combine_kernel(const T_* __restrict__ o_perm, const int32_t* __restrict__ inv_perm, const float* __restrict__ wts,
@@ -69,14 +93,28 @@ __global__ void __launch_bounds__(256)
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int r = rows[j];
-      if (r < 0) continue;
-      Vec8<T_> o;
-      o.load(o_perm + static_cast<int64_t>(r) * d + v * 8);
-      const float w = ws_[j];
+    // The k rows' loads go out together (unconditional: a slot without a row
+    // re-reads row 0, which always exists, and is then skipped), then the sum
+    // runs in slot order.
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      Raw8<T_> q[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, o.v[i], acc[i]);
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = j0 + jj;
+        const int r = (j < k) ? rows[j] : -1;
+        q[jj].load(o_perm + static_cast<int64_t>(r < 0 ? 0 : r) * d + v * 8);
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = j0 + jj;
+        if (j < k && rows[j] >= 0) {
+          float o[8];
+          q[jj].unpack(o);
+          const float w = ws_[j];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, o[i], acc[i]);
+        }
+      }
     }
     if constexpr (RESID) {
       float* rp = resid + t * d + v * 8;

@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) rows[j] = __shfl_sync(0xffffffffu, row, j < k ? j : 0);
     const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
-    for (int v = lane; v < nvec; v += 32) {
+    for (int v = lane; x_perm != nullptr && v < nvec; v += 32) {
       const uint4 val = src[v];
 #pragma unroll
       for (int j = 0; j < kMaxTopK; ++j) {
@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(256)
       const int r1 = gs[e + 1];
       for (int r = r0 + warp; r < r1; r += 8) {
         if (lane == 0) row_pair[r] = -1;
+        if (x_perm == nullptr) continue;
         uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(r) * d);
         for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
       }

@@ -45,7 +45,9 @@ enum class Epi { SwigluFwd, Store, SwigluBwd };
 // 64 B per MMA cycle instead of 96, the difference between starving and not
 // on HBM-resident weights. A 256-row tile whose second half lies past its
 // expert's rows issues only the first half.
-template <bool TF32_, bool A_MN_, bool B_MN_, Group G_, Epi EP_, int BN_, int H_ = 1>
+// O32: plain-store output in fp32 whatever the operand type (weight gradients
+// kept in fp32 for the caller's optimizer).
+template <bool TF32_, bool A_MN_, bool B_MN_, Group G_, Epi EP_, int BN_, int H_ = 1, bool O32_ = false>
 struct Cfg {
   static constexpr bool TF32 = TF32_;
   static constexpr bool A_MN = A_MN_;
@@ -55,6 +57,8 @@ struct Cfg {
   static constexpr int BN = BN_;
   static constexpr int H = H_;
   using T = std::conditional_t<TF32, float, __nv_bfloat16>;
+  static constexpr bool O32 = O32_;
+  using OutT = std::conditional_t<TF32 || O32, float, __nv_bfloat16>;
   static constexpr int BM = 128 * H;
   static constexpr int ESZ = TF32 ? 4 : 2;
   static constexpr int BK = 128 / ESZ;      // K per stage (one 128-byte swizzle row when K-major)
@@ -73,7 +77,7 @@ struct Cfg {
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   // Each epilogue warp stages a 32 x 32 output chunk in shared memory (rows
   // padded by 16 bytes against bank conflicts) and writes it back as whole rows.
-  static constexpr int STG_PITCH = 32 * ESZ + 16;
+  static constexpr int STG_PITCH = 32 * static_cast<int>(sizeof(OutT)) + 16;
   static constexpr int STG_WARP_BYTES = 32 * STG_PITCH;
   static constexpr int STG_BYTES = EPI_WARPS * STG_WARP_BYTES;
   static constexpr int MISC_BYTES = 1024 + 3 * (kMaxExperts + 1) * static_cast<int>(sizeof(int32_t));
@@ -87,6 +91,7 @@ struct Cfg {
   static_assert(H == 1 || H == 2, "tile M");
   static_assert(!(H == 2 && TF32), "256-row tiles are bf16 only");
   static_assert(!(EP == Epi::SwigluFwd && B_MN), "gate/up weights are read K-major");
+  static_assert(!O32 || EP == Epi::Store, "fp32 output only for plain stores");
 };
 
 struct Args {
@@ -281,7 +286,8 @@ __device__ __forceinline__ void warp_store_chunk(unsigned char* stg, const float
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
+                        const __grid_constant__ CUtensorMap tmB,
                         const Args a) {
   using T = typename C::T;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -324,6 +330,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
+    if constexpr (!C::A_MN) tma_prefetch_desc(&tmA32);
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
@@ -353,12 +360,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           unsigned char* sa = stage_base + static_cast<size_t>(stage) * C::STAGE_BYTES;
           unsigned char* sb = sa + C::A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], t.halves * C::A_HALF + C::B_BYTES);
-          // A operand: one 128-row half per TMA box (K-major), or 128-byte column chunks (MN-major)
+          // A operand, K-major: a 128-row box per half, or, for a half with at
+          // most 96 valid rows, 32-row boxes covering only those (the rows past
+          // them keep stale data; their accumulator rows are never stored).
+          // MN-major: 128-byte column chunks of whole halves.
           if constexpr (!C::A_MN) {
-            for (int hh = 0; hh < t.halves; ++hh)
-              tma_load_2d(&tmA, &full[stage], sa + hh * C::A_HALF, kb * C::BK, t.m0 + hh * 128);
+            int a_bytes = 0;
+            for (int hh = 0; hh < t.halves; ++hh) {
+              const int vr = max(0, min(128, t.valid - hh * 128));
+              a_bytes += (vr > 96) ? C::A_HALF : ((vr + 31) / 32) * (32 * 128);
+            }
+            mbar_arrive_expect_tx(&full[stage], a_bytes + C::B_BYTES);
+            for (int hh = 0; hh < t.halves; ++hh) {
+              const int vr = max(0, min(128, t.valid - hh * 128));
+              if (vr > 96) {
+                tma_load_2d(&tmA, &full[stage], sa + hh * C::A_HALF, kb * C::BK, t.m0 + hh * 128);
+              } else {
+                for (int q = 0; q < (vr + 31) / 32; ++q)
+                  tma_load_2d(&tmA32, &full[stage], sa + hh * C::A_HALF + q * (32 * 128), kb * C::BK,
+                              t.m0 + hh * 128 + 32 * q);
+              }
+            }
           } else {
+            mbar_arrive_expect_tx(&full[stage], t.halves * C::A_HALF + C::B_BYTES);
             for (int ch = 0; ch < t.halves * (128 / C::CH); ++ch)
               tma_load_2d(&tmA, &full[stage], sa + ch * (C::BK * 128), t.m0 + ch * C::CH,
                           t.krow0 + kb * C::BK);
@@ -461,7 +485,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int r_local = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    T* out = static_cast<T*>(a.out);
+    using OutT = typename C::OutT;
+    OutT* out = static_cast<OutT*>(a.out);
     for (int L = blockIdx.x; L < n_tiles; L += gridDim.x) {
       const Tile t = decode_tile<C>(a, gs, off, ts, L);
       if (hsel >= t.halves) {  // this half lies past the expert's rows: nothing to store
@@ -483,7 +508,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // this warp's share of the tile's output columns
       constexpr int WCOLS = C::OUT_N / 2;
       const int cw = csel * WCOLS;
-      T* obase;  // (wrow0, n0 + cw)
+      OutT* obase;  // (wrow0, n0 + cw)
       if constexpr (C::G == Group::M)
         obase = out + wrow0 * a.ld_out + t.n0 + cw;
       else
@@ -494,7 +519,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         float z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = 0.f;
-        for (int c = 0; c < WCOLS; c += 32) warp_store_chunk<T, C::STG_PITCH>(stg, z, obase + c, a.ld_out, lane);
+        for (int c = 0; c < WCOLS; c += 32) warp_store_chunk<OutT, C::STG_PITCH>(stg, z, obase + c, a.ld_out, lane);
         continue;
       }
       if (!mbar_wait(&acc_full[acc], acc_phase)) {
@@ -514,7 +539,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = row_ok ? __uint_as_float(r[i]) : 0.f;
-          warp_store_chunk<T, C::STG_PITCH>(stg, v, obase + c, a.ld_out, lane);
+          warp_store_chunk<OutT, C::STG_PITCH>(stg, v, obase + c, a.ld_out, lane);
         }
       } else if constexpr (C::EP == Epi::SwigluFwd) {
         T* pbase = (a.out2 != nullptr) ? static_cast<T*>(a.out2) + wrow0 * a.ld_out2 + t.n0 + cw : nullptr;
@@ -627,7 +652,8 @@ bool make_map(CUtensorMap* m, const void* base, bool fp32, uint64_t rows, uint64
 namespace {
 
 template <class C>
-cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Args& a, int max_tiles, cudaStream_t st) {
+cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb, const Args& a,
+                   int max_tiles, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -638,7 +664,7 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Args& a, 
   int grid = device_sm_count();
   if (max_tiles < grid) grid = max_tiles;
   if (grid <= 0) return cudaSuccess;
-  grouped_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(ta, tb, a);
+  grouped_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(ta, ta32, tb, a);
   return cudaGetLastError();
 }
 
@@ -654,16 +680,16 @@ Args base_args(const Shape& s, const int32_t* gs, const int32_t* off, int32_t* s
 int ch_elems(bool fp32) { return fp32 ? 32 : 64; }
 
 // Instantiates the kernel for the dtype, tile N and tile M (h 128-row halves).
-template <bool A_MN, bool B_MN, Group G, Epi EP>
-cudaError_t run_variant(bool fp32, int bn, int h, const CUtensorMap& ta, const CUtensorMap& tb, const Args& a,
-                        int max_tiles, cudaStream_t st) {
+template <bool A_MN, bool B_MN, Group G, Epi EP, bool O32 = false>
+cudaError_t run_variant(bool fp32, int bn, int h, const CUtensorMap& ta, const CUtensorMap& ta32,
+                        const CUtensorMap& tb, const Args& a, int max_tiles, cudaStream_t st) {
   if (fp32) {
-    if (bn == 256) return launch<Cfg<true, A_MN, B_MN, G, EP, 256, 1>>(ta, tb, a, max_tiles, st);
-    return launch<Cfg<true, A_MN, B_MN, G, EP, 128, 1>>(ta, tb, a, max_tiles, st);
+    if (bn == 256) return launch<Cfg<true, A_MN, B_MN, G, EP, 256, 1>>(ta, ta32, tb, a, max_tiles, st);
+    return launch<Cfg<true, A_MN, B_MN, G, EP, 128, 1>>(ta, ta32, tb, a, max_tiles, st);
   }
   (void)h;
-  if (bn == 256) return launch<Cfg<false, A_MN, B_MN, G, EP, 256, 1>>(ta, tb, a, max_tiles, st);
-  return launch<Cfg<false, A_MN, B_MN, G, EP, 128, 1>>(ta, tb, a, max_tiles, st);
+  if (bn == 256) return launch<Cfg<false, A_MN, B_MN, G, EP, 256, 1, O32>>(ta, ta32, tb, a, max_tiles, st);
+  return launch<Cfg<false, A_MN, B_MN, G, EP, 128, 1, O32>>(ta, ta32, tb, a, max_tiles, st);
 }
 
 // Tile M. 256-row tiles (H = 2) halve the operand bytes per MMA cycle, but two
@@ -677,14 +703,24 @@ int pick_h(const Shape&) { return 1; }
 // Tile N for a forward GEMM whose accumulator covers `n` columns per expert.
 static int pick_bn(int n) { return (n % 256 == 0) ? 256 : 128; }
 
+// Few routed rows (decode): at most min(T*k, E) expert groups of one or two
+// 128-row tiles. When 256-column tiles would leave SMs idle, 128-column tiles
+// double the number of CTAs streaming the experts' weights.
+static bool few_tiles(const Shape& s, int n_cols) {
+  const int64_t groups = (s.T * s.k < s.E) ? s.T * s.k : s.E;
+  const int64_t m_tiles = groups + (s.T * s.k) / 128;
+  return m_tiles * (n_cols / 256) < device_sm_count();
+}
+
 cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* group_start,
                            const int32_t* offsets, const void* w_gate_up, void* h, void* preact, int32_t* status,
                            cudaStream_t st) {
   // accumulator: BN/2 gate columns and BN/2 up columns of the same outputs
-  const int bn = ((s.f % 128) == 0) ? 256 : 128;
+  const int bn = few_tiles(s, 2 * s.f) ? 128 : 256;
   const int kcols = ch_elems(s.fp32);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, ta32, tb;
   if (!make_map(&ta, x_perm, s.fp32, s.P, s.d, kcols, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&ta32, x_perm, s.fp32, s.P, s.d, kcols, 32)) return cudaErrorInvalidValue;
   if (!make_map(&tb, w_gate_up, s.fp32, static_cast<uint64_t>(s.E) * 2 * s.f, s.d, kcols, bn / 2))
     return cudaErrorInvalidValue;
   Args a = base_args(s, group_start, offsets, status);
@@ -697,15 +733,16 @@ cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* gr
   a.out2 = preact;
   a.ld_out2 = 2 * s.f;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.f / (bn / 2)));
-  return run_variant<false, false, Group::M, Epi::SwigluFwd>(s.fp32, bn, pick_h(s), ta, tb, a, max_tiles, st);
+  return run_variant<false, false, Group::M, Epi::SwigluFwd>(s.fp32, bn, pick_h(s), ta, ta32, tb, a, max_tiles, st);
 }
 
 cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_start, const int32_t* offsets,
                         const void* w_down, void* o_perm, int32_t* status, cudaStream_t st) {
-  const int bn = pick_bn(s.d);
+  const int bn = few_tiles(s, s.d) ? 128 : pick_bn(s.d);
   const int kcols = ch_elems(s.fp32);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, ta32, tb;
   if (!make_map(&ta, h, s.fp32, s.P, s.f, kcols, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&ta32, h, s.fp32, s.P, s.f, kcols, 32)) return cudaErrorInvalidValue;
   if (!make_map(&tb, w_down, s.fp32, static_cast<uint64_t>(s.E) * s.d, s.f, kcols, bn))
     return cudaErrorInvalidValue;
   Args a = base_args(s, group_start, offsets, status);
@@ -715,7 +752,7 @@ cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_star
   a.out = o_perm;
   a.ld_out = s.d;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.d / bn));
-  return run_variant<false, false, Group::M, Epi::Store>(s.fp32, bn, pick_h(s), ta, tb, a, max_tiles, st);
+  return run_variant<false, false, Group::M, Epi::Store>(s.fp32, bn, pick_h(s), ta, ta32, tb, a, max_tiles, st);
 }
 
 // dG = dO W_down (K = d, B read MN-major from W_down [E*d, f]); epilogue forms
@@ -726,8 +763,9 @@ cudaError_t launch_down_backward_data(const Shape& s, const void* dout, const in
   const int bn = pick_bn(s.f);
   const int kc = ch_elems(s.fp32);
   const int bk = s.fp32 ? 32 : 64;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, ta32, tb;
   if (!make_map(&ta, dout, s.fp32, s.P, s.d, kc, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&ta32, dout, s.fp32, s.P, s.d, kc, 32)) return cudaErrorInvalidValue;
   if (!make_map(&tb, w_down, s.fp32, static_cast<uint64_t>(s.E) * s.d, s.f, kc, bk)) return cudaErrorInvalidValue;
   Args a = base_args(s, group_start, offsets, status);
   a.N_total = s.f;
@@ -739,7 +777,7 @@ cudaError_t launch_down_backward_data(const Shape& s, const void* dout, const in
   a.aux = preact;
   a.ld_aux = 2 * s.f;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.f / bn));
-  return run_variant<false, true, Group::M, Epi::SwigluBwd>(s.fp32, bn, pick_h(s), ta, tb, a, max_tiles, st);
+  return run_variant<false, true, Group::M, Epi::SwigluBwd>(s.fp32, bn, pick_h(s), ta, ta32, tb, a, max_tiles, st);
 }
 
 // dX_perm = [dA|dB] W_gate_up (K = 2f, B read MN-major from W_gate_up [E*2f, d]).
@@ -749,8 +787,9 @@ cudaError_t launch_gate_up_backward_data(const Shape& s, const void* dab, const 
   const int bn = pick_bn(s.d);
   const int kc = ch_elems(s.fp32);
   const int bk = s.fp32 ? 32 : 64;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, ta32, tb;
   if (!make_map(&ta, dab, s.fp32, s.P, 2 * s.f, kc, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&ta32, dab, s.fp32, s.P, 2 * s.f, kc, 32)) return cudaErrorInvalidValue;
   if (!make_map(&tb, w_gate_up, s.fp32, static_cast<uint64_t>(s.E) * 2 * s.f, s.d, kc, bk))
     return cudaErrorInvalidValue;
   Args a = base_args(s, group_start, offsets, status);
@@ -760,7 +799,7 @@ cudaError_t launch_gate_up_backward_data(const Shape& s, const void* dab, const 
   a.out = dx_perm;
   a.ld_out = s.d;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.d / bn));
-  return run_variant<false, true, Group::M, Epi::Store>(s.fp32, bn, pick_h(s), ta, tb, a, max_tiles, st);
+  return run_variant<false, true, Group::M, Epi::Store>(s.fp32, bn, pick_h(s), ta, ta32, tb, a, max_tiles, st);
 }
 
 namespace {
@@ -772,6 +811,7 @@ cudaError_t launch_kgrouped(const Shape& s, const void* A, int M_total, const vo
   const int bk = s.fp32 ? 32 : 64;
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, s.fp32, s.P, M_total, kc, bk)) return cudaErrorInvalidValue;
+  const CUtensorMap& ta32 = ta;  // MN-major A: whole halves only
   if (!make_map(&tb, B, s.fp32, s.P, N_total, kc, bk)) return cudaErrorInvalidValue;
   Args a = base_args(s, gs, off, status);
   a.M_total = M_total;
@@ -781,7 +821,9 @@ cudaError_t launch_kgrouped(const Shape& s, const void* A, int M_total, const vo
   a.out_expert_stride = static_cast<int64_t>(M_total) * N_total;
   const int h = pick_h(s);
   const int max_tiles = s.E * (M_total / (128 * h)) * (N_total / bn);
-  return run_variant<true, true, Group::K, Epi::Store>(s.fp32, bn, h, ta, tb, a, max_tiles, st);
+  if (s.grad32 && !s.fp32)
+    return run_variant<true, true, Group::K, Epi::Store, true>(s.fp32, bn, h, ta, ta32, tb, a, max_tiles, st);
+  return run_variant<true, true, Group::K, Epi::Store>(s.fp32, bn, h, ta, ta32, tb, a, max_tiles, st);
 }
 }  // namespace
 

@@ -45,6 +45,7 @@ int device_sm_count() {
 bool make_shape(const moe_config* cfg, Shape* s) {
   if (cfg == nullptr) return false;
   if (cfg->dtype != MOE_BF16 && cfg->dtype != MOE_FP32) return false;
+  if (cfg->grad_dtype != MOE_BF16 && cfg->grad_dtype != MOE_FP32) return false;
   const bool fp32 = cfg->dtype == MOE_FP32;
   const int dmax = fp32 ? 2048 : 4096;
   if (cfg->T < 1 || cfg->T > (int64_t(1) << 24)) return false;
@@ -58,6 +59,7 @@ bool make_shape(const moe_config* cfg, Shape* s) {
   s->k = cfg->top_k;
   s->f = cfg->d_ff;
   s->fp32 = fp32;
+  s->grad32 = fp32 || cfg->grad_dtype == MOE_FP32;
   s->esize = fp32 ? 4 : 2;
   s->P = static_cast<int64_t>(up(static_cast<size_t>(cfg->T * cfg->top_k + int64_t(cfg->n_experts) * (kRowAlign - 1)),
                                  kRowAlign));
@@ -164,23 +166,23 @@ moe_status forward_impl(const Ctx& c, const void* x, const void* w_router, const
   float* wts = at<float>(ws, L.wts);
   int32_t* gs = at<int32_t>(ws, L.group_start);
   int32_t* off = at<int32_t>(ws, L.offsets);
+  void* x_perm = at<void>(ws, L.x_perm);
   const StageMarks marks(st);
   MOE_TRY(marks.mark(0));
   if (router_tc_supported(s)) {
     // the tensor-core router also leaves the dispatch ranking in ws
     MOE_TRY(launch_router_tc(s, x, w_router, bias, idx, wts, nullptr, losses, ws, L, st));
     MOE_TRY(marks.mark(1));
-    MOE_TRY(launch_permute(s, idx, x, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv_perm), at<void>(ws, L.x_perm), ws,
-                           L, save, st));
+    MOE_TRY(launch_permute(s, idx, x, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv_perm), x_perm, ws, L, save, st));
   } else {
     MOE_TRY(launch_router(s, x, w_router, bias, idx, wts, nullptr, losses, ws, L, st));
     MOE_TRY(marks.mark(1));
     MOE_TRY(launch_dispatch_impl(s, idx, x, nullptr, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv_perm), nullptr,
-                                 at<void>(ws, L.x_perm), ws, L, save, st));
+                                 x_perm, ws, L, save, st));
   }
   MOE_TRY(marks.mark(2));
-  MOE_TRY(launch_gate_up(s, at<void>(ws, L.x_perm), gs, off, w_gate_up, at<void>(ws, L.h),
-                         save ? at<void>(ws, L.preact) : nullptr, status, st));
+  MOE_TRY(launch_gate_up(s, x_perm, gs, off, w_gate_up, at<void>(ws, L.h), save ? at<void>(ws, L.preact) : nullptr,
+                         status, st));
   MOE_TRY(marks.mark(3));
   MOE_TRY(launch_down(s, at<void>(ws, L.h), gs, off, w_down, at<void>(ws, L.o_perm), status, st));
   MOE_TRY(marks.mark(4));

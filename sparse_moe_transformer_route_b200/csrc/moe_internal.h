@@ -22,6 +22,7 @@ struct Shape {
   int64_t T;
   int d, E, k, f;
   bool fp32;
+  bool grad32;   // backward writes the weight gradients in fp32
   size_t esize;  // bytes per activation / weight element
   int64_t P;     // padded row capacity
   int64_t router_ctas() const { return (T + kRouterTokensPerCta - 1) / kRouterTokensPerCta; }
