@@ -11,7 +11,8 @@
 // One CTA takes 32 tokens (one dispatch chunk), so a 4096-token layer spreads
 // over 128 SMs:
 //   warp 0     TMA loads of x [32 x 64] and W_r [E_pad x 64] per K step into a
-//              16-deep ring. The MMA reads a 128-row A operand; rows 32..127
+//              16-deep ring, or a 7-deep one with two CTAs per SM when there
+//              are more tiles than SMs (one's epilogue overlaps the other's loads). The MMA reads a 128-row A operand; rows 32..127
 //              are whatever lies in shared memory after the 32 loaded rows,
 //              and their accumulator rows are never read.
 //   warp 1     tcgen05.mma M=128 N=E_pad K=16, fp32 accumulator in TMEM
@@ -41,19 +42,19 @@ namespace moe {
 namespace {
 
 constexpr int kTile = kDispatchChunk;  // 32 tokens
-constexpr int kStages = 16;
 constexpr int kThreads = 192;
 constexpr int kMaxE = 64;
 constexpr int kMaxSel = kMaxTopK + 3;
 constexpr int kAload = kTile * 128;                      // bytes of A loaded per stage
 constexpr int kStageMax = kAload + kMaxE * 128;          // 12 KB
-constexpr int kRing = kStages * kStageMax + 16 * 1024;   // + the over-read of the last stage's A
+// ring bytes for S stages, plus the over-read of the last stage's A
+constexpr int ring_bytes(int S) { return S * kStageMax + 16 * 1024; }
 constexpr int kLogitStride = kMaxE + 1;
-constexpr int kScanBlock = 256;                          // chunks scanned per pass in the last CTA
+constexpr int kScanBlock = 128;                          // chunks scanned per pass in the last CTA
 constexpr size_t kMiscBytes = 4096;
-constexpr size_t kSmem = 1024 + static_cast<size_t>(kRing) + kMiscBytes;
+constexpr size_t smem_bytes(int S) { return 1024 + static_cast<size_t>(ring_bytes(S)) + kMiscBytes; }
 static_assert(kTile == 32, "one mask word per expert");
-static_assert(kScanBlock * kMaxE * 8 <= kRing, "scan block fits in the ring");
+static_assert(kScanBlock * kMaxE * 8 <= ring_bytes(7), "scan block fits in the smallest ring");
 
 struct RArgs {
   int64_t T;
@@ -140,7 +141,11 @@ __device__ __forceinline__ double exact_logit_warp(const __nv_bfloat16* xr, cons
   return acc;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// STAGES-deep ring, MINB CTAs per SM: one CTA with a 16-deep ring when the
+// tiles fit on the SMs at once, two with 7-deep rings (one's epilogue then
+// overlaps the other's loads) when there are more tiles than SMs.
+template <int STAGES, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                      const RArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -148,10 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int STAGE = kAload + a.NP * 128;  // A rows 0..31, then B
   unsigned char* ring = smem;
-  unsigned char* misc = smem + kRing;
+  unsigned char* misc = smem + ring_bytes(STAGES);
   uint64_t* full = reinterpret_cast<uint64_t*>(misc);
-  uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
   uint32_t* mask = tmem_holder + 4;                          // [kMaxE]
   float* lse_s = reinterpret_cast<float*>(mask + kMaxE);      // [kTile]
@@ -172,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -197,8 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // same router-weight tile of L2 at the same moment
       const int k0 = static_cast<int>(blockIdx.x % static_cast<unsigned>(nk));
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kStages;
-        const uint32_t ph = static_cast<uint32_t>(kb / kStages) & 1u;
+        const int s = kb % STAGES;
+        const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u)) {
           report(a.status, DEV_WAIT_TIMEOUT_PRODUCER);
           break;
@@ -210,9 +215,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(&tmw, &full[s], st + kAload, kc * 64, 0);
         ++issued;
       }
-      for (int s = 0; s < kStages && s < issued; ++s) {
-        const int last = ((issued - 1 - s) / kStages) * kStages + s;
-        if (!mbar_wait(&full[s], static_cast<uint32_t>((last / kStages) & 1))) report(a.status, DEV_WAIT_TIMEOUT_DRAIN);
+      for (int s = 0; s < STAGES && s < issued; ++s) {
+        const int last = ((issued - 1 - s) / STAGES) * STAGES + s;
+        if (!mbar_wait(&full[s], static_cast<uint32_t>((last / STAGES) & 1))) report(a.status, DEV_WAIT_TIMEOUT_DRAIN);
       }
     }
   } else if (warp == 1) {
@@ -220,8 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = make_idesc(false, false, false, 128, a.NP);
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kStages;
-        if (!mbar_wait(&full[s], static_cast<uint32_t>(kb / kStages) & 1u)) {
+        const int s = kb % STAGES;
+        if (!mbar_wait(&full[s], static_cast<uint32_t>(kb / STAGES) & 1u)) {
           report(a.status, DEV_WAIT_TIMEOUT_MMA);
           ok = false;
           break;
@@ -650,8 +655,11 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router
                              cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e =
-        cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes(16)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(router_tc_kernel<7, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_bytes(7)));
     if (e != cudaSuccess) return e;
     configured = true;
   }
@@ -689,7 +697,10 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router
   a.ticket = ctrl + 1;
   a.status = ctrl;
   const unsigned grid = static_cast<unsigned>((s.T + kTile - 1) / kTile);
-  router_tc_kernel<<<grid, kThreads, kSmem, st>>>(tx, tw, a);
+  if (static_cast<int>(grid) <= device_sm_count())
+    router_tc_kernel<16, 1><<<grid, kThreads, smem_bytes(16), st>>>(tx, tw, a);
+  else
+    router_tc_kernel<7, 2><<<grid, kThreads, smem_bytes(7), st>>>(tx, tw, a);
   return cudaGetLastError();
 }
 

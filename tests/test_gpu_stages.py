@@ -119,8 +119,10 @@ def _bar(ref):
 GEMM_COUNTS = [
     [0, 1, 127, 128, 129, 300, 0, 5],
     [513, 0, 0, 2, 255, 256, 1, 64],
-    # >= 256 rows per expert on average: 256-row tiles, some with only one 128-row half
     [700, 129, 384, 0, 255, 1, 513, 128],
+    # >= 384 rows per expert on average: 256-row tiles on CTA pairs, some whose
+    # second half lies in the next expert's group (and must not be written)
+    [700, 129, 385, 0, 900, 1, 513, 640],
 ]
 
 
