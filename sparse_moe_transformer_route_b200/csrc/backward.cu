@@ -124,96 +124,158 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-constexpr int kDxTok = 16;
+// dx for a 64-token x 128-column tile per CTA: the router term dh W_r from
+// shared-memory tiles of dh and W_r (64 experts at a time; thread = 8 tokens x
+// 4 columns), then the k expert rows added in slot order.
+constexpr int kDxRows = 64;
+constexpr int kDxCols = 128;
+constexpr int kDxE = 64;
 
-// dx for 16 tokens per CTA: the k expert rows plus the router term dh W_r.
+template <typename T_>
+__device__ __forceinline__ void load4(const T_* p, float (&v)[4]) {
+  if constexpr (sizeof(T_) == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  } else {
+    const uint2 q = *reinterpret_cast<const uint2*>(p);
+    const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+    const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+    v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+  }
+}
+
+template <typename T_>
+__device__ __forceinline__ void store4(T_* p, const float (&v)[4]) {
+  if constexpr (sizeof(T_) == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  } else {
+    uint2 q;
+    q.x = pack_bf16x2(v[0], v[1]);
+    q.y = pack_bf16x2(v[2], v[3]);
+    *reinterpret_cast<uint2*>(p) = q;
+  }
+}
+
 template <typename T_>
 __global__ void __launch_bounds__(256)
     dx_kernel(const T_* __restrict__ dx_perm, const int32_t* __restrict__ inv_perm, const float* __restrict__ dh,
               const T_* __restrict__ w_router, int64_t T, int d, int E, int k, T_* __restrict__ dx) {
-  __shared__ float sdh[kDxTok * kMaxExperts];
-  __shared__ int32_t srow[kDxTok * kMaxTopK];
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kDxTok;
-  const int nt = static_cast<int>((T - t0) < kDxTok ? (T - t0) : kDxTok);
-  for (int i = threadIdx.x; i < nt * E; i += blockDim.x) sdh[i] = dh[t0 * E + i];
-  for (int i = threadIdx.x; i < nt * k; i += blockDim.x) srow[i] = inv_perm[t0 * k + i];
-  __syncthreads();
-  const int nv = d / 8;
-  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
-    float acc[kDxTok][8];
+  __shared__ float sdh[kDxRows][kDxE];
+  __shared__ __align__(16) float sw[kDxE][kDxCols];
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kDxRows;
+  const int c0 = blockIdx.y * kDxCols;
+  const int tg = threadIdx.x >> 5;        // tokens t0 + 8 tg .. +7
+  const int cg = threadIdx.x & 31;        // columns c0 + 4 cg .. +3
+  float acc[8][4];
 #pragma unroll
-    for (int t = 0; t < kDxTok; ++t)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[t][i] = 0.f;
-    for (int e = 0; e < E; ++e) {
-      float wr[8];
-      load8<T_>(w_router + static_cast<int64_t>(e) * d + v * 8, wr);
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int e0 = 0; e0 < E; e0 += kDxE) {
+    const int ne = min(kDxE, E - e0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kDxRows * kDxE; i += blockDim.x) {
+      const int r = i / kDxE, e = i - r * kDxE;
+      sdh[r][e] = (t0 + r < T && e < ne) ? dh[(t0 + r) * E + e0 + e] : 0.f;
+    }
+    for (int i = threadIdx.x; i < kDxE * (kDxCols / 4); i += blockDim.x) {
+      const int e = i / (kDxCols / 4), c = (i - e * (kDxCols / 4)) * 4;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (e < ne && c0 + c < d) load4<T_>(w_router + static_cast<int64_t>(e0 + e) * d + c0 + c, v);
+      *reinterpret_cast<float4*>(&sw[e][c]) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+    __syncthreads();
+    for (int e = 0; e < ne; ++e) {
+      const float4 w = *reinterpret_cast<const float4*>(&sw[e][4 * cg]);
 #pragma unroll
-      for (int t = 0; t < kDxTok; ++t) {
-        const float g = (t < nt) ? sdh[t * E + e] : 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[t][i] = fmaf(g, wr[i], acc[t][i]);
+      for (int i = 0; i < 8; ++i) {
+        const float g = sdh[8 * tg + i][e];
+        acc[i][0] = fmaf(g, w.x, acc[i][0]);
+        acc[i][1] = fmaf(g, w.y, acc[i][1]);
+        acc[i][2] = fmaf(g, w.z, acc[i][2]);
+        acc[i][3] = fmaf(g, w.w, acc[i][3]);
       }
     }
-    for (int t = 0; t < nt; ++t) {
-      float out[8];
+  }
+  const int col = c0 + 4 * cg;
+  if (col >= d) return;
+  for (int i = 0; i < 8; ++i) {
+    const int64_t t = t0 + 8 * tg + i;
+    if (t >= T) break;
+    float out[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const int r = inv_perm[t * k + j];
+      if (r < 0) continue;
+      float g[4];
+      load4<T_>(dx_perm + static_cast<int64_t>(r) * d + col, g);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) out[i] = 0.f;
-      for (int j = 0; j < k; ++j) {
-        const int r = srow[t * k + j];
-        if (r < 0) continue;
-        float g[8];
-        load8<T_>(dx_perm + static_cast<int64_t>(r) * d + v * 8, g);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) out[i] += g[i];
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) out[i] += acc[t][i];
-      store8<T_>(dx + (t0 + t) * d + v * 8, out);
+      for (int c = 0; c < 4; ++c) out[c] += g[c];
     }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) out[c] += acc[i][c];
+    store4<T_>(dx + t * d + col, out);
   }
 }
 
 constexpr int kWrSplit = 32;  // token splits for the router weight gradient
+constexpr int kWrTok = 32;    // tokens per shared-memory chunk
 
-// Partial dW_r over a token range: thread = (8 columns, 8 experts).
+// Partial dW_r over a token range for a 64-expert x 128-column tile: chunks of
+// 32 tokens of dh and x staged in shared memory; thread = 8 experts x 4 columns.
 template <typename T_>
 __global__ void __launch_bounds__(256)
     router_wgrad_partial(const float* __restrict__ dh, const T_* __restrict__ x, int64_t T, int d, int E,
                          float* __restrict__ part) {
-  const int colblk = blockIdx.x;  // 256 columns
+  __shared__ __align__(16) float sdh[kWrTok][64];
+  __shared__ __align__(16) float sx[kWrTok][128];
+  const int c0 = blockIdx.x * 128;
   const int split = blockIdx.y;
-  const int v = threadIdx.x & 31;   // column vector within the block
-  const int eg = blockIdx.z * 8 + (threadIdx.x >> 5);  // expert group of 8
-  const int col = colblk * 256 + v * 8;
+  const int e0 = blockIdx.z * 64;
+  const int eg = threadIdx.x >> 5;  // experts e0 + 8 eg .. +7
+  const int cg = threadIdx.x & 31;  // columns c0 + 4 cg .. +3
   const int64_t per = (T + kWrSplit - 1) / kWrSplit;
   const int64_t ta = split * per;
   const int64_t tb = (ta + per) < T ? (ta + per) : T;
-  float acc[8][8];
+  float acc[8][4];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-  const bool active = (col < d) && (eg * 8 < E);
-  if (active) {
-    for (int64_t t = ta; t < tb; ++t) {
-      float xv[8];
-      load8<T_>(x + t * d + col, xv);
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+  for (int64_t tc = ta; tc < tb; tc += kWrTok) {
+    const int nt = static_cast<int>((tb - tc) < kWrTok ? (tb - tc) : kWrTok);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kWrTok * 64; i += blockDim.x) {
+      const int r = i >> 6, e = i & 63;
+      sdh[r][e] = (r < nt && e0 + e < E) ? dh[(tc + r) * E + e0 + e] : 0.f;
+    }
+    for (int i = threadIdx.x; i < kWrTok * 32; i += blockDim.x) {
+      const int r = i >> 5, c = (i & 31) * 4;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (r < nt && c0 + c < d) load4<T_>(x + (tc + r) * d + c0 + c, v);
+      *reinterpret_cast<float4*>(&sx[r][c]) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+    __syncthreads();
+    for (int r = 0; r < nt; ++r) {
+      const float4 xv = *reinterpret_cast<const float4*>(&sx[r][4 * cg]);
+      const float4 g0 = *reinterpret_cast<const float4*>(&sdh[r][8 * eg]);
+      const float4 g1 = *reinterpret_cast<const float4*>(&sdh[r][8 * eg + 4]);
+      const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
       for (int a = 0; a < 8; ++a) {
-        const int e = eg * 8 + a;
-        const float g = (e < E) ? dh[t * E + e] : 0.f;
-#pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(g, xv[b], acc[a][b]);
+        acc[a][0] = fmaf(g[a], xv.x, acc[a][0]);
+        acc[a][1] = fmaf(g[a], xv.y, acc[a][1]);
+        acc[a][2] = fmaf(g[a], xv.z, acc[a][2]);
+        acc[a][3] = fmaf(g[a], xv.w, acc[a][3]);
       }
     }
-    for (int a = 0; a < 8; ++a) {
-      const int e = eg * 8 + a;
-      if (e >= E) break;
-      float* dst = part + (static_cast<int64_t>(split) * E + e) * d + col;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) dst[b] = acc[a][b];
-    }
+  }
+  const int col = c0 + 4 * cg;
+  if (col >= d) return;
+  for (int a = 0; a < 8; ++a) {
+    const int e = e0 + 8 * eg + a;
+    if (e >= E) break;
+    *reinterpret_cast<float4*>(part + (static_cast<int64_t>(split) * E + e) * d + col) =
+        make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
   }
 }
 
@@ -256,8 +318,8 @@ cudaError_t launch_router_backward(const Shape& s, const float* dw, const int32_
 
 cudaError_t launch_dx_combine(const Shape& s, const void* dx_perm, const int32_t* inv_perm, const float* dh,
                               const void* w_router, void* dx, cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>((s.T + kDxTok - 1) / kDxTok);
-  const int threads = s.d / 8 < 256 ? s.d / 8 : 256;
+  const dim3 grid(static_cast<unsigned>((s.T + kDxRows - 1) / kDxRows), static_cast<unsigned>((s.d + kDxCols - 1) / kDxCols));
+  const int threads = 256;
   if (s.fp32)
     dx_kernel<float><<<grid, threads, 0, st>>>(static_cast<const float*>(dx_perm), inv_perm, dh,
                                                static_cast<const float*>(w_router), s.T, s.d, s.E, s.k,
@@ -271,7 +333,7 @@ cudaError_t launch_dx_combine(const Shape& s, const void* dx_perm, const int32_t
 
 cudaError_t launch_router_weight_grad(const Shape& s, const float* dh, const void* x, void* dw_router, float* part,
                                       cudaStream_t st) {
-  dim3 grid((s.d + 255) / 256, kWrSplit, (s.E + 63) / 64);
+  dim3 grid((s.d + 127) / 128, kWrSplit, (s.E + 63) / 64);
   if (s.fp32)
     router_wgrad_partial<float><<<grid, 256, 0, st>>>(dh, static_cast<const float*>(x), s.T, s.d, s.E, part);
   else
