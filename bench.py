@@ -551,14 +551,18 @@ def run_b200(args, rank, world, local):
         "gpu_launches": KERNELS_PER_STEP * K,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_extras:
+    extras = [] if args.no_extras else [e for e in args.extras.split(",") if e]
+    if world == 1 and extras:
         # the other OLMoE-shape workloads on this GPU, each reported beside the headline
-        line["decode"] = bench_decode(M, S, dev, (wr, wgu, wd), 200, peaks)
+        if "decode" in extras:
+            line["decode"] = bench_decode(M, S, dev, (wr, wgu, wd), 200, peaks)
         del x, wr, wgu, wd, ws, y
         torch.cuda.empty_cache()
-        line["train"] = bench_train(M, S, dev, 10, peaks)
-        torch.cuda.empty_cache()
-        line["stack"] = bench_stack(M, S, dev, 5, peaks)
+        if "train" in extras:
+            line["train"] = bench_train(M, S, dev, 10, peaks)
+            torch.cuda.empty_cache()
+        if "stack" in extras:
+            line["stack"] = bench_stack(M, S, dev, 5, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, n, times, threads = oracle_sample(4096, args.cpu_budget / 2, steps=2)
         line["cpu_baseline"] = {
@@ -582,6 +586,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the decode, training-step and 16-layer stack workloads (run at N=1 only)")
+    ap.add_argument("--extras", default="decode,train,stack",
+                    help="comma list of the extra workloads to run at N=1 (decode, train, stack)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args(argv)
     rank, world, local = dist_env()
