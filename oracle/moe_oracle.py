@@ -55,6 +55,7 @@ __all__ = [
     "router_logits",
     "softmax_lse",
     "topk_no_renorm",
+    "topk_renorm",
     "near_tie_tokens",
     "load_balance_loss",
     "router_z_loss",
@@ -126,6 +127,20 @@ def topk_no_renorm(p, k):
     p = _f64(p)
     order = np.argsort(-p, axis=1, kind="stable")[:, :k]
     return order.astype(np.int64), np.take_along_axis(p, order, axis=1)
+
+
+def topk_renorm(p, k):
+    """The same choice as topk_no_renorm, with the k weights renormalised to sum
+    to one: w_tj = p_tj / sum_j' p_tj'.
+
+    [OLMoE-Guide] "Top-8 Softmax Routing Formulation" writes the router as a
+    softmax over the k largest logits; dividing the k chosen probabilities by
+    their sum is the same thing ([MoE-scratch] §2, the router-variants table:
+    "softmax, top-k, renormalise" and "top-k, softmax" agree). OLMoE itself does
+    not renormalise; this is the variant behind the library's router mode 1.
+    """
+    idx, w = topk_no_renorm(p, k)
+    return idx, w / w.sum(axis=1, keepdims=True)
 
 
 def near_tie_tokens(p, k, rel=1e-6):
@@ -283,8 +298,9 @@ def experts_dense(x, idx, w, w_gate_up, w_down):
 # --------------------------------------------------------------------------- layer
 
 
-def moe_forward(x, w_router, w_gate_up, w_down, k, router_bias=None, store=None):
+def moe_forward(x, w_router, w_gate_up, w_down, k, router_bias=None, store=None, renorm=False):
     """The whole layer: route, dispatch, experts, combine, and the two losses.
+    `renorm` selects topk_renorm's weights (the choice and both losses are unchanged).
 
     Returns a dict with
       y [T,d], idx [T,k], w [T,k], p [T,E], lse [T], h [T,E],
@@ -293,7 +309,7 @@ def moe_forward(x, w_router, w_gate_up, w_down, k, router_bias=None, store=None)
     n_experts = _f64(w_router).shape[0]
     h = router_logits(x, w_router, router_bias)
     p, lse = softmax_lse(h)
-    idx, w = topk_no_renorm(p, k)
+    idx, w = topk_renorm(p, k) if renorm else topk_no_renorm(p, k)
     y = experts_grouped(x, idx, w, w_gate_up, w_down, store)
     L_lb, counts = load_balance_loss(idx, p, n_experts)
     perm, _, offsets = dispatch_order(idx, n_experts)
@@ -313,19 +329,19 @@ def moe_forward(x, w_router, w_gate_up, w_down, k, router_bias=None, store=None)
     }
 
 
-def moe_objective(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias=None):
+def moe_objective(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias=None, renorm=False):
     """The scalar whose gradient the backward returns: <dy, y> + alpha*L_lb + beta*L_z.
 
     [OLMoE-Guide] "Router Mechanics & Loss Formulations": L = L_LM + alpha*L_balance
     + beta*L_router_z; [OLMoE-paper] 4.1.6 and 4.1.7 fix alpha = 0.01, beta = 0.001.
     The upstream gradient dy stands in for dL_LM/dy.
     """
-    out = moe_forward(x, w_router, w_gate_up, w_down, k, router_bias)
+    out = moe_forward(x, w_router, w_gate_up, w_down, k, router_bias, renorm=renorm)
     return float(np.sum(_f64(dy) * out["y"])) + alpha * out["L_lb"] + beta * out["L_z"]
 
 
 def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias=None,
-                 experts=None, store=None):
+                 experts=None, store=None, renorm=False):
     """Gradients of moe_objective with respect to x and the three weights.
 
     Chain rule through each step of moe_forward (f and the choice carry none):
@@ -340,13 +356,16 @@ def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias
     `experts` optionally restricts which experts' weight gradients are formed
     (the rest are left zero); dx and dW_r always use every expert. `store`
     (see the module notes) rounds h, o, the saved a and b, do and [da; db].
+    With `renorm` the weights are w_tj = p_tj / s_t (s_t the sum of the chosen
+    p), so the chosen probabilities receive dp_ti = (dw_tj - sum_j' dw_tj' w_tj') / s_t
+    for i = S_tj instead of dw_tj.
     Returns dict dx [T,d], dw_router [E,d], dw_gate_up [E,2f,d], dw_down [E,d,f],
     plus the forward dict under "fwd" and dw [T,k].
     """
     x = _f64(x)
     dy = _f64(dy)
     S = _store(store)
-    fwd = moe_forward(x, w_router, w_gate_up, w_down, k, router_bias, store)
+    fwd = moe_forward(x, w_router, w_gate_up, w_down, k, router_bias, store, renorm)
     idx, w, p, lse = fwd["idx"], fwd["w"], fwd["p"], fwd["lse"]
     T, d = x.shape
     n_experts = _f64(w_router).shape[0]
@@ -388,7 +407,12 @@ def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias
         dx[tok] += da @ wgu[:f] + db @ wgu[f:]
 
     dp = np.zeros((T, n_experts))
-    np.add.at(dp, (np.arange(T)[:, None].repeat(k, axis=1), idx), dw)
+    if renorm:
+        s_chosen = np.take_along_axis(p, idx, axis=1).sum(axis=1, keepdims=True)
+        dsel = (dw - np.sum(dw * w, axis=1, keepdims=True)) / s_chosen
+        np.add.at(dp, (np.arange(T)[:, None].repeat(k, axis=1), idx), dsel)
+    else:
+        np.add.at(dp, (np.arange(T)[:, None].repeat(k, axis=1), idx), dw)
     frac = counts / float(T * k)
     dp += alpha * n_experts * frac[None, :] / T
     dh = p * (dp - np.sum(dp * p, axis=1, keepdims=True))

@@ -72,9 +72,11 @@ def test_router_variants_worked_example():
     ref_w = np.array([[m[e] for e in row] for m, row in zip(ref_by_expert, idx.tolist())])
     assert f"{np.abs(w - ref_w).max():.2e}" == table["softmax_topk"][1]
     assert f"{w.sum(axis=1).mean():.3f}" == table["softmax_topk"][2]
-    renorm = w / w.sum(axis=1, keepdims=True)
+    idx_r, renorm = O.topk_renorm(p, 8)
+    assert np.array_equal(idx_r, idx)
     # exact identity in real arithmetic; the page's 1.79e-07 is its fp32 rounding
     assert np.abs(renorm - ref_w).max() < 1e-12
+    assert np.allclose(renorm.sum(axis=1), 1.0, atol=1e-14, rtol=0)
     assert float(table["softmax_topk_renorm"][1]) < 1e-6
 
 
@@ -276,8 +278,8 @@ def test_olmoe_parameter_counts():
 # ------------------------------------------------------------------ gradients
 
 
-def _fd_check(L, dy, alpha, beta, name, seed, eps=1e-6):
-    g = O.moe_backward(dy=dy, alpha=alpha, beta=beta, **L)
+def _fd_check(L, dy, alpha, beta, name, seed, eps=1e-6, renorm=False):
+    g = O.moe_backward(dy=dy, alpha=alpha, beta=beta, renorm=renorm, **L)
     assert not g["fwd"]["near_tie"].any()
     r = _rng(seed)
     key = {"x": "dx", "w_router": "dw_router", "w_gate_up": "dw_gate_up",
@@ -288,8 +290,8 @@ def _fd_check(L, dy, alpha, beta, name, seed, eps=1e-6):
         Lp[name] = L[name] + eps * v
         Lm = dict(L)
         Lm[name] = L[name] - eps * v
-        jp = O.moe_objective(dy=dy, alpha=alpha, beta=beta, **Lp)
-        jm = O.moe_objective(dy=dy, alpha=alpha, beta=beta, **Lm)
+        jp = O.moe_objective(dy=dy, alpha=alpha, beta=beta, renorm=renorm, **Lp)
+        jm = O.moe_objective(dy=dy, alpha=alpha, beta=beta, renorm=renorm, **Lm)
         # the choice must not change inside the step, or the difference is meaningless
         ip = O.moe_forward(**Lp)["idx"]
         im = O.moe_forward(**Lm)["idx"]
@@ -305,6 +307,13 @@ def test_gradients_by_finite_differences(name):
     dy = _rng(10).standard_normal((12, 16))
     # alpha, beta far above OLMoE's so the loss terms are visible in the check
     _fd_check(L, dy, alpha=0.7, beta=0.3, name=name, seed=11)
+
+
+@pytest.mark.parametrize("name", ["x", "w_router", "w_gate_up"])
+def test_renormalised_router_gradients_by_finite_differences(name):
+    L = _small_layer(26, T=12, d=16, E=8, k=3, f=6, std=0.4)
+    dy = _rng(27).standard_normal((12, 16))
+    _fd_check(L, dy, alpha=0.7, beta=0.3, name=name, seed=28, renorm=True)
 
 
 def test_loss_gradients_alone_by_finite_differences():
