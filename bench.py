@@ -249,6 +249,16 @@ def oracle_sample(n_tokens_max, budget_s, steps=None, seed=1):
     return n / statistics.mean(times), n, times, threads
 
 
+def workload_config(T, world, d=2048, E=64, k=8, f=1024):
+    """The `config` object of the bench line (both arms)."""
+    return {
+        "workload": WORKLOAD if T == 4096 else WORKLOAD.replace("T=4096 (1x4096 context)", f"T={T}"),
+        "T": T, "d_model": d, "n_experts": E, "top_k": k, "d_ff": f,
+        "global_batch_tokens": world * T, "parallelism": f"replicas{world}",
+        "l2": "no flush: each step reads 805 MB of expert weights, above the 126 MB L2",
+    }
+
+
 def run_reference(args, rank, world):
     """The reference arm: the oracle on the host cores (rank 0 only)."""
     if rank != 0:
@@ -259,11 +269,11 @@ def run_reference(args, rank, world):
     value = n / statistics.mean(timed)
     sample = f"{n} contiguous tokens of the T=4096 workload per step (routing, experts, losses), fp64"
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(timed) * 4096 / n,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": WORKLOAD, "T": 4096, "sample_tokens": n},
+        "config": dict(workload_config(4096, world), sample_tokens=n),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -526,12 +536,7 @@ def run_b200(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": WORKLOAD if T == 4096 else WORKLOAD.replace("T=4096 (1x4096 context)", f"T={T}"),
-            "T": T, "d_model": d, "n_experts": E, "top_k": k, "d_ff": f,
-            "global_batch_tokens": world * T, "parallelism": f"replicas{world}",
-            "l2": "no flush: each step reads 805 MB of expert weights, above the 126 MB L2",
-        },
+        "config": workload_config(T, world, d, E, k, f),
         "tflops": layer_tflops,
         "layer_roofline": {
             "floor_ms_nominal": floor_ms_nominal, "frac_nominal": floor_ms_nominal / ms_max,

@@ -50,7 +50,7 @@ extern "C" {
 struct CUstream_st;
 typedef struct CUstream_st* cudaStream_t;
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 #define MOE_ROW_ALIGN 128
 
 typedef enum moe_status {
@@ -64,6 +64,14 @@ typedef enum moe_status {
 } moe_status;
 
 typedef enum moe_dtype { MOE_BF16 = 0, MOE_FP32 = 1 } moe_dtype;
+
+/* Router weights. MOE_ROUTER_SOFTMAX_TOPK (OLMoE, the default): softmax over
+ * all experts, the k largest probabilities are both the choice and the weights,
+ * not renormalised ("Mixture-of-experts LLMs from scratch with OLMoE", sections
+ * 2 and 3, norm_topk_prob False). MOE_ROUTER_RENORM: the same choice, weights
+ * divided by their sum, i.e. a softmax over the k largest logits ("OLMoE Guide",
+ * "Top-8 Softmax Routing Formulation"). Losses are the same in both modes. */
+typedef enum moe_router_mode { MOE_ROUTER_SOFTMAX_TOPK = 0, MOE_ROUTER_RENORM = 1 } moe_router_mode;
 
 /* Shapes and loss weights of one layer. Supported: 1 <= T <= 2^24;
  * d_model a multiple of 128 in [128, 4096] (bf16) or [128, 2048] (fp32);
@@ -85,6 +93,7 @@ typedef struct moe_config {
   float alpha_lb;
   float beta_z;
   int32_t grad_dtype; /* moe_dtype of dw_router, dw_gate_up, dw_down */
+  int32_t router_mode; /* moe_router_mode */
 } moe_config;
 
 /* Human-readable name of a status code. Never NULL. */
@@ -252,6 +261,19 @@ moe_status moe_stack_forward(const moe_config* cfg, int32_t n_layers, const void
                              const float* const* router_biases, const void* const* w_gate_up,
                              const void* const* w_down, float* resid, void* ws, size_t ws_bytes,
                              cudaStream_t stream);
+
+/* moe_stack_forward that also exports, per layer, what the router did ("Mixture-
+ * of-experts LLMs from scratch with OLMoE", section 3 MoE.forward's routing
+ * trace and section 6's per-layer expert usage). Each output may be NULL:
+ *   counts    [device] [n_layers, E] int32: rows routed to each expert;
+ *   losses    [device] [n_layers, 2] fp32: L_lb and L_z of each layer;
+ *   topk_idx  [device] [n_layers, T, k] int32: the experts each token chose, in
+ *             slot order (descending probability).
+ * The residual stream is bit-identical to moe_stack_forward's. */
+moe_status moe_stack_forward_trace(const moe_config* cfg, int32_t n_layers, const void* const* w_router,
+                                   const float* const* router_biases, const void* const* w_gate_up,
+                                   const void* const* w_down, float* resid, int32_t* counts, float* losses,
+                                   int32_t* topk_idx, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Stage timing for profiling. When `events` is non-NULL, the next call of
  * moe_forward records events[0] on its stream before the router and events[i]

@@ -32,6 +32,7 @@ from .binding import (  # noqa: F401
     moe_route_static,
     moe_set_stage_events,
     moe_stack_forward,
+    moe_stack_forward_trace,
     moe_workspace_bytes,
     moe_workspace_init,
     status_string,

@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_BF16 = 0
 MOE_FP32 = 1
+MOE_ROUTER_SOFTMAX_TOPK = 0
+MOE_ROUTER_RENORM = 1
 ROW_ALIGN = 128
 
 STATUS_NAMES = {
@@ -37,7 +39,7 @@ EXPORTS = (
     "moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_route_static", "moe_dispatch",
     "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_forward",
     "moe_forward_host", "moe_backward", "moe_rmsnorm", "moe_combine_residual",
-    "moe_stack_forward", "moe_set_stage_events", "moe_get_device_status",
+    "moe_stack_forward", "moe_stack_forward_trace", "moe_set_stage_events", "moe_get_device_status",
 )
 STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "gate_up", "down", "combine")
@@ -60,6 +62,7 @@ class moe_config(ctypes.Structure):
         ("alpha_lb", ctypes.c_float),
         ("beta_z", ctypes.c_float),
         ("grad_dtype", ctypes.c_int32),
+        ("router_mode", ctypes.c_int32),
     ]
 
 
@@ -88,6 +91,8 @@ _SIGS = {
     "moe_combine_residual": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
     "moe_stack_forward": (ctypes.c_int, [_CFG, ctypes.c_int32, _P, _P, _P, _P, _P, _P,
                                          ctypes.c_size_t, _P]),
+    "moe_stack_forward_trace": (ctypes.c_int, [_CFG, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                               ctypes.c_size_t, _P]),
     "moe_set_stage_events": (ctypes.c_int, [_P]),
     "moe_get_device_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), _P]),
 }
@@ -120,16 +125,17 @@ def _check(status, where):
 
 
 def config(T, d_model, n_experts, top_k, d_ff, dtype=torch.bfloat16, alpha_lb=0.01, beta_z=0.001,
-           grad_dtype=None):
+           grad_dtype=None, renorm=False):
     """A moe_config. `dtype` is torch.bfloat16 or torch.float32; `grad_dtype`, the
-    type of the weight gradients moe_backward writes, defaults to `dtype`."""
+    type of the weight gradients moe_backward writes, defaults to `dtype`;
+    `renorm` selects the renormalised top-k weights (MOE_ROUTER_RENORM)."""
     grad_dtype = dtype if grad_dtype is None else grad_dtype
     for t in (dtype, grad_dtype):
         if t not in (torch.bfloat16, torch.float32):
             raise ValueError("dtypes must be torch.bfloat16 or torch.float32")
     code = lambda t: MOE_BF16 if t == torch.bfloat16 else MOE_FP32
     return moe_config(int(T), int(d_model), int(n_experts), int(top_k), int(d_ff), code(dtype), float(alpha_lb),
-                      float(beta_z), code(grad_dtype))
+                      float(beta_z), code(grad_dtype), 1 if renorm else 0)
 
 
 def torch_dtype(cfg) -> torch.dtype:
@@ -355,6 +361,27 @@ def moe_backward(cfg, dy, x, w_router, w_gate_up, w_down, dx, dw_router, dw_gate
     _check(st, "moe_backward")
 
 
+def moe_stack_forward_trace(cfg, layers, resid, ws, counts=None, losses=None, topk_idx=None, stream=None):
+    """moe_stack_forward that also fills, when given, counts [L, E] int32,
+    losses [L, 2] fp32 and topk_idx [L, T, k] int32 (device tensors)."""
+    dt = torch_dtype(cfg)
+    T, d, E, k, f = cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff
+    n = len(layers)
+    arr = ctypes.c_void_p * n
+    wr = arr(*[_ptr(L["w_router"], dt, (E, d), "w_router") for L in layers])
+    wgu = arr(*[_ptr(L["w_gate_up"], dt, (E, 2 * f, d), "w_gate_up") for L in layers])
+    wd = arr(*[_ptr(L["w_down"], dt, (E, d, f), "w_down") for L in layers])
+    bs = arr(*[_ptr(L.get("router_bias"), torch.float32, (E,), "router_bias", allow_none=True)
+               for L in layers])
+    st = lib().moe_stack_forward_trace(
+        _cfgp(cfg), n, wr, bs, wgu, wd, _ptr(resid, torch.float32, (T, d), "resid"),
+        _ptr(counts, torch.int32, (n, E), "counts", allow_none=True),
+        _ptr(losses, torch.float32, (n, 2), "losses", allow_none=True),
+        _ptr(topk_idx, torch.int32, (n, T, k), "topk_idx", allow_none=True),
+        _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
+    _check(st, "moe_stack_forward_trace")
+
+
 def moe_stack_forward(cfg, layers, resid, ws, stream=None):
     """`layers`: list of dicts with w_router, w_gate_up, w_down and optional router_bias
     (device tensors). `resid` [T, d] fp32 is updated in place."""
@@ -404,18 +431,20 @@ class MoELayer:
     """
 
     def __init__(self, w_router, w_gate_up, w_down, router_bias=None, top_k=8, alpha_lb=0.01,
-                 beta_z=0.001, grad_dtype=None):
+                 beta_z=0.001, grad_dtype=None, renorm=False):
         self.w_router, self.w_gate_up, self.w_down = w_router, w_gate_up, w_down
         self.router_bias = router_bias
         self.top_k = top_k
         self.alpha_lb, self.beta_z = alpha_lb, beta_z
         self.grad_dtype = grad_dtype
+        self.renorm = renorm
         self._ws = {}
 
     def cfg(self, T):
         E, d = self.w_router.shape
         f = self.w_down.shape[2]
-        return config(T, d, E, self.top_k, f, self.w_router.dtype, self.alpha_lb, self.beta_z, self.grad_dtype)
+        return config(T, d, E, self.top_k, f, self.w_router.dtype, self.alpha_lb, self.beta_z, self.grad_dtype,
+                      self.renorm)
 
     def ws(self, T, train):
         key = (T, bool(train))

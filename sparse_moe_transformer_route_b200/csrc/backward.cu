@@ -92,10 +92,30 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     router_bwd_kernel(const float* __restrict__ dw, const int32_t* __restrict__ idx, const float* __restrict__ probs,
                       const float* __restrict__ lse, const int32_t* __restrict__ counts, int64_t T, int E, int k,
-                      float alpha, float beta, float* __restrict__ dh) {
+                      float alpha, float beta, int renorm, float* __restrict__ dh) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp;
   if (t >= T) return;
+  // Renormalised weights w_j = p_j / s (s = sum of the chosen p): the chosen
+  // probabilities receive (dw_j - <dw, w>) / s instead of dw_j. Lane j < k holds
+  // slot j; the two sums use a fixed butterfly.
+  float inv_s = 1.f, shift = 0.f;
+  if (renorm) {
+    float pj = 0.f, dwj = 0.f;
+    if (lane < k) {
+      const int e = idx[t * k + lane];
+      pj = (e >= 0 && e < E) ? probs[t * E + e] : 0.f;
+      dwj = dw[t * k + lane];
+    }
+    float ssum = pj, wdot = dwj * pj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+      wdot += __shfl_xor_sync(0xffffffffu, wdot, o);
+    }
+    inv_s = ssum > 0.f ? 1.f / ssum : 0.f;
+    shift = wdot * inv_s;  // <dw, w>
+  }
   constexpr int Q = kMaxExperts / 32;
   const float Tf = static_cast<float>(T);
   float dp[Q], p[Q];
@@ -109,7 +129,7 @@ __global__ void __launch_bounds__(256)
       p[q] = probs[t * E + e];
       float g = alpha * static_cast<float>(E) * (static_cast<float>(counts[e]) / (Tf * k)) / Tf;
       for (int j = 0; j < k; ++j)
-        if (idx[t * k + j] == e) g += dw[t * k + j];
+        if (idx[t * k + j] == e) g += renorm ? (dw[t * k + j] - shift) * inv_s : dw[t * k + j];
       dp[q] = g;
       dot = fmaf(g, p[q], dot);
     }
@@ -312,7 +332,8 @@ cudaError_t launch_router_backward(const Shape& s, const float* dw, const int32_
                                    const float* lse, const int32_t* counts, float alpha, float beta, float* dh,
                                    cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((s.T + 7) / 8);
-  router_bwd_kernel<<<grid, 256, 0, st>>>(dw, idx, probs, lse, counts, s.T, s.E, s.k, alpha, beta, dh);
+  router_bwd_kernel<<<grid, 256, 0, st>>>(dw, idx, probs, lse, counts, s.T, s.E, s.k, alpha, beta,
+                                          s.renorm ? 1 : 0, dh);
   return cudaGetLastError();
 }
 

@@ -46,6 +46,7 @@ bool make_shape(const moe_config* cfg, Shape* s) {
   if (cfg == nullptr) return false;
   if (cfg->dtype != MOE_BF16 && cfg->dtype != MOE_FP32) return false;
   if (cfg->grad_dtype != MOE_BF16 && cfg->grad_dtype != MOE_FP32) return false;
+  if (cfg->router_mode != MOE_ROUTER_SOFTMAX_TOPK && cfg->router_mode != MOE_ROUTER_RENORM) return false;
   const bool fp32 = cfg->dtype == MOE_FP32;
   const int dmax = fp32 ? 2048 : 4096;
   if (cfg->T < 1 || cfg->T > (int64_t(1) << 24)) return false;
@@ -60,6 +61,7 @@ bool make_shape(const moe_config* cfg, Shape* s) {
   s->f = cfg->d_ff;
   s->fp32 = fp32;
   s->grad32 = fp32 || cfg->grad_dtype == MOE_FP32;
+  s->renorm = cfg->router_mode == MOE_ROUTER_RENORM;
   s->esize = fp32 ? 4 : 2;
   s->P = static_cast<int64_t>(up(static_cast<size_t>(cfg->T * cfg->top_k + int64_t(cfg->n_experts) * (kRowAlign - 1)),
                                  kRowAlign));
@@ -158,7 +160,7 @@ struct StageMarks {
 
 moe_status forward_impl(const Ctx& c, const void* x, const void* w_router, const float* bias, const void* w_gate_up,
                         const void* w_down, void* y, float* losses, float* resid, int32_t* topk_idx, float* topk_w,
-                        bool save, void* ws, cudaStream_t st) {
+                        bool save, void* ws, cudaStream_t st, int32_t* counts = nullptr) {
   const Shape& s = c.s;
   const Workspace& L = c.L;
   int32_t* status = at<int32_t>(ws, L.ctrl);
@@ -171,11 +173,11 @@ moe_status forward_impl(const Ctx& c, const void* x, const void* w_router, const
   MOE_TRY(marks.mark(0));
   if (router_tc_supported(s)) {
     // the tensor-core router also leaves the dispatch ranking in ws
-    MOE_TRY(launch_router_tc(s, x, w_router, bias, idx, wts, nullptr, losses, ws, L, st));
+    MOE_TRY(launch_router_tc(s, x, w_router, bias, idx, wts, counts, losses, ws, L, st));
     MOE_TRY(marks.mark(1));
     MOE_TRY(launch_permute(s, idx, x, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv_perm), x_perm, ws, L, save, st));
   } else {
-    MOE_TRY(launch_router(s, x, w_router, bias, idx, wts, nullptr, losses, ws, L, st));
+    MOE_TRY(launch_router(s, x, w_router, bias, idx, wts, counts, losses, ws, L, st));
     MOE_TRY(marks.mark(1));
     MOE_TRY(launch_dispatch_impl(s, idx, x, nullptr, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv_perm), nullptr,
                                  x_perm, ws, L, save, st));
@@ -412,10 +414,10 @@ moe_status moe_rmsnorm(const moe_config* cfg, const float* resid, const float* w
   return MOE_OK;
 }
 
-moe_status moe_stack_forward(const moe_config* cfg, int32_t n_layers, const void* const* w_router,
-                             const float* const* router_biases, const void* const* w_gate_up,
-                             const void* const* w_down, float* resid, void* ws, size_t ws_bytes,
-                             cudaStream_t stream) {
+moe_status moe_stack_forward_trace(const moe_config* cfg, int32_t n_layers, const void* const* w_router,
+                                   const float* const* router_biases, const void* const* w_gate_up,
+                                   const void* const* w_down, float* resid, int32_t* counts, float* losses,
+                                   int32_t* topk_idx, void* ws, size_t ws_bytes, cudaStream_t stream) {
   Ctx c;
   moe_status r = prepare(cfg, ws, ws_bytes, false, &c);
   if (r != MOE_OK) return r;
@@ -425,14 +427,25 @@ moe_status moe_stack_forward(const moe_config* cfg, int32_t n_layers, const void
   for (int l = 0; l < n_layers; ++l)
     if (w_router[l] == nullptr || w_gate_up[l] == nullptr || w_down[l] == nullptr) return MOE_ERR_INVALID_ARG;
   void* xn = at<void>(ws, c.L.x_dev);
+  const int64_t tk = c.s.T * c.s.k;
   for (int l = 0; l < n_layers; ++l) {
     MOE_TRY(launch_rmsnorm(c.s, resid, nullptr, 1e-5f, xn, stream));
     const float* bias = (router_biases != nullptr) ? router_biases[l] : nullptr;
-    r = forward_impl(c, xn, w_router[l], bias, w_gate_up[l], w_down[l], nullptr, nullptr, resid, nullptr, nullptr,
-                     false, ws, stream);
+    r = forward_impl(c, xn, w_router[l], bias, w_gate_up[l], w_down[l], nullptr,
+                     losses != nullptr ? losses + 2 * l : nullptr, resid,
+                     topk_idx != nullptr ? topk_idx + l * tk : nullptr, nullptr, false, ws, stream,
+                     counts != nullptr ? counts + static_cast<int64_t>(l) * c.s.E : nullptr);
     if (r != MOE_OK) return r;
   }
   return MOE_OK;
+}
+
+moe_status moe_stack_forward(const moe_config* cfg, int32_t n_layers, const void* const* w_router,
+                             const float* const* router_biases, const void* const* w_gate_up,
+                             const void* const* w_down, float* resid, void* ws, size_t ws_bytes,
+                             cudaStream_t stream) {
+  return moe_stack_forward_trace(cfg, n_layers, w_router, router_biases, w_gate_up, w_down, resid, nullptr, nullptr,
+                                 nullptr, ws, ws_bytes, stream);
 }
 
 moe_status moe_set_stage_events(void* const* events) {

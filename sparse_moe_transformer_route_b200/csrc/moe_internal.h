@@ -23,6 +23,7 @@ struct Shape {
   int d, E, k, f;
   bool fp32;
   bool grad32;   // backward writes the weight gradients in fp32
+  bool renorm;   // router weights renormalised over the k chosen experts
   size_t esize;  // bytes per activation / weight element
   int64_t P;     // padded row capacity
   int64_t router_ctas() const { return (T + kRouterTokensPerCta - 1) / kRouterTokensPerCta; }

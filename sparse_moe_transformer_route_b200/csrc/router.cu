@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(kThreads) router_kernel(
     int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out, float* __restrict__ probs,
     float* __restrict__ lse_out, int32_t* __restrict__ counts_part, float* __restrict__ psum_part,
     double* __restrict__ zsum_part, int32_t* __restrict__ counts_ws, int32_t* __restrict__ counts_user,
-    float* __restrict__ losses_ws, float* __restrict__ losses_user, int32_t* __restrict__ ticket) {
+    float* __restrict__ losses_ws, float* __restrict__ losses_user, int32_t* __restrict__ ticket, int renorm) {
   extern __shared__ __align__(16) unsigned char smem[];
   Tin* xs = reinterpret_cast<Tin*>(smem);                                            // [kTok][d]
   double* logit = reinterpret_cast<double*>(smem + static_cast<size_t>(kTok) * d * sizeof(Tin));  // [kTok][E]
@@ -120,6 +120,7 @@ __global__ void __launch_bounds__(kThreads) router_kernel(
     const float lse = m + logf(s);
 
     uint32_t taken = 0;  // bit q: expert lane+32q already chosen
+    float chosen_sum = 0.f;  // renormalised weights: the chosen probabilities' sum, in slot order
     for (int j = 0; j < k; ++j) {
       double bv = -static_cast<double>(INFINITY);
       int bi = 0x7fffffff;
@@ -148,12 +149,15 @@ __global__ void __launch_bounds__(kThreads) router_kernel(
         if (q == qq) mine = p[q];
       const float pw = __shfl_sync(0xffffffffu, mine, bi & 31);
       if (bi >= 0 && lane == (bi & 31)) taken |= 1u << qq;
+      if (bi >= 0) chosen_sum += pw;
       if (lane == 0) {
         idx_out[tg * k + j] = bi;
         w_out[tg * k + j] = (bi >= 0) ? pw : 0.f;
         if (bi >= 0) atomicAdd(&cnt[bi], 1);
       }
     }
+    if (renorm && lane == 0 && chosen_sum > 0.f)
+      for (int j = 0; j < k; ++j) w_out[tg * k + j] = w_out[tg * k + j] / chosen_sum;
     if (lane == 0) {
       lses[t] = lse;
       lse_out[tg] = lse;
@@ -249,7 +253,8 @@ cudaError_t run(const Shape& s, const void* x, const void* w_router, const float
   router_kernel<Tin><<<grid, kThreads, smem, st>>>(
       static_cast<const Tin*>(x), static_cast<const Tin*>(w_router), bias, s.T, s.d, s.E, s.k, idx, wts,
       at<float>(ws, L.probs), at<float>(ws, L.lse), at<int32_t>(ws, L.counts_part), at<float>(ws, L.psum_part),
-      at<double>(ws, L.zsum_part), at<int32_t>(ws, L.counts), counts, at<float>(ws, L.losses), losses, ctrl + 1);
+      at<double>(ws, L.zsum_part), at<int32_t>(ws, L.counts), counts, at<float>(ws, L.losses), losses, ctrl + 1,
+      s.renorm ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -358,7 +363,7 @@ cudaError_t run_static(const Shape& s, const void* x, const void* w_router, cons
       reinterpret_cast<float*>(scratch + L.probs), reinterpret_cast<float*>(scratch + L.lse),
       reinterpret_cast<int32_t*>(scratch + L.counts_part), reinterpret_cast<float*>(scratch + L.psum_part),
       reinterpret_cast<double*>(scratch + L.zsum_part), reinterpret_cast<int32_t*>(scratch + L.counts), counts,
-      reinterpret_cast<float*>(scratch + L.losses), losses, ticket);
+      reinterpret_cast<float*>(scratch + L.losses), losses, ticket, s.renorm ? 1 : 0);
   return cudaGetLastError();
 }
 

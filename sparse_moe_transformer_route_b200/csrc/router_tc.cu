@@ -78,6 +78,9 @@ struct RArgs {
   int32_t* gs_ws;
   int32_t* ticket;
   int32_t* status;
+  float* logit_part;  // split form: [ksplit][T][E] partial logits
+  int ksplit;         // split form: K ranges per 128-token tile
+  int renorm;         // weights divided by the sum of the k chosen probabilities
 };
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -367,12 +370,21 @@ __device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& s
   }
   // ---- outputs: thread qp writes slots qp, qp+4, ...
   if (valid) {
+    // the weights' denominator: all experts' exponentials, or (renormalised)
+    // the k chosen ones summed in slot order
+    float den = s;
+    if (a.renorm) {
+      den = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j)
+        if (j < k) den += expf(hv[j] - m);
+    }
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
       if (j < k && (j & 3) == qp) {
         const int e = ord[j];
         a.idx_out[t * k + j] = e;
-        a.w_out[t * k + j] = expf(hv[j] - m) / s;
+        a.w_out[t * k + j] = expf(hv[j] - m) / den;
         chosen[r * kMaxTopK + j] = e;
         atomicOr(&mask[e], 1u << r);
       }
@@ -686,13 +698,12 @@ __global__ void __launch_bounds__(kThreads, MINB)
 
 
 // ------------------------------------------------------------------ split form
-// When the 32-token tiles outnumber the SMs the router runs as two kernels
-// (measured at T = 16384: 87 us against 102 us fused; at T = 4096, one wave,
-// the fused kernel is faster: 41 us against 51 us): logits for 128
-// tokens per CTA (the M=128 MMA then carries 128 real rows, so the tcgen05
-// issue cost, which bounds this phase, is spread over 4x the tokens), written
-// with the offset into the probability rows of the workspace; then the
-// epilogue above on 32-token tiles, several CTAs per SM.
+// Two kernels: logits for 128 tokens per CTA (the M=128 MMA then carries 128
+// real rows, so the tcgen05 issue cost, which bounds this phase, is spread
+// over 4x the tokens), with the K steps divided among `ksplit` CTAs per tile
+// when there are fewer tiles than SMs, as fp32 partials in the workspace; then
+// the epilogue above on 32-token tiles, two CTAs per SM, which sums the
+// partials in a fixed order.
 constexpr int kLogitTile = 128;
 constexpr int kLogitStages = 8;
 constexpr int kLogitStage = kLogitTile * 128 + kMaxE * 128;  // x rows, then W_r rows (per 64-wide K step)
@@ -714,7 +725,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = empty + kLogitStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nk = a.d / 64;
+  // this CTA's share of the 64-wide K steps
+  const int ks = blockIdx.y;
+  const int kb_lo = (ks * (a.d / 64)) / a.ksplit;
+  const int nk = ((ks + 1) * (a.d / 64)) / a.ksplit - kb_lo;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kLogitTile;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kLogitStages; ++s) {
@@ -748,8 +762,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         unsigned char* st = ring + static_cast<size_t>(s) * STAGE;
         mbar_arrive_expect_tx(&full[s], STAGE);
-        tma_load_2d(&tmx, &full[s], st, kc * 64, static_cast<int32_t>(t0));
-        tma_load_2d(&tmw, &full[s], st + kLogitTile * 128, kc * 64, 0);
+        tma_load_2d(&tmx, &full[s], st, (kb_lo + kc) * 64, static_cast<int32_t>(t0));
+        tma_load_2d(&tmw, &full[s], st + kLogitTile * 128, (kb_lo + kc) * 64, 0);
         ++issued;
         if (++s == kLogitStages) {
           s = 0;
@@ -801,10 +815,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c), v);
       tmem_ld_wait();
       if (t < a.T) {
+        float* dst = a.logit_part + (static_cast<int64_t>(ks) * a.T + t) * a.E;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int e = c + i;
-          if (e < a.E) a.probs[t * a.E + e] = __uint_as_float(v[i]) + (a.bias != nullptr ? a.bias[e] : 0.f);
+          if (e < a.E) dst[e] = __uint_as_float(v[i]);
         }
       }
     }
@@ -838,10 +853,24 @@ __global__ void __launch_bounds__(128, 2) router_epi_kernel(const RArgs a) {
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
   if (tid < kMaxE) mask[tid] = 0u;
   if (tid == 0) *qn = 0;
-  // this tile's logits (offset included) from the logits kernel
+  // this tile's logits: the K-range partials (all loads in flight, then summed
+  // in a fixed order), plus the offset
   for (int i = tid; i < kTile * kMaxE; i += 128) {
     const int r = i / kMaxE, e = i - r * kMaxE;
-    S[r * kLogitStride + e] = (t0 + r < a.T && e < a.E) ? a.probs[(t0 + r) * a.E + e] : -INFINITY;
+    float h = -INFINITY;
+    if (t0 + r < a.T && e < a.E) {
+      const float* src = a.logit_part + (t0 + r) * a.E + e;
+      const int64_t step = a.T * a.E;
+      float v[16];
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) v[ks] = (ks < a.ksplit) ? __ldcg(src + ks * step) : 0.f;
+      h = v[0];
+#pragma unroll
+      for (int ks = 1; ks < 16; ++ks)
+        if (ks < a.ksplit) h += v[ks];
+      if (a.bias != nullptr) h += a.bias[e];
+    }
+    S[r * kLogitStride + e] = h;
   }
   epi_sync();
   const EpiSmem sm{S, P, chosen, queue, exact, qn, mask, lse_s, s_last, tot, tot_p, zred, ring};
@@ -901,15 +930,34 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router
   a.gs_ws = at<int32_t>(ws, L.group_start);
   a.ticket = ctrl + 1;
   a.status = ctrl;
+  a.renorm = s.renorm ? 1 : 0;
   const unsigned grid = static_cast<unsigned>((s.T + kTile - 1) / kTile);
-  if (static_cast<int>(grid) <= device_sm_count()) {  // one wave: the fused kernel
+  // A few tokens: logits split over K among many CTAs, then the epilogue
+  // (T=1: 24.5 us against 28.7 us fused, warm; T=32: 32.8 against ~28.7).
+  // Up to one wave of 32-token tiles: the fused kernel (T=64: 28.7 us against
+  // 41.0 us split; T=4096: 40.9 us against 49.2 us). More tiles than SMs: the
+  // split form (T=16384: 87-94 us against 102 us fused).
+  if (s.T > 8 && static_cast<int>(grid) <= device_sm_count()) {
     router_tc_kernel<16, 1><<<grid, kThreads, smem_bytes(16), st>>>(tx, tw, a);
     return cudaGetLastError();
   }
   CUtensorMap tx128;
   if (!make_map(&tx128, x, false, static_cast<uint64_t>(s.T), s.d, 64, kLogitTile)) return cudaErrorInvalidValue;
   const unsigned grid_l = static_cast<unsigned>((s.T + kLogitTile - 1) / kLogitTile);
-  router_logits_kernel<<<grid_l, kThreads, kLogitSmem, st>>>(tx128, tw, a);
+  // K ranges per tile: enough CTAs to cover the SMs, at least two K steps each,
+  // and no more partials than the scratch (the permuted-rows region, unused yet) holds
+  int ks = device_sm_count() / static_cast<int>(grid_l);
+  ks = ks < 1 ? 1 : (ks > 16 ? 16 : ks);
+  while (ks > 1 && s.d / 64 / ks < 2) --ks;
+  const size_t cap = static_cast<size_t>(s.P) * s.d * s.esize;
+  while (ks > 1 && static_cast<size_t>(ks) * s.T * s.E * 4 > cap) --ks;
+  if (static_cast<size_t>(ks) * s.T * s.E * 4 > cap) {  // tiny layers: the fused kernel
+    router_tc_kernel<16, 1><<<grid, kThreads, smem_bytes(16), st>>>(tx, tw, a);
+    return cudaGetLastError();
+  }
+  a.logit_part = at<float>(ws, L.x_perm);
+  a.ksplit = ks;
+  router_logits_kernel<<<dim3(grid_l, static_cast<unsigned>(ks)), kThreads, kLogitSmem, st>>>(tx128, tw, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   router_epi_kernel<<<grid, 128, kEpiSmem, st>>>(a);

@@ -9,10 +9,10 @@ from oracle import moe_oracle as O
 from tests._parity import LazyF64, assert_close, assert_loss_close, f64, index_parity
 
 
-def run_forward(inp, train=False, bias=None):
+def run_forward(inp, train=False, bias=None, renorm=False):
     x, wr, wgu, wd = (t.cuda() for t in (inp.x, inp.w_router, inp.w_gate_up, inp.w_down))
     sh = inp.shape
-    cfg = M.config(sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff, x.dtype)
+    cfg = M.config(sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff, x.dtype, renorm=renorm)
     ws = M.workspace(cfg, train)
     y = torch.empty_like(x)
     losses = torch.empty(2, device="cuda")
@@ -25,7 +25,7 @@ def run_forward(inp, train=False, bias=None):
     return dict(cfg=cfg, ws=ws, y=y, losses=losses, idx=idx, w=w, dev=(x, wr, wgu, wd, b))
 
 
-def check_forward(inp, out, bias=None, sample=None):
+def check_forward(inp, out, bias=None, sample=None, renorm=False):
     """Routing for every token; outputs on `sample` tokens (all when None)."""
     x = f64(inp.x)
     wr = f64(inp.w_router)
@@ -34,7 +34,7 @@ def check_forward(inp, out, bias=None, sample=None):
     b = f64(bias) if bias is not None else None
     h = O.router_logits(x, wr, b)
     p, lse = O.softmax_lse(h)
-    ref_idx, ref_w = O.topk_no_renorm(p, k)
+    ref_idx, ref_w = O.topk_renorm(p, k) if renorm else O.topk_no_renorm(p, k)
     near = O.near_tie_tokens(p, k)
     gidx = out["idx"].cpu().numpy()
     bad, n_near, diff = index_parity(gidx, ref_idx, near)

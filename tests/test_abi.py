@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol():
 def test_library_has_no_gpu_only_load_dependencies():
     # static CUDA runtime: the .so must load here, where there is no driver
     lib = M.lib()
-    assert lib.moe_abi_version() == 2
+    assert lib.moe_abi_version() == 3
 
 
 def test_status_strings():
@@ -65,10 +65,14 @@ def test_config_validation():
         M.config(16, 2048, 300, 8, 1024),          # E > 256
         M.config(16, 4096, 64, 8, 1024, torch.float32),  # fp32 router tile limit
     ]
+    odd = M.config(16, 2048, 64, 8, 1024)
+    odd.router_mode = 2                            # no such router mode
+    bad.append(odd)
     for cfg in bad:
         assert M.moe_check_config(cfg) == 2
         assert M.moe_workspace_bytes(cfg) == 0
         assert M.moe_padded_rows(cfg) == -1
+    assert M.moe_check_config(M.config(16, 2048, 64, 8, 1024, renorm=True)) == 0
 
 
 @pytest.mark.parametrize("T,E,k", [(1, 64, 8), (128, 64, 8), (4096, 64, 8), (300, 16, 4)])

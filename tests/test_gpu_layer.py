@@ -147,10 +147,10 @@ def test_host_buffer_entry_point_matches_device():
     assert torch.equal(yh, a["y"].cpu()) and torch.equal(lh, a["losses"].cpu())
 
 
-def check_backward(inp, alpha=0.01, beta=0.001, experts=None, tol_scale=1.0):
+def check_backward(inp, alpha=0.01, beta=0.001, experts=None, tol_scale=1.0, renorm=False):
     sh = inp.shape
     x, wr, wgu, wd, dy = (t.cuda() for t in (inp.x, inp.w_router, inp.w_gate_up, inp.w_down, inp.dy))
-    cfg = M.config(sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff, x.dtype, alpha, beta)
+    cfg = M.config(sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff, x.dtype, alpha, beta, renorm=renorm)
     ws = M.workspace(cfg, True)
     y = torch.empty_like(x)
     losses = torch.empty(2, device="cuda")
@@ -162,7 +162,7 @@ def check_backward(inp, alpha=0.01, beta=0.001, experts=None, tol_scale=1.0):
     torch.cuda.synchronize()
     assert M.moe_get_device_status(ws) == 0
     ref = O.moe_backward(f64(inp.x), f64(inp.w_router), LazyF64(inp.w_gate_up), LazyF64(inp.w_down), sh.top_k,
-                         f64(inp.dy), alpha, beta, experts=experts)
+                         f64(inp.dy), alpha, beta, experts=experts, renorm=renorm)
     # gradients sum over tokens, so the routing must agree on every token (near-ties
     # included: the router decides on logits accumulated in fp64 from exact products)
     assert np.array_equal(idx.cpu().numpy(), ref["fwd"]["idx"]), "routing differs from the oracle"
@@ -206,3 +206,23 @@ def test_backward_loss_terms_alone():
     inp = S.layer_inputs(sh, seed=21, dtype=torch.bfloat16, with_grad=True)
     inp.dy = torch.zeros_like(inp.dy)
     check_backward(inp, alpha=0.5, beta=0.25)
+
+
+# ------------------------------------------------------------------ renormalised router
+
+
+@pytest.mark.parametrize("T,d,E,k,f,dtype", [(128, 512, 64, 8, 256, torch.float32),   # SIMT router
+                                             (1000, 512, 64, 8, 256, torch.bfloat16),  # tensor-core router
+                                             (5000, 256, 16, 4, 128, torch.bfloat16)])  # split router
+def test_renormalised_router_forward(T, d, E, k, f, dtype):
+    """Router mode 1: the same experts, weights summing to one per token."""
+    inp = S.layer_inputs(S.LayerShape(T, d, E, k, f), seed=T + 7, dtype=dtype, normalised=dtype != torch.float32)
+    out = run_forward(inp, renorm=True)
+    sample = None if T <= 1000 else np.arange(0, T, 97)
+    check_forward(inp, out, sample=sample, renorm=True)
+    assert torch.allclose(out["w"].sum(dim=1), torch.ones(T, device="cuda"), atol=1e-5)
+
+
+def test_renormalised_router_backward():
+    inp = S.layer_inputs(S.LayerShape(384, 256, 16, 4, 256), seed=44, with_grad=True)
+    check_backward(inp, alpha=0.3, beta=0.2, renorm=True)

@@ -243,6 +243,44 @@ def test_stack_small_shapes_every_token():
     assert_close(got[ok], ref[~tainted], "stack residual")
 
 
+def test_stack_trace_counts_losses_and_choices():
+    """The per-layer routing trace of the stack: the residual is bit-identical to
+    the plain stack, each layer's counts are the bincount of its choices, and
+    layer 0 (whose input rows of +-1 normalise and round to themselves, so the
+    oracle sees exactly the GPU's input) chooses and scores as the oracle does."""
+    sh = S.LayerShape(T=300, d_model=512, n_experts=64, top_k=8, d_ff=256)
+    n = 3
+    _, layers = S.stack_inputs(sh, n, seed=11)
+    g = torch.Generator().manual_seed(12)
+    x0 = torch.where(torch.rand(sh.T, sh.d_model, generator=g) < 0.5, -1.0, 1.0)
+    cfg = M.config(sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff)
+    ws = M.workspace(cfg, False)
+    dev = [{k: (v.cuda() if v is not None else None) for k, v in L.items()} for L in layers]
+    r1 = x0.clone().cuda()
+    M.moe_stack_forward(cfg, dev, r1, ws)
+    r2 = x0.clone().cuda()
+    counts = torch.empty(n, sh.n_experts, dtype=torch.int32, device="cuda")
+    losses = torch.empty(n, 2, device="cuda")
+    idx = torch.empty(n, sh.T, sh.top_k, dtype=torch.int32, device="cuda")
+    M.moe_stack_forward_trace(cfg, dev, r2, ws, counts, losses, idx)
+    torch.cuda.synchronize()
+    assert M.moe_get_device_status(ws) == 0
+    assert torch.equal(r1, r2)
+    counts, losses, idx = counts.cpu().numpy(), losses.cpu().numpy(), idx.cpu().numpy()
+    for l in range(n):
+        assert np.array_equal(np.bincount(idx[l].reshape(-1), minlength=sh.n_experts), counts[l])
+        assert counts[l].sum() == sh.T * sh.top_k and np.all(np.isfinite(losses[l]))
+    xn = f64(x0)  # RMSNorm of +-1 rows is +-1 after rounding to bf16
+    p, lse = O.softmax_lse(O.router_logits(xn, f64(layers[0]["w_router"]), f64(layers[0]["router_bias"])))
+    ref_idx, _ = O.topk_no_renorm(p, sh.top_k)
+    near = O.near_tie_tokens(p, sh.top_k)
+    assert np.array_equal(idx[0][~near], ref_idx[~near])
+    if not near.any():
+        L_lb, _ = O.load_balance_loss(ref_idx, p, sh.n_experts)
+        assert_loss_close(losses[0, 0], L_lb, "layer-0 L_lb")
+    assert_loss_close(losses[0, 1], O.router_z_loss(lse), "layer-0 L_z")
+
+
 def test_stack_16_layers_8192_tokens_sampled():
     """The Zipf-skewed stack at T=8192 on sampled tokens. Four layers are held to
     both bars; after all 16, each layer's bf16 input having been rounded from a
