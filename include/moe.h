@@ -284,7 +284,9 @@ moe_status moe_stack_forward_trace(const moe_config* cfg, int32_t n_layers, cons
 moe_status moe_set_stage_events(void* const* events);
 
 /* Reads the workspace status word (0 = no failure recorded) into *code and clears
- * it. Synchronises `stream`. Returns MOE_ERR_DEVICE_CHECK when *code != 0. */
+ * it, together with the workspace's completion counters (so a workspace whose
+ * kernel gave up part-way can be used again). Synchronises `stream`. Returns
+ * MOE_ERR_DEVICE_CHECK when *code != 0. */
 moe_status moe_get_device_status(void* ws, int32_t* code, cudaStream_t stream);
 
 #ifdef __cplusplus

@@ -173,9 +173,9 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_dispatch_impl(const Shape& s, const int32_t* idx, const void* x, int32_t* offsets,
                                  int32_t* perm, int32_t* inv_perm, int32_t* group_start, void* x_perm, void* ws,
                                  const Workspace& L, bool zero_pads, cudaStream_t st) {
+  // ctrl[2] is zero between calls (moe_workspace_init, then each launch's last CTA)
   int32_t* ctrl = at<int32_t>(ws, L.ctrl);
-  cudaError_t e = cudaMemsetAsync(ctrl + 2, 0, sizeof(int32_t), st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   const int nchunks = static_cast<int>(s.chunks());
   rank_kernel<<<nchunks, kDispatchChunk, 0, st>>>(idx, s.T, s.E, s.k, at<int32_t>(ws, L.local_rank),
                                                   at<int32_t>(ws, L.chunk_count), at<int32_t>(ws, L.chunk_base),

@@ -965,13 +965,9 @@ namespace {
 template <class C>
 cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb, const Args& a,
                    int max_tiles, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::SMEM_BYTES));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<size_t> smem_set[kMaxDevices];
+  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(grouped_gemm_kernel<C>), C::SMEM_BYTES, smem_set);
+  if (e != cudaSuccess) return e;
   int grid = device_sm_count();
   if (max_tiles < grid) grid = max_tiles;
   if (grid <= 0) return cudaSuccess;
@@ -982,13 +978,9 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtenso
 template <class P>
 cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const Args& a, int max_pair_tiles,
                         cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(pair_gemm_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(P::SMEM_BYTES));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<size_t> smem_set[kMaxDevices];
+  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(pair_gemm_kernel<P>), P::SMEM_BYTES, smem_set);
+  if (e != cudaSuccess) return e;
   int clusters = device_sm_count() / 2;
   if (max_pair_tiles < clusters) clusters = max_pair_tiles;
   if (clusters <= 0) return cudaSuccess;

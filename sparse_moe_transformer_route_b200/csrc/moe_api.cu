@@ -37,6 +37,19 @@ bool current_device(DeviceInfo* out) {
 }
 }  // namespace
 
+cudaError_t raise_smem_limit(const void* func, size_t bytes, std::atomic<size_t>* cache) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  if (dev >= 0 && dev < kMaxDevices && cache[dev].load() >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
+    size_t cur = cache[dev].load();
+    while (cur < bytes && !cache[dev].compare_exchange_weak(cur, bytes)) {
+    }
+  }
+  return e;
+}
+
 int device_sm_count() {
   DeviceInfo d;
   return current_device(&d) ? d.sms : 148;
@@ -466,7 +479,9 @@ moe_status moe_get_device_status(void* ws, int32_t* code, cudaStream_t stream) {
   int32_t v = 0;
   MOE_TRY(cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, stream));
   MOE_TRY(cudaStreamSynchronize(stream));
-  MOE_TRY(cudaMemsetAsync(ws, 0, sizeof(int32_t), stream));
+  // the status word and, with it, the completion counters: a launch that gave
+  // up part-way may have left a counter behind
+  MOE_TRY(cudaMemsetAsync(ws, 0, 3 * sizeof(int32_t), stream));
   *code = v;
   return v == 0 ? MOE_OK : MOE_ERR_DEVICE_CHECK;
 }

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
@@ -107,6 +108,13 @@ cudaError_t launch_router_weight_grad(const Shape& s, const float* dh, const voi
 size_t router_wgrad_partial_bytes(const Shape& s);
 
 int device_sm_count();
+
+// Raises `func`'s dynamic shared-memory limit to at least `bytes` on the current
+// device. `cache` (one entry per device id < 64, zero-initialised, owned by the
+// call site) remembers the largest limit already set, so each device is
+// configured once however many devices a process drives.
+constexpr int kMaxDevices = 64;
+cudaError_t raise_smem_limit(const void* func, size_t bytes, std::atomic<size_t>* cache);
 
 // 2-D TMA descriptor over a row-major [rows, cols] bf16/fp32 matrix with a
 // [box_rows, box_cols] box and 128-byte swizzle (out-of-range boxes read zeros).

@@ -239,16 +239,13 @@ cudaError_t run(const Shape& s, const void* x, const void* w_router, const float
                 int32_t* counts, float* losses, void* ws, const Workspace& L, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(kTok) * s.d * sizeof(Tin) + static_cast<size_t>(kTok) * s.E * 12 +
                       kTok * 4 + s.E * 4;
-  static size_t configured = 0;
-  if (smem > 48 * 1024 && configured < smem) {
-    cudaError_t e =
-        cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  static std::atomic<size_t> smem_set[kMaxDevices];
+  if (smem > 48 * 1024) {
+    cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(router_kernel<Tin>), smem, smem_set);
     if (e != cudaSuccess) return e;
-    configured = smem;
   }
+  // ctrl[1] is zero between calls (moe_workspace_init, then each launch's last CTA)
   int32_t* ctrl = at<int32_t>(ws, L.ctrl);
-  cudaError_t e = cudaMemsetAsync(ctrl + 1, 0, sizeof(int32_t), st);
-  if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(s.router_ctas());
   router_kernel<Tin><<<grid, kThreads, smem, st>>>(
       static_cast<const Tin*>(x), static_cast<const Tin*>(w_router), bias, s.T, s.d, s.E, s.k, idx, wts,

@@ -884,26 +884,22 @@ bool router_tc_supported(const Shape& s) { return !s.fp32 && s.E <= kMaxE && s.k
 cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
                              float* wts, int32_t* counts, float* losses, void* ws, const Workspace& L,
                              cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes(16)));
+  {
+    static std::atomic<size_t> set_fused[kMaxDevices], set_logits[kMaxDevices], set_epi[kMaxDevices];
+    cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(router_tc_kernel<16, 1>), smem_bytes(16), set_fused);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kLogitSmem));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(router_epi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kEpiSmem));
+      e = raise_smem_limit(reinterpret_cast<const void*>(router_logits_kernel), kLogitSmem, set_logits);
+    if (e == cudaSuccess) e = raise_smem_limit(reinterpret_cast<const void*>(router_epi_kernel), kEpiSmem, set_epi);
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   const int NP = (s.E + 15) / 16 * 16;
   CUtensorMap tx, tw;
   if (!make_map(&tx, x, false, static_cast<uint64_t>(s.T), s.d, 64, kTile)) return cudaErrorInvalidValue;
   if (!make_map(&tw, w_router, false, static_cast<uint64_t>(s.E), s.d, 64, NP)) return cudaErrorInvalidValue;
+  // ctrl[1], the completion counter, is zero between calls: moe_workspace_init
+  // clears it and the last CTA of every router launch puts it back to zero
   int32_t* ctrl = at<int32_t>(ws, L.ctrl);
-  cudaError_t e = cudaMemsetAsync(ctrl + 1, 0, sizeof(int32_t), st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   RArgs a{};
   a.T = s.T;
   a.d = s.d;
