@@ -17,6 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
+ABI_VERSION = 3  # MOE_ABI_VERSION of include/moe.h this binding marshals for
 MOE_BF16 = 0
 MOE_FP32 = 1
 MOE_ROUTER_SOFTMAX_TOPK = 0
@@ -111,6 +112,9 @@ def lib():
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
+        if L.moe_abi_version() != ABI_VERSION:
+            raise RuntimeError(f"{LIB_PATH} implements ABI {L.moe_abi_version()}, this binding ABI {ABI_VERSION}: "
+                               "rebuild with `python -m sparse_moe_transformer_route_b200.build`")
         _lib = L
     return _lib
 
