@@ -34,6 +34,16 @@ the design notes):
     the backward objective  <dy, y> + alpha * L_lb + beta * L_z.
   * No gradient flows through the expert choice or through f ([OLMoE-Guide]
     computes f with bincount, a count).
+  * Expert choice (the alternative the paper summary compares in section
+    4.1.4, "Expert Choice vs. Token Choice": experts pick tokens instead of
+    tokens picking experts). The pages give no formula; the plain reading
+    taken: the same router probabilities p = softmax(h) over experts; each
+    expert e takes the C tokens with the largest p[t, e] (ties to the lower
+    token index); C = ceil(T*k/E) capped at T, so the expert work equals token
+    choice's; the weight of (t, e) is p[t, e]; a token sums over the experts
+    that took it in ascending expert order and gets zero when none did; the
+    z-loss is unchanged and there is no load-balancing loss (every expert
+    holds exactly C tokens).
   * Storage precision (optional `store` argument of the expert functions,
     moe_forward and moe_backward): the pages fix no precision for the expert
     activations. By default nothing is rounded. Given a rounding function,
@@ -74,6 +84,10 @@ __all__ = [
     "expert_weight_grad_slices",
     "rms_norm",
     "stack_forward",
+    "ec_capacity",
+    "expert_choice",
+    "experts_expert_choice",
+    "moe_forward_expert_choice",
 ]
 
 
@@ -549,3 +563,89 @@ def stack_forward(x0, layers, k, eps=1e-5, round_input=None):
         r = r + out["y"]
         outs.append(out)
     return r, outs
+
+
+# --------------------------------------------------------------------------- expert choice
+
+
+def ec_capacity(n_tokens, k, n_experts):
+    """Tokens per expert under expert choice: ceil(T*k/E), at most T.
+
+    With this capacity the E experts process about T*k rows in total, the same
+    expert work as top-k token choice ([OLMoE-paper] section 4.1.4 compares the
+    two at equal compute).
+    """
+    return min(int(n_tokens), -(-int(n_tokens) * int(k) // int(n_experts)))
+
+
+def expert_choice(p, capacity):
+    """Each expert picks its `capacity` highest-probability tokens.
+
+    [OLMoE-paper] section 4.1.4 "Expert Choice vs. Token Choice": the experts
+    choose the tokens. For expert e the candidates are the column p[:, e] of
+    the softmax over experts; the C largest are kept, equal values going to the
+    lower token index (a stable sort of -p[:, e]). The chosen tokens are listed
+    in ascending token order (the order of the expert's rows).
+    Returns (sel [E, C] int64 token indices, gates [E, C] float64 = p[sel, e]).
+    """
+    p = _f64(p)
+    T, E = p.shape
+    C = int(capacity)
+    sel = np.zeros((E, C), dtype=np.int64)
+    gates = np.zeros((E, C))
+    for e in range(E):
+        top = np.argsort(-p[:, e], kind="stable")[:C]
+        top = np.sort(top)
+        sel[e] = top
+        gates[e] = p[top, e]
+    return sel, gates
+
+
+def experts_expert_choice(x, sel, gates, w_gate_up, w_down, store=None):
+    """y_t = sum over experts e that chose t (ascending e) of p[t, e] * Expert_e(x_t).
+
+    Each expert runs once on its C rows (as in [MoE-scratch] section 2
+    `dispatch`, with the rows given by the expert's choice); a token that no
+    expert chose gets y_t = 0.
+    """
+    x = _f64(x)
+    sel = np.asarray(sel)
+    gates = _f64(gates)
+    y = np.zeros_like(x)
+    for e in range(sel.shape[0]):
+        if sel.shape[1] == 0:
+            continue
+        out = swiglu_expert(x[sel[e]], w_gate_up[e], w_down[e], store)
+        # an expert picks a token at most once, so sel[e] has no repeats
+        y[sel[e]] += gates[e][:, None] * out
+    return y
+
+
+def moe_forward_expert_choice(x, w_router, w_gate_up, w_down, k, router_bias=None, capacity=None,
+                              store=None):
+    """The layer with expert-choice routing (see the module notes for the reading).
+
+    Returns a dict with y [T,d], sel [E,C], gates [E,C], p [T,E], lse [T], h [T,E],
+    capacity C, fanout [T] (experts per token), L_lb (0: no balance loss), L_z.
+    """
+    x = _f64(x)
+    T = x.shape[0]
+    E = _f64(w_router).shape[0]
+    C = ec_capacity(T, k, E) if capacity is None else int(capacity)
+    h = router_logits(x, w_router, router_bias)
+    p, lse = softmax_lse(h)
+    sel, gates = expert_choice(p, C)
+    y = experts_expert_choice(x, sel, gates, w_gate_up, w_down, store)
+    fanout = np.bincount(sel.reshape(-1), minlength=T)
+    return {
+        "y": y,
+        "sel": sel,
+        "gates": gates,
+        "p": p,
+        "lse": lse,
+        "h": h,
+        "capacity": C,
+        "fanout": fanout,
+        "L_lb": 0.0,
+        "L_z": router_z_loss(lse),
+    }

@@ -439,3 +439,92 @@ def test_zipf_offset_matches_its_calibration():
     spec.loader.exec_module(cal)
     x, wr = cal.layer0_inputs()
     assert abs(cal.top8_share(S.ZIPF_LAMBDA, x, wr) - 0.5) <= 0.01
+
+
+# ------------------------------------------------------------------ expert-choice pins
+
+
+def test_expert_choice_hand_case():
+    """Four tokens, two experts, capacity 2, worked by hand. Expert 0's column
+    (0.5, 0.2, 0.9, 0.5): token 2, then the tie at 0.5 goes to token 0. Expert 1's
+    column (0.5, 0.8, 0.1, 0.5): token 1, then token 0 over token 3."""
+    p = np.array([[0.5, 0.5], [0.2, 0.8], [0.9, 0.1], [0.5, 0.5]])
+    sel, gates = O.expert_choice(p, 2)
+    assert sel.tolist() == [[0, 2], [0, 1]]
+    assert gates.tolist() == [[0.5, 0.9], [0.5, 0.8]]
+
+
+def test_expert_choice_selection_by_brute_force():
+    """Every chosen token beats every unchosen one in the expert's column (or ties
+    it with a lower index), checked pair by pair; the list is in token order and
+    holds exactly C distinct tokens. Equal values are planted so ties occur."""
+    r = _rng(21)
+    for T, E, C in [(9, 3, 4), (13, 5, 1), (16, 4, 16), (11, 2, 7)]:
+        p = r.integers(0, 4, size=(T, E)) / 4.0  # many exact ties
+        sel, gates = O.expert_choice(p, C)
+        for e in range(E):
+            chosen = [int(t) for t in sel[e]]
+            assert len(chosen) == C == len(set(chosen))
+            assert chosen == sorted(chosen)
+            for t in chosen:
+                assert gates[e][chosen.index(t)] == p[t, e]
+                for u in range(T):
+                    if u in chosen:
+                        continue
+                    assert p[t, e] > p[u, e] or (p[t, e] == p[u, e] and t < u)
+
+
+def test_expert_choice_capacity():
+    """ceil(T k / E), capped at T: OLMoE's shapes give T/8 tokens per expert."""
+    assert O.ec_capacity(4096, 8, 64) == 512
+    assert O.ec_capacity(16384, 8, 64) == 2048
+    assert O.ec_capacity(1, 8, 64) == 1
+    assert O.ec_capacity(100, 3, 7) == 43  # 300 / 7 = 42.86
+    assert O.ec_capacity(5, 8, 4) == 5  # 10 would exceed T
+
+
+def test_expert_choice_full_capacity_is_the_dense_softmax_layer():
+    """With C = T every expert takes every token, so y = sum_e p[t, e] Expert_e(x_t):
+    the page's every-expert-on-every-token layer with the full softmax as gate."""
+    L = _small_layer(22, T=10, E=6, k=6)
+    out = O.moe_forward_expert_choice(**L)
+    assert out["capacity"] == 10
+    assert np.all(out["fanout"] == 6)
+    T, E = out["p"].shape
+    idx = np.tile(np.arange(E), (T, 1))
+    yd = O.experts_dense(L["x"], idx, out["p"], L["w_gate_up"], L["w_down"])
+    assert np.abs(out["y"] - yd).max() < 1e-12
+
+
+def test_expert_choice_single_expert_is_a_plain_swiglu_mlp():
+    """E = 1: p = 1 and the one expert takes all T tokens: y = SwiGLU(x)."""
+    r = _rng(23)
+    T, d, f = 12, 16, 8
+    x = r.standard_normal((T, d))
+    wgu = r.standard_normal((1, 2 * f, d)) * 0.3
+    wd = r.standard_normal((1, d, f)) * 0.3
+    out = O.moe_forward_expert_choice(x, np.zeros((1, d)), wgu, wd, k=1)
+    assert out["sel"].tolist() == [list(range(T))]
+    xt = torch.from_numpy(x)
+    ref = (torch.nn.functional.silu(xt @ torch.from_numpy(wgu[0, :f]).T) * (xt @ torch.from_numpy(wgu[0, f:]).T)) @ \
+        torch.from_numpy(wd[0]).T
+    assert np.abs(out["y"] - ref.numpy()).max() < 1e-13
+
+
+def test_expert_choice_dropped_tokens_get_zero_and_z_loss_is_unchanged():
+    """With C = 1 most tokens are chosen by no expert; their rows are zero. The
+    chosen ones equal the dense layer restricted to the (token, expert) pairs
+    picked. L_z is the token-choice z-loss of the same logits."""
+    L = _small_layer(24, T=30, E=4, k=1)
+    out = O.moe_forward_expert_choice(**L, capacity=1)
+    gate = np.zeros_like(out["p"])
+    for e in range(4):
+        t = int(out["sel"][e, 0])
+        assert t == int(np.argmax(out["p"][:, e]))  # the column's largest (no ties here)
+        gate[t, e] = out["p"][t, e]
+    idx = np.tile(np.arange(4), (30, 1))
+    yd = O.experts_dense(L["x"], idx, gate, L["w_gate_up"], L["w_down"])
+    assert np.abs(out["y"] - yd).max() < 1e-12
+    assert np.all(out["y"][out["fanout"] == 0] == 0.0)
+    assert out["L_z"] == O.moe_forward(**L)["L_z"]
+    assert out["L_lb"] == 0.0
