@@ -192,16 +192,20 @@ __device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& s
   const unsigned qm = quad_mask();
   m = fmaxf(m, __shfl_xor_sync(qm, m, 1));
   m = fmaxf(m, __shfl_xor_sync(qm, m, 2));
+  float ex[16];  // exp(h - m), computed once for the sum and the probabilities
   float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) s += (eb + i < E) ? expf(h[i] - m) : 0.f;
+  for (int i = 0; i < 16; ++i) {
+    ex[i] = (eb + i < E) ? expf(h[i] - m) : 0.f;
+    s += ex[i];
+  }
   s += __shfl_xor_sync(qm, s, 1);
   s += __shfl_xor_sync(qm, s, 2);
   const float lse = m + logf(s);
   {
     float pv[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) pv[i] = (valid && eb + i < E) ? expf(h[i] - m) / s : 0.f;
+    for (int i = 0; i < 16; ++i) pv[i] = valid ? ex[i] / s : 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) P[r * kMaxE + eb + i] = pv[i];
     if (valid && eb < E) {

@@ -226,3 +226,22 @@ def test_renormalised_router_forward(T, d, E, k, f, dtype):
 def test_renormalised_router_backward():
     inp = S.layer_inputs(S.LayerShape(384, 256, 16, 4, 256), seed=44, with_grad=True)
     check_backward(inp, alpha=0.3, beta=0.2, renorm=True)
+
+
+# ------------------------------------------------------------------ edge cases
+
+
+@pytest.mark.parametrize("T,d,E,k,f", [
+    (100, 128, 1, 1, 128),     # one expert: p = w = 1, the layer is a plain SwiGLU MLP
+    (50, 256, 2, 2, 128),      # every expert chosen by every token
+    (3, 128, 64, 16, 128),     # the largest k, fewer tokens than one tile
+    (33, 4096, 16, 4, 4096),   # the largest d and f (bf16)
+    (260, 256, 256, 16, 128),  # the most experts (SIMT router) with the largest k
+    (257, 512, 40, 5, 256),    # E not a multiple of 16, ragged last tile
+])
+def test_edge_shapes(T, d, E, k, f):
+    inp = S.layer_inputs(S.LayerShape(T, d, E, k, f), seed=T + E)
+    out = run_forward(inp)
+    check_forward(inp, out)
+    if E == 1:
+        assert torch.all(out["w"] == 1) and torch.all(out["idx"] == 0)
