@@ -441,6 +441,46 @@ def bench_stack(M, S, dev, steps, peaks):
     }
 
 
+def bench_expert_choice(M, S, dev, cfg, x, weights, steps, peaks, ms_token_choice):
+    """The same T=4096 layer (weights, tokens) under expert-choice routing: every
+    expert takes its C = T*k/E best tokens, so the expert GEMMs do the same work
+    as token choice on perfectly even groups. CUDA events per stage, as the
+    headline; inputs larger than L2 (805 MB of weights per step)."""
+    import torch
+    wr, wgu, wd = weights
+    T, E = cfg.T, cfg.n_experts
+    C = M.moe_expert_choice_capacity(cfg)
+    ws = M.workspace(cfg, False, dev)
+    y = torch.empty_like(x)
+    losses = torch.empty(2, device=dev)
+    for _ in range(3):
+        M.moe_forward_expert_choice(cfg, x, wr, None, wgu, wd, y, losses, None, None, ws)
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(M.binding.STAGE_EVENTS)] for _ in range(steps)]
+    for row in ev:
+        for e in row:
+            e.record()
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        M.moe_set_stage_events(ev[i])
+        M.moe_forward_expert_choice(cfg, x, wr, None, wgu, wd, y, losses, None, None, ws)
+    torch.cuda.synchronize(dev)
+    status = M.moe_get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device check failed under expert choice: 0x{status:x}")
+    ms = statistics.median(ev[i][0].elapsed_time(ev[i][-1]) for i in range(steps))
+    stage_ms = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps))
+                for j, name in enumerate(("router", "select_gather", "gate_up", "down", "combine"))}
+    gu = 2.0 * E * C * cfg.d_model * 2 * cfg.d_ff
+    return {
+        "T": T, "capacity": C, "ms": ms, "steps": steps, "tokens_per_s": T / (ms * 1e-3),
+        "stage_ms": stage_ms, "vs_token_choice": ms_token_choice / ms,
+        "gate_up_tflops": gu / (stage_ms["gate_up"] * 1e-3) / 1e12,
+        "gate_up_frac_of_measured": gu / (stage_ms["gate_up"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "timing": "CUDA events per stage, median over steps, no L2 flush (weights exceed L2)",
+    }
+
+
 def run_b200(args, rank, world, local):
     import torch
     import sparse_moe_transformer_route_b200 as M
@@ -459,8 +499,13 @@ def run_b200(args, rank, world, local):
     y = torch.empty_like(x)
     losses = torch.empty(2, device=dev)
 
+    expert_choice = args.routing == "expert"
+
     def step():
-        M.moe_forward(cfg, x, wr, None, wgu, wd, y, losses, None, None, False, ws)
+        if expert_choice:
+            M.moe_forward_expert_choice(cfg, x, wr, None, wgu, wd, y, losses, None, None, ws)
+        else:
+            M.moe_forward(cfg, x, wr, None, wgu, wd, y, losses, None, None, False, ws)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -553,12 +598,17 @@ def run_b200(args, rank, world, local):
             "value": world * T / e2e_s, "unit": UNIT,
             "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2 + 8,
         },
-        "gpu_launches": KERNELS_PER_STEP * K,
+        "gpu_launches": (KERNELS_PER_STEP + (1 if expert_choice else 0)) * K,
         "clocks": clocks,
     }
+    if expert_choice:
+        line["config"]["routing"] = "expert choice (profiling run; the headline is token choice)"
     extras = [] if args.no_extras else [e for e in args.extras.split(",") if e]
     if world == 1 and extras:
         # the other OLMoE-shape workloads on this GPU, each reported beside the headline
+        if "ec" in extras and not expert_choice:
+            line["expert_choice"] = bench_expert_choice(M, S, dev, cfg, x, (wr, wgu, wd), 50, peaks, ms)
+            torch.cuda.empty_cache()
         if "decode" in extras:
             line["decode"] = bench_decode(M, S, dev, (wr, wgu, wd), 200, peaks)
         del x, wr, wgu, wd, ws, y
@@ -590,9 +640,11 @@ def main(argv=None):
                     help="tokens per layer call (4096 is the benchmarked workload; others are for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the decode, training-step and 16-layer stack workloads (run at N=1 only)")
-    ap.add_argument("--extras", default="decode,train,stack",
-                    help="comma list of the extra workloads to run at N=1 (decode, train, stack)")
+                    help="skip the expert-choice, decode, training-step and 16-layer stack workloads (N=1 only)")
+    ap.add_argument("--extras", default="ec,decode,train,stack",
+                    help="comma list of the extra workloads to run at N=1 (ec, decode, train, stack)")
+    ap.add_argument("--routing", choices=("token", "expert"), default="token",
+                    help="token choice (OLMoE, the benchmarked layer) or expert choice (for profiling)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args(argv)
     rank, world, local = dist_env()

@@ -50,7 +50,7 @@ extern "C" {
 struct CUstream_st;
 typedef struct CUstream_st* cudaStream_t;
 
-#define MOE_ABI_VERSION 3
+#define MOE_ABI_VERSION 4
 #define MOE_ROW_ALIGN 128
 
 typedef enum moe_status {
@@ -274,6 +274,48 @@ moe_status moe_stack_forward_trace(const moe_config* cfg, int32_t n_layers, cons
                                    const float* const* router_biases, const void* const* w_gate_up,
                                    const void* const* w_down, float* resid, int32_t* counts, float* losses,
                                    int32_t* topk_idx, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Expert-choice routing ("OLMoE: Open Mixture-of-Experts Language Models",
+ * section 4.1.4 "Expert Choice vs. Token Choice": the experts choose the tokens;
+ * the pages give no formula, so this is its plain reading). The router
+ * probabilities are token choice's, p = softmax over experts of W_r x (+ bias);
+ * expert e takes the C tokens with the largest p[t, e] (equal values: the lower
+ * token index) as its rows, in ascending token order, each weighted by p[t, e];
+ * a token sums its experts' outputs in ascending expert order, in fp32, rounded
+ * once, and is zero when no expert took it. There is no load-balancing loss
+ * (losses[0] = 0); losses[1] is the z-loss, as in token choice.
+ * Supported for bf16 layers with E <= 64 and router_mode 0; other configs return
+ * MOE_ERR_UNSUPPORTED_SHAPE. `capacity` is C: 0 takes the default
+ * moe_expert_choice_capacity(cfg); otherwise 1 <= C <= T and the E groups of C
+ * rows, each padded to MOE_ROW_ALIGN, must fit in moe_padded_rows(cfg) rows
+ * (always true for the default), else MOE_ERR_INVALID_ARG. The workspace is
+ * moe_workspace_bytes(cfg, 0) bytes; forward only (no backward). */
+
+/* The default capacity ceil(T * k / E), capped at T: the experts then process
+ * about T * k rows, the expert work of top-k token choice. -1 for a bad cfg. */
+int64_t moe_expert_choice_capacity(const moe_config* cfg);
+
+/* Routing only.
+ *   x, w_router, router_bias as in moe_route
+ *   sel    [device] [E, C] int32 out   chosen tokens of each expert, ascending
+ *   gates  [device] [E, C] fp32 out    their probabilities p[sel, e]
+ *   probs  [device] [T, E] fp32 out or NULL: the softmax probabilities
+ *   counts [device] [E] int32 out or NULL: rows per expert (all C)
+ *   losses [device] [2] fp32 out or NULL: {0, L_z} */
+moe_status moe_route_expert_choice(const moe_config* cfg, int64_t capacity, const void* x, const void* w_router,
+                                   const float* router_bias, int32_t* sel, float* gates, float* probs,
+                                   int32_t* counts, float* losses, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* The whole layer under expert choice: route, gather each expert's C rows, the
+ * two grouped expert GEMMs (the token-choice kernels), and the combine.
+ *   y      [device] [T, d] out
+ *   losses [device] [2] fp32 out or NULL: {0, L_z}
+ *   sel    [device] [E, C] int32 out or NULL;  gates [device] [E, C] fp32 out or NULL
+ * moe_set_stage_events marks the same six points as for moe_forward. */
+moe_status moe_forward_expert_choice(const moe_config* cfg, int64_t capacity, const void* x, const void* w_router,
+                                     const float* router_bias, const void* w_gate_up, const void* w_down, void* y,
+                                     float* losses, int32_t* sel, float* gates, void* ws, size_t ws_bytes,
+                                     cudaStream_t stream);
 
 /* Stage timing for profiling. When `events` is non-NULL, the next call of
  * moe_forward records events[0] on its stream before the router and events[i]

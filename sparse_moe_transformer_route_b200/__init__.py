@@ -20,15 +20,18 @@ from .binding import (  # noqa: F401
     moe_combine,
     moe_combine_residual,
     moe_dispatch,
+    moe_expert_choice_capacity,
     moe_expert_down,
     moe_expert_ffn,
     moe_expert_gate_up,
     moe_forward,
+    moe_forward_expert_choice,
     moe_forward_host,
     moe_get_device_status,
     moe_padded_rows,
     moe_rmsnorm,
     moe_route,
+    moe_route_expert_choice,
     moe_route_static,
     moe_set_stage_events,
     moe_stack_forward,

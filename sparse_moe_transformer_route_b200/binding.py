@@ -17,7 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
-ABI_VERSION = 3  # MOE_ABI_VERSION of include/moe.h this binding marshals for
+ABI_VERSION = 4  # MOE_ABI_VERSION of include/moe.h this binding marshals for
 MOE_BF16 = 0
 MOE_FP32 = 1
 MOE_ROUTER_SOFTMAX_TOPK = 0
@@ -40,7 +40,8 @@ EXPORTS = (
     "moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_route_static", "moe_dispatch",
     "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_forward",
     "moe_forward_host", "moe_backward", "moe_rmsnorm", "moe_combine_residual",
-    "moe_stack_forward", "moe_stack_forward_trace", "moe_set_stage_events", "moe_get_device_status",
+    "moe_stack_forward", "moe_stack_forward_trace", "moe_expert_choice_capacity", "moe_route_expert_choice",
+    "moe_forward_expert_choice", "moe_set_stage_events", "moe_get_device_status",
 )
 STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "gate_up", "down", "combine")
@@ -94,6 +95,11 @@ _SIGS = {
                                          ctypes.c_size_t, _P]),
     "moe_stack_forward_trace": (ctypes.c_int, [_CFG, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                                ctypes.c_size_t, _P]),
+    "moe_expert_choice_capacity": (ctypes.c_int64, [_CFG]),
+    "moe_route_expert_choice": (ctypes.c_int, [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                               ctypes.c_size_t, _P]),
+    "moe_forward_expert_choice": (ctypes.c_int, [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                 ctypes.c_size_t, _P]),
     "moe_set_stage_events": (ctypes.c_int, [_P]),
     "moe_get_device_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), _P]),
 }
@@ -335,6 +341,46 @@ def moe_forward(cfg, x, w_router, router_bias, w_gate_up, w_down, y, losses, top
         _ptr(topk_w, torch.float32, (T, k), "topk_w", allow_none=True),
         1 if save_for_backward else 0, _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
     _check(st, "moe_forward")
+
+
+def moe_expert_choice_capacity(cfg) -> int:
+    """Default expert-choice capacity ceil(T*k/E), capped at T."""
+    c = lib().moe_expert_choice_capacity(_cfgp(cfg))
+    if c < 0:
+        raise MoeError(2, "moe_expert_choice_capacity")
+    return c
+
+
+def moe_route_expert_choice(cfg, x, w_router, router_bias, sel, gates, probs, counts, losses, ws, capacity=0,
+                            stream=None):
+    dt = torch_dtype(cfg)
+    T, d, E = cfg.T, cfg.d_model, cfg.n_experts
+    C = capacity if capacity > 0 else moe_expert_choice_capacity(cfg)
+    st = lib().moe_route_expert_choice(
+        _cfgp(cfg), capacity, _ptr(x, dt, (T, d), "x"), _ptr(w_router, dt, (E, d), "w_router"),
+        _ptr(router_bias, torch.float32, (E,), "router_bias", allow_none=True),
+        _ptr(sel, torch.int32, (E, C), "sel"), _ptr(gates, torch.float32, (E, C), "gates"),
+        _ptr(probs, torch.float32, (T, E), "probs", allow_none=True),
+        _ptr(counts, torch.int32, (E,), "counts", allow_none=True),
+        _ptr(losses, torch.float32, (2,), "losses", allow_none=True),
+        _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
+    _check(st, "moe_route_expert_choice")
+
+
+def moe_forward_expert_choice(cfg, x, w_router, router_bias, w_gate_up, w_down, y, losses, sel, gates, ws,
+                              capacity=0, stream=None):
+    dt = torch_dtype(cfg)
+    T, d, E, f = cfg.T, cfg.d_model, cfg.n_experts, cfg.d_ff
+    C = capacity if capacity > 0 else moe_expert_choice_capacity(cfg)
+    st = lib().moe_forward_expert_choice(
+        _cfgp(cfg), capacity, _ptr(x, dt, (T, d), "x"), _ptr(w_router, dt, (E, d), "w_router"),
+        _ptr(router_bias, torch.float32, (E,), "router_bias", allow_none=True),
+        _ptr(w_gate_up, dt, (E, 2 * f, d), "w_gate_up"), _ptr(w_down, dt, (E, d, f), "w_down"),
+        _ptr(y, dt, (T, d), "y"), _ptr(losses, torch.float32, (2,), "losses", allow_none=True),
+        _ptr(sel, torch.int32, (E, C), "sel", allow_none=True),
+        _ptr(gates, torch.float32, (E, C), "gates", allow_none=True),
+        _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
+    _check(st, "moe_forward_expert_choice")
 
 
 def moe_forward_host(cfg, x_host, w_router, router_bias, w_gate_up, w_down, y_host, losses_host, ws,

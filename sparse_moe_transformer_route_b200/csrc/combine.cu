@@ -133,6 +133,66 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Expert-choice combine: token t's experts are the e with slot_row[t, e] >= 0,
+// taken in ascending e with weight p[t, e]; warp 0 compacts the list with
+// ballots first (so the launch has at least 32 threads), then the loads of up
+// to eight rows go out together; a token no expert took gets zero.
+template <typename T_>
+__global__ void __launch_bounds__(256)
+    combine_ec_kernel(const T_* __restrict__ o_perm, const int32_t* __restrict__ slot_row,
+                      const float* __restrict__ probs, int64_t T, int d, int E, T_* __restrict__ y) {
+  __shared__ int32_t rows[kMaxExperts];
+  __shared__ float ws_[kMaxExperts];
+  __shared__ int s_n;
+  const int64_t t = blockIdx.x;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int n = 0;
+    for (int c = 0; c < E; c += 32) {
+      const int e = c + lane;
+      const int r = e < E ? slot_row[t * E + e] : -1;
+      const unsigned b = __ballot_sync(0xffffffffu, r >= 0);
+      if (r >= 0) {
+        const int p = n + __popc(b & ((1u << lane) - 1u));
+        rows[p] = r;
+        ws_[p] = probs[t * E + e];
+      }
+      n += __popc(b);
+    }
+    if (lane == 0) s_n = n;
+  }
+  __syncthreads();
+  const int n = s_n;
+  const int nv = d / 8;
+  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int j0 = 0; j0 < n; j0 += 8) {
+      Raw8<T_> q[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = j0 + jj < n ? j0 + jj : n - 1;  // past the list: re-read the last row, skipped below
+        q[jj].load(o_perm + static_cast<int64_t>(rows[j]) * d + v * 8);
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        if (j0 + jj < n) {
+          float o[8];
+          q[jj].unpack(o);
+          const float w = ws_[j0 + jj];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, o[i], acc[i]);
+        }
+      }
+    }
+    Vec8<T_> out;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out.v[i] = acc[i];
+    out.store(y + t * d + v * 8);
+  }
+}
+
 template <typename T_>
 __global__ void __launch_bounds__(256)
     rmsnorm_kernel(const float* __restrict__ resid, const float* __restrict__ weight, float eps, int d,
@@ -160,6 +220,16 @@ __global__ void __launch_bounds__(256)
 }
 
 }  // namespace
+
+cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t* slot_row, const float* probs,
+                              void* y, cudaStream_t st) {
+  if (s.fp32) return cudaErrorInvalidValue;  // expert choice runs on the bf16 tensor-core router
+  // at least one whole warp: warp 0 compacts the expert list with ballots
+  const int threads = s.d / 8 < 32 ? 32 : (s.d / 8 < 256 ? s.d / 8 : 256);
+  combine_ec_kernel<__nv_bfloat16><<<static_cast<unsigned>(s.T), threads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o_perm), slot_row, probs, s.T, s.d, s.E, static_cast<__nv_bfloat16*>(y));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const Shape& s, const void* o_perm, const int32_t* inv_perm, const float* wts, void* y,
                            float* resid, cudaStream_t st) {

@@ -114,6 +114,9 @@ Workspace layout(const Shape& s) {
   L.o_perm = take(P * s.d * s.esize);
   L.x_dev = take(T * s.d * s.esize);
   L.y_dev = take(T * s.d * s.esize);
+  L.ec_sel = take(P * 4);
+  L.ec_gate = take(P * 4);
+  L.ec_slot = take(T * E * 4);
   L.fwd_bytes = o;
   L.preact = take(P * 2 * s.f * s.esize);
   L.dw = take(T * k * 4);
@@ -206,6 +209,16 @@ moe_status forward_impl(const Ctx& c, const void* x, const void* w_router, const
   const size_t nk = static_cast<size_t>(s.T) * s.k;
   if (topk_idx != nullptr) MOE_TRY(cudaMemcpyAsync(topk_idx, idx, nk * 4, cudaMemcpyDeviceToDevice, st));
   if (topk_w != nullptr) MOE_TRY(cudaMemcpyAsync(topk_w, wts, nk * 4, cudaMemcpyDeviceToDevice, st));
+  return MOE_OK;
+}
+
+// Checks shared by the expert-choice entry points; *C receives the capacity.
+moe_status ec_prepare(const moe_config* cfg, int64_t capacity, void* ws, size_t ws_bytes, Ctx* c, int64_t* C) {
+  const moe_status r = prepare(cfg, ws, ws_bytes, false, c);
+  if (r != MOE_OK) return r;
+  if (!router_tc_supported(c->s) || c->s.renorm) return MOE_ERR_UNSUPPORTED_SHAPE;
+  *C = capacity > 0 ? capacity : ec_default_capacity(c->s);
+  if (capacity < 0 || !ec_capacity_ok(c->s, *C)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -412,6 +425,70 @@ moe_status moe_backward(const moe_config* cfg, const void* dy, const void* x, co
                               gs, dw_down, dw_gate_up, status, stream));
   MOE_TRY(launch_dx_combine(s, at<void>(ws, L.dx_perm), at<int32_t>(ws, L.inv_perm), dh, w_router, dx, stream));
   MOE_TRY(launch_router_weight_grad(s, dh, x, dw_router, at<float>(ws, L.wr_part), stream));
+  return MOE_OK;
+}
+
+int64_t moe_expert_choice_capacity(const moe_config* cfg) {
+  Shape s;
+  return make_shape(cfg, &s) ? ec_default_capacity(s) : -1;
+}
+
+
+moe_status moe_route_expert_choice(const moe_config* cfg, int64_t capacity, const void* x, const void* w_router,
+                                   const float* router_bias, int32_t* sel, float* gates, float* probs,
+                                   int32_t* counts, float* losses, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  Ctx c;
+  int64_t C = 0;
+  const moe_status r = ec_prepare(cfg, capacity, ws, ws_bytes, &c, &C);
+  if (r != MOE_OK) return r;
+  if (x == nullptr || w_router == nullptr || sel == nullptr || gates == nullptr || !aligned16(x) ||
+      !aligned16(w_router))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(launch_router_probs(c.s, x, w_router, router_bias, ws, c.L, stream));
+  MOE_TRY(launch_ec_select(c.s, C, counts, losses, ws, c.L, stream));
+  const size_t n = static_cast<size_t>(c.s.E) * static_cast<size_t>(C);
+  MOE_TRY(cudaMemcpyAsync(sel, at<int32_t>(ws, c.L.ec_sel), n * 4, cudaMemcpyDeviceToDevice, stream));
+  MOE_TRY(cudaMemcpyAsync(gates, at<float>(ws, c.L.ec_gate), n * 4, cudaMemcpyDeviceToDevice, stream));
+  if (probs != nullptr)
+    MOE_TRY(cudaMemcpyAsync(probs, at<float>(ws, c.L.probs), static_cast<size_t>(c.s.T) * c.s.E * 4,
+                            cudaMemcpyDeviceToDevice, stream));
+  return MOE_OK;
+}
+
+moe_status moe_forward_expert_choice(const moe_config* cfg, int64_t capacity, const void* x, const void* w_router,
+                                     const float* router_bias, const void* w_gate_up, const void* w_down, void* y,
+                                     float* losses, int32_t* sel, float* gates, void* ws, size_t ws_bytes,
+                                     cudaStream_t stream) {
+  Ctx c;
+  int64_t C = 0;
+  const moe_status r = ec_prepare(cfg, capacity, ws, ws_bytes, &c, &C);
+  if (r != MOE_OK) return r;
+  if (x == nullptr || w_router == nullptr || w_gate_up == nullptr || w_down == nullptr || y == nullptr ||
+      !aligned16(x) || !aligned16(w_router) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y))
+    return MOE_ERR_INVALID_ARG;
+  const Shape& s = c.s;
+  const Workspace& L = c.L;
+  int32_t* status = at<int32_t>(ws, L.ctrl);
+  int32_t* gs = at<int32_t>(ws, L.group_start);
+  int32_t* off = at<int32_t>(ws, L.offsets);
+  void* x_perm = at<void>(ws, L.x_perm);
+  const StageMarks marks(stream);
+  MOE_TRY(marks.mark(0));
+  MOE_TRY(launch_router_probs(s, x, w_router, router_bias, ws, L, stream));
+  MOE_TRY(marks.mark(1));
+  MOE_TRY(launch_ec_select(s, C, nullptr, losses, ws, L, stream));
+  MOE_TRY(launch_ec_gather(s, C, x, ws, L, stream));
+  MOE_TRY(marks.mark(2));
+  MOE_TRY(launch_gate_up(s, x_perm, gs, off, w_gate_up, at<void>(ws, L.h), nullptr, status, stream));
+  MOE_TRY(marks.mark(3));
+  MOE_TRY(launch_down(s, at<void>(ws, L.h), gs, off, w_down, at<void>(ws, L.o_perm), status, stream));
+  MOE_TRY(marks.mark(4));
+  MOE_TRY(launch_combine_ec(s, at<void>(ws, L.o_perm), at<int32_t>(ws, L.ec_slot), at<float>(ws, L.probs), y, stream));
+  MOE_TRY(marks.mark(5));
+  const size_t n = static_cast<size_t>(s.E) * static_cast<size_t>(C);
+  if (sel != nullptr) MOE_TRY(cudaMemcpyAsync(sel, at<int32_t>(ws, L.ec_sel), n * 4, cudaMemcpyDeviceToDevice, stream));
+  if (gates != nullptr)
+    MOE_TRY(cudaMemcpyAsync(gates, at<float>(ws, L.ec_gate), n * 4, cudaMemcpyDeviceToDevice, stream));
   return MOE_OK;
 }
 

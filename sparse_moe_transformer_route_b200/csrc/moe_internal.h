@@ -45,6 +45,7 @@ struct Workspace {
   size_t preact;                              // [P, 2f] (training)
   size_t dw, dh, dout, dab, dx_perm, wr_part; // backward scratch
   size_t x_dev, y_dev;                        // staging for the host-buffer entry point
+  size_t ec_sel, ec_gate, ec_slot;            // expert choice: [E, C] tokens and weights, [T, E] rows
   size_t fwd_bytes, bwd_bytes;
 };
 
@@ -79,6 +80,18 @@ cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_star
                         const void* w_down, void* o_perm, int32_t* status, cudaStream_t st);
 cudaError_t launch_combine(const Shape& s, const void* o_perm, const int32_t* inv_perm, const float* wts,
                            void* y, float* resid, cudaStream_t st);
+// Expert choice: the router's probabilities and log-normaliser only (no top-k),
+// then each expert's top-C tokens, the row gather and the combine.
+cudaError_t launch_router_probs(const Shape& s, const void* x, const void* w_router, const float* bias, void* ws,
+                                const Workspace& L, cudaStream_t st);
+int64_t ec_default_capacity(const Shape& s);
+bool ec_capacity_ok(const Shape& s, int64_t C);
+cudaError_t launch_ec_select(const Shape& s, int64_t C, int32_t* counts, float* losses, void* ws, const Workspace& L,
+                             cudaStream_t st);
+cudaError_t launch_ec_gather(const Shape& s, int64_t C, const void* x, void* ws, const Workspace& L,
+                             cudaStream_t st);
+cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t* slot_row, const float* probs,
+                              void* y, cudaStream_t st);
 cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, float eps, void* out,
                            cudaStream_t st);
 

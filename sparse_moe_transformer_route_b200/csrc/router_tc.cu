@@ -31,6 +31,8 @@
 // per-chunk counts (block by block, through shared memory) into chunk bases,
 // the bincount offsets and the padded group starts, and reduces the loss
 // partials. Every sum runs in a fixed order, so the results are deterministic.
+// For expert-choice routing the same kernels stop after the probabilities and
+// the log-normaliser (launch_router_probs); the selection runs afterwards.
 #include <cfloat>
 #include <cmath>
 
@@ -81,6 +83,7 @@ struct RArgs {
   float* logit_part;  // split form: [ksplit][T][E] partial logits
   int ksplit;         // split form: K ranges per 128-token tile
   int renorm;         // weights divided by the sum of the k chosen probabilities
+  int probs_only;     // stop after p and lse (expert choice selects from p afterwards)
 };
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -223,6 +226,7 @@ __device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& s
     lse_s[r] = valid ? lse : 0.f;
     if (valid) a.lse_out[t] = lse;
   }
+  if (a.probs_only) return;  // uniform over the CTA
 
   // ---- top (k+3) in fp32 by quad arg-max (uniform within the quad); nearm bit j
   //      marks ranks j and j+1 as closer than the fp32 uncertainty
@@ -885,9 +889,10 @@ __global__ void __launch_bounds__(128, 2) router_epi_kernel(const RArgs a) {
 
 bool router_tc_supported(const Shape& s) { return !s.fp32 && s.E <= kMaxE && s.k + 3 <= kMaxSel; }
 
-cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
-                             float* wts, int32_t* counts, float* losses, void* ws, const Workspace& L,
-                             cudaStream_t st) {
+namespace {
+cudaError_t router_tc_impl(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
+                           float* wts, int32_t* counts, float* losses, void* ws, const Workspace& L, bool probs_only,
+                           cudaStream_t st) {
   {
     static std::atomic<size_t> set_fused[kMaxDevices], set_logits[kMaxDevices], set_epi[kMaxDevices];
     cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(router_tc_kernel<16, 1>), smem_bytes(16), set_fused);
@@ -931,6 +936,7 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router
   a.ticket = ctrl + 1;
   a.status = ctrl;
   a.renorm = s.renorm ? 1 : 0;
+  a.probs_only = probs_only ? 1 : 0;
   const unsigned grid = static_cast<unsigned>((s.T + kTile - 1) / kTile);
   // A few tokens: logits split over K among many CTAs, then the epilogue
   // (T=1: 24.5 us against 28.7 us fused, warm; T=32: 32.8 against ~28.7).
@@ -962,6 +968,18 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router
   if (e != cudaSuccess) return e;
   router_epi_kernel<<<grid, 128, kEpiSmem, st>>>(a);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_router_tc(const Shape& s, const void* x, const void* w_router, const float* bias, int32_t* idx,
+                             float* wts, int32_t* counts, float* losses, void* ws, const Workspace& L,
+                             cudaStream_t st) {
+  return router_tc_impl(s, x, w_router, bias, idx, wts, counts, losses, ws, L, false, st);
+}
+
+cudaError_t launch_router_probs(const Shape& s, const void* x, const void* w_router, const float* bias, void* ws,
+                                const Workspace& L, cudaStream_t st) {
+  return router_tc_impl(s, x, w_router, bias, nullptr, nullptr, nullptr, nullptr, ws, L, true, st);
 }
 
 }  // namespace moe

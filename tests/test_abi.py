@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol():
 def test_library_has_no_gpu_only_load_dependencies():
     # static CUDA runtime: the .so must load here, where there is no driver
     lib = M.lib()
-    assert lib.moe_abi_version() == B.ABI_VERSION == 3
+    assert lib.moe_abi_version() == B.ABI_VERSION == 4
 
 
 def test_status_strings():
@@ -83,6 +83,25 @@ def test_padded_rows_bound(T, E, k):
     # every expert's group is padded to a multiple of 128: sum_e roundup(c_e) <= T*k + E*127
     assert P >= T * k + E * (B.ROW_ALIGN - 1)
     assert P < T * k + E * (B.ROW_ALIGN - 1) + B.ROW_ALIGN
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 64, 8), (7, 64, 8), (4096, 64, 8), (16384, 64, 8), (300, 16, 4),
+                                   (129, 64, 1), (5, 4, 4)])
+def test_expert_choice_capacity_and_groups_fit(T, E, k):
+    """The default capacity is ceil(T k / E) capped at T (the oracle's ec_capacity),
+    and E groups of it, each padded to 128 rows, fit in the padded row count."""
+    cfg = M.config(T, 512, E, k, 256)
+    C = M.moe_expert_choice_capacity(cfg)
+    assert C == min(T, -(-T * k // E))
+    cpad = -(-C // B.ROW_ALIGN) * B.ROW_ALIGN
+    assert E * cpad <= M.moe_padded_rows(cfg)
+
+
+def test_expert_choice_capacity_rejects_a_bad_config():
+    bad = M.config(4, 128, 8, 2, 128)
+    bad.d_model = 100
+    with pytest.raises(M.MoeError):
+        M.moe_expert_choice_capacity(bad)
 
 
 def test_workspace_sizes_grow_with_training():
