@@ -150,12 +150,14 @@ __global__ void __launch_bounds__(256)
     int n = 0;
     for (int c = 0; c < E; c += 32) {
       const int e = c + lane;
-      const int r = e < E ? slot_row[t * E + e] : -1;
+      // both loads issued before the ballot, so they overlap
+      const int r = e < E ? __ldg(slot_row + t * E + e) : -1;
+      const float pw = e < E ? __ldg(probs + t * E + e) : 0.f;
       const unsigned b = __ballot_sync(0xffffffffu, r >= 0);
       if (r >= 0) {
         const int p = n + __popc(b & ((1u << lane) - 1u));
         rows[p] = r;
-        ws_[p] = probs[t * E + e];
+        ws_[p] = pw;
       }
       n += __popc(b);
     }
