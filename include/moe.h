@@ -50,7 +50,7 @@ extern "C" {
 struct CUstream_st;
 typedef struct CUstream_st* cudaStream_t;
 
-#define MOE_ABI_VERSION 4
+#define MOE_ABI_VERSION 5
 #define MOE_ROW_ALIGN 128
 
 typedef enum moe_status {
@@ -219,6 +219,23 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
                        float* topk_w, int32_t save_for_backward, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
+/* moe_forward for a decode-sized batch as one kernel: routing, both expert
+ * projections and the combine in a single persistent cooperative launch (one
+ * CTA per SM, two grid-wide barriers), reading each touched expert's weights
+ * once ("Mixture-of-experts LLMs from scratch with OLMoE", section 6: at a batch
+ * of one token the layer reads only the chosen experts). The router logits are
+ * summed in fp64 from exact products, so the choice is the exact one (equal
+ * logits: the lower expert index). Same arguments and results as moe_forward
+ * without save_for_backward (counts are not written). moe_forward takes this
+ * path by itself for T <= 8 when nothing is saved for the backward, and
+ * moe_stack_forward(_trace) runs each layer of such a batch as one launch of
+ * it with the RMSNorm and the residual add fused.
+ * Supported: bf16, T <= 8, E <= 64, T*d*2 and T*k*f*2 bytes each at most
+ * 160 KiB; otherwise MOE_ERR_UNSUPPORTED_SHAPE. */
+moe_status moe_forward_decode(const moe_config* cfg, const void* x, const void* w_router, const float* router_bias,
+                              const void* w_gate_up, const void* w_down, void* y, float* losses, int32_t* topk_idx,
+                              float* topk_w, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* moe_forward on host buffers, for callers whose tokens live in host memory:
  * copies x_host [host] [T, d] to the device (inside ws), runs moe_forward with
  * the device-resident weights, copies y back to y_host [host] [T, d] and the two
@@ -319,8 +336,8 @@ moe_status moe_forward_expert_choice(const moe_config* cfg, int64_t capacity, co
 
 /* Stage timing for profiling. When `events` is non-NULL, the next call of
  * moe_forward records events[0] on its stream before the router and events[i]
- * after stage i (1 router, 2 dispatch, 3 gate/up GEMM, 4 down GEMM, 5 combine),
- * then forgets them; `events` holds MOE_STAGE_EVENTS cudaEvent_t handles owned by
+ * after stage i (1 router, 2 dispatch, 3 gate/up GEMM, 4 down GEMM, 5 combine;
+ * on the one-kernel decode path all five follow that kernel), then forgets them; `events` holds MOE_STAGE_EVENTS cudaEvent_t handles owned by
  * the caller. Per host thread. */
 #define MOE_STAGE_EVENTS 6
 moe_status moe_set_stage_events(void* const* events);

@@ -25,6 +25,7 @@ from .binding import (  # noqa: F401
     moe_expert_ffn,
     moe_expert_gate_up,
     moe_forward,
+    moe_forward_decode,
     moe_forward_expert_choice,
     moe_forward_host,
     moe_get_device_status,

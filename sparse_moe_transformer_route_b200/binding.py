@@ -17,7 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
-ABI_VERSION = 4  # MOE_ABI_VERSION of include/moe.h this binding marshals for
+ABI_VERSION = 5  # MOE_ABI_VERSION of include/moe.h this binding marshals for
 MOE_BF16 = 0
 MOE_FP32 = 1
 MOE_ROUTER_SOFTMAX_TOPK = 0
@@ -39,7 +39,7 @@ EXPORTS = (
     "moe_status_string", "moe_abi_version", "moe_check_config", "moe_padded_rows",
     "moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_route_static", "moe_dispatch",
     "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_forward",
-    "moe_forward_host", "moe_backward", "moe_rmsnorm", "moe_combine_residual",
+    "moe_forward_decode", "moe_forward_host", "moe_backward", "moe_rmsnorm", "moe_combine_residual",
     "moe_stack_forward", "moe_stack_forward_trace", "moe_expert_choice_capacity", "moe_route_expert_choice",
     "moe_forward_expert_choice", "moe_set_stage_events", "moe_get_device_status",
 )
@@ -87,6 +87,7 @@ _SIGS = {
     "moe_combine": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P,
                                    ctypes.c_size_t, _P]),
+    "moe_forward_decode": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_forward_host": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_backward": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_rmsnorm": (ctypes.c_int, [_CFG, _P, _P, ctypes.c_float, _P, _P]),
@@ -341,6 +342,23 @@ def moe_forward(cfg, x, w_router, router_bias, w_gate_up, w_down, y, losses, top
         _ptr(topk_w, torch.float32, (T, k), "topk_w", allow_none=True),
         1 if save_for_backward else 0, _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
     _check(st, "moe_forward")
+
+
+def moe_forward_decode(cfg, x, w_router, router_bias, w_gate_up, w_down, y, losses, topk_idx, topk_w, ws,
+                       stream=None):
+    """The one-kernel decode layer (T <= 8); moe_forward picks it by itself when
+    nothing is saved for the backward."""
+    dt = torch_dtype(cfg)
+    T, d, E, k, f = cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff
+    st = lib().moe_forward_decode(
+        _cfgp(cfg), _ptr(x, dt, (T, d), "x"), _ptr(w_router, dt, (E, d), "w_router"),
+        _ptr(router_bias, torch.float32, (E,), "router_bias", allow_none=True),
+        _ptr(w_gate_up, dt, (E, 2 * f, d), "w_gate_up"), _ptr(w_down, dt, (E, d, f), "w_down"),
+        _ptr(y, dt, (T, d), "y"), _ptr(losses, torch.float32, (2,), "losses", allow_none=True),
+        _ptr(topk_idx, torch.int32, (T, k), "topk_idx", allow_none=True),
+        _ptr(topk_w, torch.float32, (T, k), "topk_w", allow_none=True),
+        _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
+    _check(st, "moe_forward_decode")
 
 
 def moe_expert_choice_capacity(cfg) -> int:

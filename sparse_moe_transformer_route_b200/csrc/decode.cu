@@ -1,0 +1,492 @@
+// The whole MoE layer for a decode-sized batch (T <= 8 tokens) in one
+// persistent cooperative kernel: router, gate/up + SwiGLU, down and combine,
+// optionally with the block's RMSNorm in front and the residual add behind.
+//
+// Method: the layer of "Mixture-of-experts LLMs from scratch with OLMoE",
+// section 2 (softmax over all experts, top-k without renormalisation, each
+// expert once on its tokens, weighted sum back) and section 3 (the Block:
+// r + MoE(RMSNorm(r)) on an fp32 residual), the SwiGLU expert of "OLMoE
+// Guide", "Top-8 Softmax Routing Formulation", and its losses ("Router
+// Mechanics & Loss Formulations"). Section 6 of the lesson notes that at a
+// batch of one token the layer reads only the k chosen experts' weights, so
+// decoding is bound by streaming those weights; this kernel exists to stream
+// them with nothing else in the way (one launch, two grid barriers).
+//
+// One CTA per SM (grid = SM count, cooperative launch, 16 warps):
+//   prologue  every CTA stages the T input rows in shared memory (with the
+//             RMSNorm applied when the input is the fp32 residual).
+//   phase 0   the T*E router logits, one warp per (token, expert): products of
+//             bf16 values are exact in fp32 and are summed in fp64, so the
+//             logits are exact to ~1e-16 and the top-k matches an exact
+//             computation except for exactly equal logits (lower index wins).
+//   barrier
+//   phase 0b  every CTA: softmax (fp64), top-k, weights, the list of touched
+//             experts with their tokens; CTA 0 writes the losses, counts and
+//             the optional top-k outputs.
+//   phase 1   one warp per (touched expert, hidden row i): the gate row i and
+//             the up row i stream once from HBM and meet every token that chose
+//             the expert; h = SiLU(g) * u is stored in bf16 (as the grouped
+//             GEMM stores it).
+//   barrier
+//   phase 2   every CTA stages h; one warp per output column c: row c of each
+//             touched expert's down matrix streams once, its dot products with
+//             the tokens' h rows are summed per token in slot order in fp32,
+//             weighted, and written once (bf16 y, or added to the residual).
+// The grid barrier is an arrival counter and a generation word in the
+// workspace; each wait gives up after about a second, records a status and
+// lets the kernel finish.
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kDecThreads = 512;
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kDecMaxT = 8;
+constexpr int kDecMaxE = 64;
+constexpr int kDecSlots = kDecMaxT * kMaxTopK;            // (token, slot) pairs
+constexpr size_t kDecActBytes = 160 * 1024;               // staged x, then h
+constexpr size_t kDecMiscBytes = 24 * 1024;
+constexpr size_t kDecSmem = kDecActBytes + kDecMiscBytes;
+
+struct DecArgs {
+  int T, d, E, k, f;
+  int renorm;
+  float eps;
+  const __nv_bfloat16* x;    // [T, d] layer input, or null when `resid` is the input
+  float* resid;              // [T, d] fp32 residual (in/out), or null
+  const __nv_bfloat16* wr;   // [E, d]
+  const float* bias;         // [E] or null
+  const __nv_bfloat16* wgu;  // [E, 2f, d]
+  const __nv_bfloat16* wd;   // [E, d, f]
+  __nv_bfloat16* y;          // [T, d] out (null with `resid`)
+  double* logits;            // [T, E] workspace
+  __nv_bfloat16* h;          // [T*k, f] workspace
+  int32_t* idx_out;          // [T, k] or null
+  float* w_out;              // [T, k] or null
+  int32_t* counts;           // [E] or null
+  float* losses;             // [2] or null
+  float* losses_ws;          // [2] workspace copy
+  unsigned* bar;             // [2] arrival count, generation
+  int32_t* status;
+};
+
+struct DecSmem {
+  int sel_e[kDecSlots];
+  float sel_w[kDecSlots];
+  float ps[kDecWarps][kDecSlots];  // per-warp dot products of one output column
+  int touched[kDecMaxE];           // experts chosen by some token, ascending
+  int n_tok[kDecMaxE];             // by expert id: tokens that chose it
+  int tok_t[kDecMaxE][kDecMaxT];   // by expert id: the token, in token order
+  int tok_j[kDecMaxE][kDecMaxT];   // by expert id: the slot that token used
+  int n_touched;
+  int ok;
+  float inv_rms[kDecMaxT];
+  double p[kDecMaxT][kDecMaxE];
+  double lse[kDecMaxT];
+};
+static_assert(sizeof(DecSmem) <= kDecMiscBytes, "decode bookkeeping fits");
+
+// Grid-wide barrier (all CTAs co-resident: cooperative launch). Returns false
+// when the wait gave up; the failure is recorded and every CTA then unwinds.
+__device__ bool grid_barrier(unsigned* bar, unsigned n, int32_t* status, int* ok_s) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile unsigned* gen = bar + 1;
+    const unsigned g = *gen;
+    __threadfence();
+    int ok = 1;
+    if (atomicAdd(bar, 1u) == n - 1) {
+      atomicExch(bar, 0u);
+      __threadfence();
+      atomicAdd(bar + 1, 1u);
+    } else {
+      const uint64_t t0 = global_timer_ns();
+      uint32_t spins = 0;
+      while (*gen == g) {
+        __nanosleep(64);
+        if (((++spins) & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+          report(status, DEV_WAIT_TIMEOUT_GRID);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    *ok_s = ok;
+  }
+  __syncthreads();
+  return *ok_s != 0;
+}
+
+__device__ __forceinline__ void bf16x8(const uint4& q, float (&v)[8]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+    v[2 * j] = f2.x;
+    v[2 * j + 1] = f2.y;
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __nv_bfloat16* act = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // x [T, d], later h [T*k, f]
+  DecSmem& m = *reinterpret_cast<DecSmem*>(smem_raw + kDecActBytes);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = a.T, d = a.d, E = a.E, k = a.k, f = a.f;
+  const int nvd = d / 8, nvf = f / 8;  // 16-byte vectors per row
+  const int gw = blockIdx.x * kDecWarps + warp;
+  const int nw = gridDim.x * kDecWarps;
+
+  // ---- prologue: the T input rows, bf16, in shared memory
+  if (a.resid != nullptr) {
+    if (warp < T) {  // RMSNorm (unit weight) of token `warp`: mean of squares in a fixed order
+      const float* r = a.resid + static_cast<int64_t>(warp) * d;
+      float ss = 0.f;
+      for (int i = lane; i < d; i += 32) ss = fmaf(r[i], r[i], ss);
+      ss = warp_sum(ss);
+      if (lane == 0) m.inv_rms[warp] = rsqrtf(ss / static_cast<float>(d) + a.eps);
+    }
+    __syncthreads();
+    for (int i = tid; i < T * d; i += kDecThreads) act[i] = __float2bfloat16_rn(a.resid[i] * m.inv_rms[i / d]);
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(a.x);
+    uint4* dst = reinterpret_cast<uint4*>(act);
+    for (int i = tid; i < T * nvd; i += kDecThreads) dst[i] = __ldg(src + i);
+  }
+  if (tid < kDecMaxE) m.n_tok[tid] = 0;
+  __syncthreads();
+
+  // ---- phase 0: exact router logits, a warp per (token, expert)
+  for (int pr = gw; pr < T * E; pr += nw) {
+    const int t = pr / E, e = pr - t * E;
+    const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<int64_t>(e) * d);
+    const uint4* xrow = reinterpret_cast<const uint4*>(act + static_cast<int64_t>(t) * d);
+    double acc = 0.0;
+    for (int v0 = 0; v0 < nvd; v0 += 32 * 8) {
+      uint4 wq[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int v = v0 + j * 32 + lane;
+        if (v < nvd) wq[j] = __ldg(wrow + v);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int v = v0 + j * 32 + lane;
+        if (v < nvd) {
+          float xv[8], wv[8];
+          bf16x8(xrow[v], xv);
+          bf16x8(wq[j], wv);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc += static_cast<double>(xv[i] * wv[i]);  // exact product
+        }
+      }
+    }
+    acc = warp_sum_d(acc);
+    if (lane == 0) a.logits[pr] = acc;
+  }
+  if (!grid_barrier(a.bar, gridDim.x, a.status, &m.ok)) return;
+
+  // ---- phase 0b (every CTA): softmax, top-k, weights; warp t takes token t,
+  //      lane l holds experts l and l + 32
+  if (warp < T) {
+    const int t = warp;
+    const int e0 = lane, e1 = lane + 32;
+    double h0 = -INFINITY, h1 = -INFINITY;
+    if (e0 < E) h0 = __ldcg(a.logits + t * E + e0) + (a.bias != nullptr ? static_cast<double>(a.bias[e0]) : 0.0);
+    if (e1 < E) h1 = __ldcg(a.logits + t * E + e1) + (a.bias != nullptr ? static_cast<double>(a.bias[e1]) : 0.0);
+    double mx = fmax(h0, h1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const double x0 = e0 < E ? exp(h0 - mx) : 0.0, x1 = e1 < E ? exp(h1 - mx) : 0.0;
+    const double s = warp_sum_d(x0 + x1);
+    const double p0 = x0 / s, p1 = x1 / s;
+    if (e0 < E) m.p[t][e0] = p0;
+    if (e1 < E) m.p[t][e1] = p1;
+    if (lane == 0) m.lse[t] = mx + log(s);
+    // top-k by logit: larger wins, equal values go to the lower expert index
+    bool tk0 = e0 >= E, tk1 = e1 >= E;
+    double wsum = 0.0;
+    double pj[kMaxTopK];
+    int ej[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j < k) {
+        double v = -INFINITY;
+        int bi = 0x7fffffff;
+        if (!tk0) {
+          v = h0;
+          bi = e0;
+        }
+        if (!tk1 && (bi == 0x7fffffff || h1 > v)) {
+          v = h1;
+          bi = e1;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const double ov = __shfl_xor_sync(0xffffffffu, v, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > v || (ov == v && oi < bi))) {
+            v = ov;
+            bi = oi;
+          }
+        }
+        if (bi == e0) tk0 = true;
+        if (bi == e1) tk1 = true;
+        const double pw = __shfl_sync(0xffffffffu, bi >= 32 ? p1 : p0, bi & 31);
+        pj[j] = pw;
+        ej[j] = bi;
+        wsum += pw;
+      }
+    }
+    if (lane == 0) {
+      for (int j = 0; j < k; ++j) {
+        const float w = static_cast<float>(a.renorm ? pj[j] / wsum : pj[j]);
+        m.sel_e[t * k + j] = ej[j];
+        m.sel_w[t * k + j] = w;
+        if (blockIdx.x == 0) {
+          if (a.idx_out != nullptr) a.idx_out[t * k + j] = ej[j];
+          if (a.w_out != nullptr) a.w_out[t * k + j] = w;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // tokens of each expert, in token order (thread e scans the choices)
+  if (tid < E) {
+    int n = 0;
+    for (int t = 0; t < T; ++t)
+      for (int j = 0; j < k; ++j)
+        if (m.sel_e[t * k + j] == tid) {
+          m.tok_t[tid][n] = t;
+          m.tok_j[tid][n] = j;
+          ++n;
+        }
+    m.n_tok[tid] = n;
+  }
+  __syncthreads();
+  if (warp == 0) {  // the touched experts, ascending
+    int base = 0;
+    for (int c = 0; c < E; c += 32) {
+      const int e = c + lane;
+      const bool on = e < E && m.n_tok[e] > 0;
+      const unsigned b = __ballot_sync(0xffffffffu, on);
+      if (on) m.touched[base + __popc(b & ((1u << lane) - 1u))] = e;
+      base += __popc(b);
+    }
+    if (lane == 0) m.n_touched = base;
+    if (blockIdx.x == 0) {  // losses and counts: E * sum_e (c_e / (T k)) (P_e / T), mean lse^2
+      double lb = 0.0;
+      for (int c = 0; c < E; c += 32) {
+        const int e = c + lane;
+        if (e < E) {
+          double pe = 0.0;
+          for (int t = 0; t < T; ++t) pe += m.p[t][e];
+          lb += static_cast<double>(m.n_tok[e]) * pe;
+          if (a.counts != nullptr) a.counts[e] = m.n_tok[e];
+        }
+      }
+      lb = warp_sum_d(lb);
+      if (lane == 0) {
+        double z = 0.0;
+        for (int t = 0; t < T; ++t) z += m.lse[t] * m.lse[t];
+        const double Td = static_cast<double>(T);
+        const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(z / Td);
+        a.losses_ws[0] = l0;
+        a.losses_ws[1] = l1;
+        if (a.losses != nullptr) {
+          a.losses[0] = l0;
+          a.losses[1] = l1;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int nt = m.n_touched;
+
+  // ---- phase 1: gate/up rows of the touched experts, a warp per (expert, row)
+  for (int item = gw; item < nt * f; item += nw) {
+    const int u = item / f, i = item - u * f;
+    const int e = m.touched[u];
+    const int n = m.n_tok[e];
+    const uint4* grow = reinterpret_cast<const uint4*>(a.wgu + (static_cast<int64_t>(e) * 2 * f + i) * d);
+    const uint4* urow = grow + static_cast<int64_t>(f) * nvd;
+    float ag[kDecMaxT], au[kDecMaxT];
+#pragma unroll
+    for (int q = 0; q < kDecMaxT; ++q) ag[q] = au[q] = 0.f;
+    for (int v0 = 0; v0 < nvd; v0 += 32 * 4) {
+      uint4 gq[4], uq[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int v = v0 + j * 32 + lane;
+        if (v < nvd) {
+          gq[j] = __ldg(grow + v);
+          uq[j] = __ldg(urow + v);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int v = v0 + j * 32 + lane;
+        if (v < nvd) {
+          float gv[8], uv[8];
+          bf16x8(gq[j], gv);
+          bf16x8(uq[j], uv);
+#pragma unroll
+          for (int q = 0; q < kDecMaxT; ++q) {
+            if (q < n) {
+              float xv[8];
+              bf16x8(reinterpret_cast<const uint4*>(act + static_cast<int64_t>(m.tok_t[e][q]) * d)[v], xv);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                ag[q] = fmaf(gv[c], xv[c], ag[q]);
+                au[q] = fmaf(uv[c], xv[c], au[q]);
+              }
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kDecMaxT; ++q) {
+      if (q < n) {
+        const float g = warp_sum(ag[q]), uu = warp_sum(au[q]);
+        if (lane == 0) {
+          const int slot = m.tok_t[e][q] * k + m.tok_j[e][q];
+          a.h[static_cast<int64_t>(slot) * f + i] = __float2bfloat16_rn(silu_fast(g) * uu);
+        }
+      }
+    }
+  }
+  if (!grid_barrier(a.bar, gridDim.x, a.status, &m.ok)) return;
+
+  // ---- phase 2: h in shared memory, then a warp per output column
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.h);
+    uint4* dst = reinterpret_cast<uint4*>(act);
+    for (int i = tid; i < T * k * nvf; i += kDecThreads) dst[i] = __ldcg(src + i);
+  }
+  __syncthreads();
+  for (int c = gw; c < d; c += nw) {
+    for (int u0 = 0; u0 < nt; u0 += 4) {
+      uint4 wq[4][4];  // four experts' rows, four 16-byte vectors per lane at a time
+      for (int v0 = 0; v0 < nvf; v0 += 32 * 4) {
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+          if (u0 + uu < nt) {
+            const uint4* row =
+                reinterpret_cast<const uint4*>(a.wd + (static_cast<int64_t>(m.touched[u0 + uu]) * d + c) * f);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int v = v0 + j * 32 + lane;
+              if (v < nvf) wq[uu][j] = __ldg(row + v);
+            }
+          }
+        }
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+          if (u0 + uu < nt) {
+            const int e = m.touched[u0 + uu];
+            const int n = m.n_tok[e];
+            for (int q = 0; q < n; ++q) {
+              const int slot = m.tok_t[e][q] * k + m.tok_j[e][q];
+              const uint4* hrow = reinterpret_cast<const uint4*>(act + static_cast<int64_t>(slot) * f);
+              float acc = 0.f;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int v = v0 + j * 32 + lane;
+                if (v < nvf) {
+                  float wv[8], hv[8];
+                  bf16x8(wq[uu][j], wv);
+                  bf16x8(hrow[v], hv);
+#pragma unroll
+                  for (int cc = 0; cc < 8; ++cc) acc = fmaf(wv[cc], hv[cc], acc);
+                }
+              }
+              acc = warp_sum(acc);
+              if (lane == 0) m.ps[warp][slot] = (v0 == 0 ? 0.f : m.ps[warp][slot]) + acc;
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane < T) {  // token `lane`: weighted sum over its slots, in slot order
+      float acc = 0.f;
+      for (int j = 0; j < k; ++j) acc = fmaf(m.sel_w[lane * k + j], m.ps[warp][lane * k + j], acc);
+      const int64_t o = static_cast<int64_t>(lane) * d + c;
+      if (a.resid != nullptr)
+        a.resid[o] += acc;
+      else
+        a.y[o] = __float2bfloat16_rn(acc);
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+bool decode_supported(const Shape& s) {
+  if (s.fp32 || s.T > kDecMaxT || s.E > kDecMaxE || s.k > kMaxTopK) return false;
+  const size_t x_bytes = static_cast<size_t>(s.T) * s.d * 2, h_bytes = static_cast<size_t>(s.T) * s.k * s.f * 2;
+  return x_bytes <= kDecActBytes && h_bytes <= kDecActBytes;
+}
+
+cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, float eps, const void* w_router,
+                                const float* bias, const void* w_gate_up, const void* w_down, void* y,
+                                int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,
+                                const Workspace& L, cudaStream_t st) {
+  static std::atomic<size_t> set_smem[kMaxDevices];
+  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(decode_layer_kernel), kDecSmem, set_smem);
+  if (e != cudaSuccess) return e;
+  DecArgs a{};
+  a.T = static_cast<int>(s.T);
+  a.d = s.d;
+  a.E = s.E;
+  a.k = s.k;
+  a.f = s.f;
+  a.renorm = s.renorm ? 1 : 0;
+  a.eps = eps;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.resid = resid;
+  a.wr = static_cast<const __nv_bfloat16*>(w_router);
+  a.bias = bias;
+  a.wgu = static_cast<const __nv_bfloat16*>(w_gate_up);
+  a.wd = static_cast<const __nv_bfloat16*>(w_down);
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.logits = at<double>(ws, L.o_perm);
+  a.h = at<__nv_bfloat16>(ws, L.h);
+  a.idx_out = topk_idx;
+  a.w_out = topk_w;
+  a.counts = counts;
+  a.losses = losses;
+  a.losses_ws = at<float>(ws, L.losses);
+  a.bar = reinterpret_cast<unsigned*>(at<int32_t>(ws, L.ctrl) + 3);
+  a.status = at<int32_t>(ws, L.ctrl);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(device_sm_count()));
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = kDecSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_layer_kernel, a);
+}
+
+}  // namespace moe

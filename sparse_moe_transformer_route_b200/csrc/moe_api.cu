@@ -187,6 +187,13 @@ moe_status forward_impl(const Ctx& c, const void* x, const void* w_router, const
   void* x_perm = at<void>(ws, L.x_perm);
   const StageMarks marks(st);
   MOE_TRY(marks.mark(0));
+  if (!save && resid == nullptr && decode_supported(s)) {
+    // a decode-sized batch: the whole layer in one kernel (every stage mark after it)
+    MOE_TRY(launch_decode_layer(s, x, nullptr, 0.f, w_router, bias, w_gate_up, w_down, y, topk_idx, topk_w, counts,
+                                losses, ws, L, st));
+    for (int i = 1; i <= 5; ++i) MOE_TRY(marks.mark(i));
+    return MOE_OK;
+  }
   if (router_tc_supported(s)) {
     // the tensor-core router also leaves the dispatch ranking in ws
     MOE_TRY(launch_router_tc(s, x, w_router, bias, idx, wts, counts, losses, ws, L, st));
@@ -370,6 +377,21 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
                       save_for_backward != 0, ws, stream);
 }
 
+moe_status moe_forward_decode(const moe_config* cfg, const void* x, const void* w_router, const float* router_bias,
+                              const void* w_gate_up, const void* w_down, void* y, float* losses, int32_t* topk_idx,
+                              float* topk_w, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  Ctx c;
+  moe_status r = prepare(cfg, ws, ws_bytes, false, &c);
+  if (r != MOE_OK) return r;
+  if (!decode_supported(c.s)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (x == nullptr || w_router == nullptr || w_gate_up == nullptr || w_down == nullptr || y == nullptr ||
+      !aligned16(x) || !aligned16(w_router) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(launch_decode_layer(c.s, x, nullptr, 0.f, w_router, router_bias, w_gate_up, w_down, y, topk_idx, topk_w,
+                              nullptr, losses, ws, c.L, stream));
+  return MOE_OK;
+}
+
 moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const void* w_router,
                             const float* router_bias, const void* w_gate_up, const void* w_down, void* y_host,
                             float* losses_host, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -518,6 +540,16 @@ moe_status moe_stack_forward_trace(const moe_config* cfg, int32_t n_layers, cons
     if (w_router[l] == nullptr || w_gate_up[l] == nullptr || w_down[l] == nullptr) return MOE_ERR_INVALID_ARG;
   void* xn = at<void>(ws, c.L.x_dev);
   const int64_t tk = c.s.T * c.s.k;
+  if (decode_supported(c.s)) {  // decode-sized batch: RMSNorm, layer and residual add in one kernel per layer
+    for (int l = 0; l < n_layers; ++l) {
+      const float* bias = (router_biases != nullptr) ? router_biases[l] : nullptr;
+      MOE_TRY(launch_decode_layer(c.s, nullptr, resid, 1e-5f, w_router[l], bias, w_gate_up[l], w_down[l], nullptr,
+                                  topk_idx != nullptr ? topk_idx + l * tk : nullptr, nullptr,
+                                  counts != nullptr ? counts + static_cast<int64_t>(l) * c.s.E : nullptr,
+                                  losses != nullptr ? losses + 2 * l : nullptr, ws, c.L, stream));
+    }
+    return MOE_OK;
+  }
   for (int l = 0; l < n_layers; ++l) {
     MOE_TRY(launch_rmsnorm(c.s, resid, nullptr, 1e-5f, xn, stream));
     const float* bias = (router_biases != nullptr) ? router_biases[l] : nullptr;
@@ -558,7 +590,7 @@ moe_status moe_get_device_status(void* ws, int32_t* code, cudaStream_t stream) {
   MOE_TRY(cudaStreamSynchronize(stream));
   // the status word and, with it, the completion counters: a launch that gave
   // up part-way may have left a counter behind
-  MOE_TRY(cudaMemsetAsync(ws, 0, 3 * sizeof(int32_t), stream));
+  MOE_TRY(cudaMemsetAsync(ws, 0, 4 * sizeof(int32_t), stream));
   *code = v;
   return v == 0 ? MOE_OK : MOE_ERR_DEVICE_CHECK;
 }

@@ -33,7 +33,8 @@ struct Shape {
 
 // Byte offsets of every region inside the caller's workspace.
 struct Workspace {
-  // control words: [0] status, [1] router ticket, [2] dispatch ticket
+  // control words: [0] status, [1] router ticket, [2] dispatch ticket,
+  // [3] grid-barrier arrivals, [4] grid-barrier generation
   size_t ctrl;
   size_t counts_part, psum_part, zsum_part;  // router per-CTA partials
   size_t counts, losses;                     // router totals
@@ -92,6 +93,15 @@ cudaError_t launch_ec_gather(const Shape& s, int64_t C, const void* x, void* ws,
                              cudaStream_t st);
 cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t* slot_row, const float* probs,
                               void* y, cudaStream_t st);
+// Fused decode layer (T <= 8, bf16, E <= 64, staged rows within shared memory):
+// the whole forward in one cooperative kernel. With `resid` non-null the input
+// is RMSNorm(resid) (unit weight, eps) and the output is added to resid;
+// otherwise x -> y. Forward only (nothing is kept for the backward).
+bool decode_supported(const Shape& s);
+cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, float eps, const void* w_router,
+                                const float* bias, const void* w_gate_up, const void* w_down, void* y,
+                                int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,
+                                const Workspace& L, cudaStream_t st);
 cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, float eps, void* out,
                            cudaStream_t st);
 

@@ -19,6 +19,7 @@ enum DeviceCode : int32_t {
   DEV_WAIT_TIMEOUT_MMA = 0x102,
   DEV_WAIT_TIMEOUT_EPILOGUE = 0x103,
   DEV_WAIT_TIMEOUT_DRAIN = 0x104,
+  DEV_WAIT_TIMEOUT_GRID = 0x105,
   DEV_BAD_EXPERT_INDEX = 0x201,
   DEV_COUNT_MISMATCH = 0x202,
 };

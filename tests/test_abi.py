@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol():
 def test_library_has_no_gpu_only_load_dependencies():
     # static CUDA runtime: the .so must load here, where there is no driver
     lib = M.lib()
-    assert lib.moe_abi_version() == B.ABI_VERSION == 4
+    assert lib.moe_abi_version() == B.ABI_VERSION == 5
 
 
 def test_status_strings():
