@@ -227,9 +227,10 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
  * summed in fp64 from exact products, so the choice is the exact one (equal
  * logits: the lower expert index). Same arguments and results as moe_forward
  * without save_for_backward (counts are not written). moe_forward takes this
- * path by itself for T <= 8 when nothing is saved for the backward, and
- * moe_stack_forward(_trace) runs each layer of such a batch as one launch of
- * it with the RMSNorm and the residual add fused.
+ * path by itself for T <= 4 when nothing is saved for the backward (beyond
+ * that the layered tensor-core path is as fast), and moe_stack_forward(_trace)
+ * runs each layer of such a batch as one launch of it with the RMSNorm and the
+ * residual add fused.
  * Supported: bf16, T <= 8, E <= 64, T*d*2 and T*k*f*2 bytes each at most
  * 160 KiB; otherwise MOE_ERR_UNSUPPORTED_SHAPE. */
 moe_status moe_forward_decode(const moe_config* cfg, const void* x, const void* w_router, const float* router_bias,

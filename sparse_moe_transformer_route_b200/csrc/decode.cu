@@ -20,11 +20,13 @@
 //             logits are exact to ~1e-16 and the top-k matches an exact
 //             computation except for exactly equal logits (lower index wins).
 //   barrier
-//   phase 0b  every CTA: softmax (fp64), top-k, weights, the list of touched
-//             experts with their tokens; CTA 0 writes the losses, counts and
-//             the optional top-k outputs.
+//   phase 0b  every CTA: each expert's rank among a token's logits gives the
+//             top-k at once (no sequential selection); softmax in fp32; the
+//             tokens of each expert as a bit mask; CTA 0 writes the losses,
+//             counts and the optional top-k outputs.
 //   phase 1   one warp per (touched expert, hidden row i): the gate row i and
-//             the up row i stream once from HBM and meet every token that chose
+//             the up row i stream once from HBM (all of the pair's loads in
+//             flight before any arithmetic) and meet every token that chose
 //             the expert; h = SiLU(g) * u is stored in bf16 (as the grouped
 //             GEMM stores it).
 //   barrier
@@ -34,7 +36,8 @@
 //             weighted, and written once (bf16 y, or added to the residual).
 // The grid barrier is an arrival counter and a generation word in the
 // workspace; each wait gives up after about a second, records a status and
-// lets the kernel finish.
+// lets the kernel finish. Every single-lane section rejoins its warp
+// (__syncwarp) before a block-wide barrier.
 #include "moe_internal.h"
 #include "sm100.cuh"
 
@@ -47,7 +50,7 @@ constexpr int kDecMaxT = 8;
 constexpr int kDecMaxE = 64;
 constexpr int kDecSlots = kDecMaxT * kMaxTopK;            // (token, slot) pairs
 constexpr size_t kDecActBytes = 160 * 1024;               // staged x, then h
-constexpr size_t kDecMiscBytes = 24 * 1024;
+constexpr size_t kDecMiscBytes = 28 * 1024;
 constexpr size_t kDecSmem = kDecActBytes + kDecMiscBytes;
 
 struct DecArgs {
@@ -76,21 +79,22 @@ struct DecSmem {
   int sel_e[kDecSlots];
   float sel_w[kDecSlots];
   float ps[kDecWarps][kDecSlots];  // per-warp dot products of one output column
+  unsigned tokmask[kDecMaxE];      // bit t: token t chose the expert
+  int slot_of[kDecMaxT][kDecMaxE]; // slot of expert e among token t's choices, or -1
   int touched[kDecMaxE];           // experts chosen by some token, ascending
-  int n_tok[kDecMaxE];             // by expert id: tokens that chose it
-  int tok_t[kDecMaxE][kDecMaxT];   // by expert id: the token, in token order
-  int tok_j[kDecMaxE][kDecMaxT];   // by expert id: the slot that token used
   int n_touched;
   int ok;
   float inv_rms[kDecMaxT];
-  double p[kDecMaxT][kDecMaxE];
-  double lse[kDecMaxT];
+  double hd[kDecMaxT][kDecMaxE];   // logits (+ offset)
+  float p[kDecMaxT][kDecMaxE];
+  float lse[kDecMaxT];
 };
 static_assert(sizeof(DecSmem) <= kDecMiscBytes, "decode bookkeeping fits");
 
 // Grid-wide barrier (all CTAs co-resident: cooperative launch). Returns false
 // when the wait gave up; the failure is recorded and every CTA then unwinds.
 __device__ bool grid_barrier(unsigned* bar, unsigned n, int32_t* status, int* ok_s) {
+  __syncwarp();
   __syncthreads();
   if (threadIdx.x == 0) {
     volatile unsigned* gen = bar + 1;
@@ -105,8 +109,8 @@ __device__ bool grid_barrier(unsigned* bar, unsigned n, int32_t* status, int* ok
       const uint64_t t0 = global_timer_ns();
       uint32_t spins = 0;
       while (*gen == g) {
-        __nanosleep(64);
-        if (((++spins) & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+        if (++spins > 1024u) __nanosleep(32);
+        if ((spins & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
           report(status, DEV_WAIT_TIMEOUT_GRID);
           ok = 0;
           break;
@@ -116,6 +120,7 @@ __device__ bool grid_barrier(unsigned* bar, unsigned n, int32_t* status, int* ok
     __threadfence();
     *ok_s = ok;
   }
+  __syncwarp();  // warp 0 whole again before the block barrier
   __syncthreads();
   return *ok_s != 0;
 }
@@ -160,6 +165,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
       for (int i = lane; i < d; i += 32) ss = fmaf(r[i], r[i], ss);
       ss = warp_sum(ss);
       if (lane == 0) m.inv_rms[warp] = rsqrtf(ss / static_cast<float>(d) + a.eps);
+      __syncwarp();
     }
     __syncthreads();
     for (int i = tid; i < T * d; i += kDecThreads) act[i] = __float2bfloat16_rn(a.resid[i] * m.inv_rms[i / d]);
@@ -168,7 +174,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
     uint4* dst = reinterpret_cast<uint4*>(act);
     for (int i = tid; i < T * nvd; i += kDecThreads) dst[i] = __ldg(src + i);
   }
-  if (tid < kDecMaxE) m.n_tok[tid] = 0;
+  if (tid < kDecMaxE) m.tokmask[tid] = 0u;
+  if (tid < kDecSlots) m.sel_e[tid] = 0;  // defined even if non-finite logits leave a slot unranked
   __syncthreads();
 
   // ---- phase 0: exact router logits, a warp per (token, expert)
@@ -201,109 +208,87 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
   }
   if (!grid_barrier(a.bar, gridDim.x, a.status, &m.ok)) return;
 
-  // ---- phase 0b (every CTA): softmax, top-k, weights; warp t takes token t,
-  //      lane l holds experts l and l + 32
+  // ---- phase 0b (every CTA): warp t takes token t; lane l holds experts l, l + 32
   if (warp < T) {
     const int t = warp;
     const int e0 = lane, e1 = lane + 32;
     double h0 = -INFINITY, h1 = -INFINITY;
     if (e0 < E) h0 = __ldcg(a.logits + t * E + e0) + (a.bias != nullptr ? static_cast<double>(a.bias[e0]) : 0.0);
     if (e1 < E) h1 = __ldcg(a.logits + t * E + e1) + (a.bias != nullptr ? static_cast<double>(a.bias[e1]) : 0.0);
+    if (e0 < E) m.hd[t][e0] = h0;
+    if (e1 < E) m.hd[t][e1] = h1;
+    __syncwarp();
+    // rank by (logit descending, index ascending): the experts ranked below k are the choice
+    int r0 = 0, r1 = 0;
+    for (int e = 0; e < E; ++e) {
+      const double v = m.hd[t][e];
+      r0 += (v > h0 || (v == h0 && e < e0)) ? 1 : 0;
+      r1 += (v > h1 || (v == h1 && e < e1)) ? 1 : 0;
+    }
+    if (e0 < E) {
+      m.slot_of[t][e0] = r0 < k ? r0 : -1;
+      if (r0 < k) {
+        m.sel_e[t * k + r0] = e0;
+        atomicOr(&m.tokmask[e0], 1u << t);
+      }
+    }
+    if (e1 < E) {
+      m.slot_of[t][e1] = r1 < k ? r1 : -1;
+      if (r1 < k) {
+        m.sel_e[t * k + r1] = e1;
+        atomicOr(&m.tokmask[e1], 1u << t);
+      }
+    }
+    // softmax over all experts in fp32 from the exact logits
     double mx = fmax(h0, h1);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const double x0 = e0 < E ? exp(h0 - mx) : 0.0, x1 = e1 < E ? exp(h1 - mx) : 0.0;
-    const double s = warp_sum_d(x0 + x1);
-    const double p0 = x0 / s, p1 = x1 / s;
-    if (e0 < E) m.p[t][e0] = p0;
-    if (e1 < E) m.p[t][e1] = p1;
-    if (lane == 0) m.lse[t] = mx + log(s);
-    // top-k by logit: larger wins, equal values go to the lower expert index
-    bool tk0 = e0 >= E, tk1 = e1 >= E;
-    double wsum = 0.0;
-    double pj[kMaxTopK];
-    int ej[kMaxTopK];
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < k) {
-        double v = -INFINITY;
-        int bi = 0x7fffffff;
-        if (!tk0) {
-          v = h0;
-          bi = e0;
-        }
-        if (!tk1 && (bi == 0x7fffffff || h1 > v)) {
-          v = h1;
-          bi = e1;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const double ov = __shfl_xor_sync(0xffffffffu, v, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > v || (ov == v && oi < bi))) {
-            v = ov;
-            bi = oi;
-          }
-        }
-        if (bi == e0) tk0 = true;
-        if (bi == e1) tk1 = true;
-        const double pw = __shfl_sync(0xffffffffu, bi >= 32 ? p1 : p0, bi & 31);
-        pj[j] = pw;
-        ej[j] = bi;
-        wsum += pw;
-      }
-    }
-    if (lane == 0) {
+    const float x0 = e0 < E ? expf(static_cast<float>(h0 - mx)) : 0.f;
+    const float x1 = e1 < E ? expf(static_cast<float>(h1 - mx)) : 0.f;
+    const float sum = warp_sum(x0 + x1);
+    if (e0 < E) m.p[t][e0] = x0 / sum;
+    if (e1 < E) m.p[t][e1] = x1 / sum;
+    if (lane == 0) m.lse[t] = static_cast<float>(mx) + logf(sum);
+    __syncwarp();
+    if (lane == 0) {  // weights in slot order (renormalised: over the k chosen, summed in slot order)
+      float den = 0.f;
+      for (int j = 0; j < k; ++j) den += m.p[t][m.sel_e[t * k + j]];
       for (int j = 0; j < k; ++j) {
-        const float w = static_cast<float>(a.renorm ? pj[j] / wsum : pj[j]);
-        m.sel_e[t * k + j] = ej[j];
+        const int e = m.sel_e[t * k + j];
+        const float w = a.renorm ? m.p[t][e] / den : m.p[t][e];
         m.sel_w[t * k + j] = w;
         if (blockIdx.x == 0) {
-          if (a.idx_out != nullptr) a.idx_out[t * k + j] = ej[j];
+          if (a.idx_out != nullptr) a.idx_out[t * k + j] = e;
           if (a.w_out != nullptr) a.w_out[t * k + j] = w;
         }
       }
     }
+    __syncwarp();
   }
   __syncthreads();
-  // tokens of each expert, in token order (thread e scans the choices)
-  if (tid < E) {
-    int n = 0;
-    for (int t = 0; t < T; ++t)
-      for (int j = 0; j < k; ++j)
-        if (m.sel_e[t * k + j] == tid) {
-          m.tok_t[tid][n] = t;
-          m.tok_j[tid][n] = j;
-          ++n;
-        }
-    m.n_tok[tid] = n;
-  }
-  __syncthreads();
-  if (warp == 0) {  // the touched experts, ascending
+  if (warp == 0) {  // the touched experts, ascending; CTA 0: counts and losses
     int base = 0;
+    double lb = 0.0;
     for (int c = 0; c < E; c += 32) {
       const int e = c + lane;
-      const bool on = e < E && m.n_tok[e] > 0;
+      const bool on = e < E && m.tokmask[e] != 0u;
       const unsigned b = __ballot_sync(0xffffffffu, on);
       if (on) m.touched[base + __popc(b & ((1u << lane) - 1u))] = e;
       base += __popc(b);
+      if (blockIdx.x == 0 && e < E) {
+        const int ce = __popc(m.tokmask[e]);
+        double pe = 0.0;
+        for (int t = 0; t < T; ++t) pe += m.p[t][e];
+        lb += static_cast<double>(ce) * pe;
+        if (a.counts != nullptr) a.counts[e] = ce;
+      }
     }
     if (lane == 0) m.n_touched = base;
-    if (blockIdx.x == 0) {  // losses and counts: E * sum_e (c_e / (T k)) (P_e / T), mean lse^2
-      double lb = 0.0;
-      for (int c = 0; c < E; c += 32) {
-        const int e = c + lane;
-        if (e < E) {
-          double pe = 0.0;
-          for (int t = 0; t < T; ++t) pe += m.p[t][e];
-          lb += static_cast<double>(m.n_tok[e]) * pe;
-          if (a.counts != nullptr) a.counts[e] = m.n_tok[e];
-        }
-      }
+    if (blockIdx.x == 0) {  // E * sum_e (c_e / (T k)) (P_e / T), and the mean of lse^2
       lb = warp_sum_d(lb);
       if (lane == 0) {
         double z = 0.0;
-        for (int t = 0; t < T; ++t) z += m.lse[t] * m.lse[t];
+        for (int t = 0; t < T; ++t) z += static_cast<double>(m.lse[t]) * m.lse[t];
         const double Td = static_cast<double>(T);
         const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(z / Td);
         a.losses_ws[0] = l0;
@@ -314,24 +299,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
         }
       }
     }
+    __syncwarp();
   }
   __syncthreads();
   const int nt = m.n_touched;
 
-  // ---- phase 1: gate/up rows of the touched experts, a warp per (expert, row)
+  // ---- phase 1: gate/up rows of the touched experts, a warp per (expert, row);
+  //      the whole row pair's loads are in flight before any arithmetic
   for (int item = gw; item < nt * f; item += nw) {
     const int u = item / f, i = item - u * f;
     const int e = m.touched[u];
-    const int n = m.n_tok[e];
+    const unsigned tmask = m.tokmask[e];
     const uint4* grow = reinterpret_cast<const uint4*>(a.wgu + (static_cast<int64_t>(e) * 2 * f + i) * d);
     const uint4* urow = grow + static_cast<int64_t>(f) * nvd;
     float ag[kDecMaxT], au[kDecMaxT];
 #pragma unroll
     for (int q = 0; q < kDecMaxT; ++q) ag[q] = au[q] = 0.f;
-    for (int v0 = 0; v0 < nvd; v0 += 32 * 4) {
-      uint4 gq[4], uq[4];
+    for (int v0 = 0; v0 < nvd; v0 += 32 * 8) {
+      uint4 gq[8], uq[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const int v = v0 + j * 32 + lane;
         if (v < nvd) {
           gq[j] = __ldg(grow + v);
@@ -339,7 +326,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
         }
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const int v = v0 + j * 32 + lane;
         if (v < nvd) {
           float gv[8], uv[8];
@@ -347,9 +334,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
           bf16x8(uq[j], uv);
 #pragma unroll
           for (int q = 0; q < kDecMaxT; ++q) {
-            if (q < n) {
+            if ((tmask >> q) & 1u) {
               float xv[8];
-              bf16x8(reinterpret_cast<const uint4*>(act + static_cast<int64_t>(m.tok_t[e][q]) * d)[v], xv);
+              bf16x8(reinterpret_cast<const uint4*>(act + static_cast<int64_t>(q) * d)[v], xv);
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
                 ag[q] = fmaf(gv[c], xv[c], ag[q]);
@@ -362,10 +349,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
     }
 #pragma unroll
     for (int q = 0; q < kDecMaxT; ++q) {
-      if (q < n) {
+      if ((tmask >> q) & 1u) {
         const float g = warp_sum(ag[q]), uu = warp_sum(au[q]);
         if (lane == 0) {
-          const int slot = m.tok_t[e][q] * k + m.tok_j[e][q];
+          const int slot = q * k + m.slot_of[q][e];
           a.h[static_cast<int64_t>(slot) * f + i] = __float2bfloat16_rn(silu_fast(g) * uu);
         }
       }
@@ -400,9 +387,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
         for (int uu = 0; uu < 4; ++uu) {
           if (u0 + uu < nt) {
             const int e = m.touched[u0 + uu];
-            const int n = m.n_tok[e];
-            for (int q = 0; q < n; ++q) {
-              const int slot = m.tok_t[e][q] * k + m.tok_j[e][q];
+            unsigned tm = m.tokmask[e];
+            while (tm != 0u) {
+              const int t = __ffs(tm) - 1;
+              tm &= tm - 1u;
+              const int slot = t * k + m.slot_of[t][e];
               const uint4* hrow = reinterpret_cast<const uint4*>(act + static_cast<int64_t>(slot) * f);
               float acc = 0.f;
 #pragma unroll

@@ -337,6 +337,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     tmem_alloc(tmem_holder, C::TMEM_COLS);
     tmem_relinquish();
   }
+  __syncwarp();  // single-lane roles rejoin their warp before the block barrier
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -607,6 +608,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   }
 
+  __syncwarp();  // single-lane roles rejoin their warp before the block barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -917,6 +919,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
     }
   }
 
+  __syncwarp();  // single-lane roles rejoin their warp before the block barrier
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();

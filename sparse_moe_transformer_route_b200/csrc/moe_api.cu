@@ -187,7 +187,7 @@ moe_status forward_impl(const Ctx& c, const void* x, const void* w_router, const
   void* x_perm = at<void>(ws, L.x_perm);
   const StageMarks marks(st);
   MOE_TRY(marks.mark(0));
-  if (!save && resid == nullptr && decode_supported(s)) {
+  if (!save && resid == nullptr && s.T <= kDecodeAutoTokens && decode_supported(s)) {
     // a decode-sized batch: the whole layer in one kernel (every stage mark after it)
     MOE_TRY(launch_decode_layer(s, x, nullptr, 0.f, w_router, bias, w_gate_up, w_down, y, topk_idx, topk_w, counts,
                                 losses, ws, L, st));
@@ -540,7 +540,7 @@ moe_status moe_stack_forward_trace(const moe_config* cfg, int32_t n_layers, cons
     if (w_router[l] == nullptr || w_gate_up[l] == nullptr || w_down[l] == nullptr) return MOE_ERR_INVALID_ARG;
   void* xn = at<void>(ws, c.L.x_dev);
   const int64_t tk = c.s.T * c.s.k;
-  if (decode_supported(c.s)) {  // decode-sized batch: RMSNorm, layer and residual add in one kernel per layer
+  if (c.s.T <= kDecodeAutoTokens && decode_supported(c.s)) {  // RMSNorm, layer and residual add in one kernel
     for (int l = 0; l < n_layers; ++l) {
       const float* bias = (router_biases != nullptr) ? router_biases[l] : nullptr;
       MOE_TRY(launch_decode_layer(c.s, nullptr, resid, 1e-5f, w_router[l], bias, w_gate_up[l], w_down[l], nullptr,

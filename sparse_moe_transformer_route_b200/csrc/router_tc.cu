@@ -696,6 +696,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     const EpiSmem sm{S, P, chosen, queue, exact, qn, mask, lse_s, s_last, tot, tot_p, zred, ring};
     router_epilogue(a, sm, t0, tid, lane);
   }
+  __syncwarp();  // single-lane roles rejoin their warp before the block barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -832,6 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+  __syncwarp();  // single-lane roles rejoin their warp before the block barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

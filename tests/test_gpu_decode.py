@@ -1,11 +1,11 @@
 """The one-kernel decode layer (T <= 8) against the oracle.
 
-moe_forward takes this path by itself for decode-sized batches when nothing is
-saved for the backward, and moe_stack_forward runs each layer of such a batch
-as one launch with the RMSNorm and the residual add fused; moe_forward_decode
-calls it explicitly. Its router sums exact products in fp64, so the chosen
-experts are checked bit for bit on every token (no near-tie allowance) and the
-weights to 1e-6; outputs at the usual bars (max-abs 2e-2, relative L2 1e-2);
+moe_forward takes this path by itself for batches of up to 4 tokens when
+nothing is saved for the backward, and moe_stack_forward runs each layer of
+such a batch as one launch with the RMSNorm and the residual add fused;
+moe_forward_decode calls it explicitly for up to 8 tokens. Its router sums
+exact products in fp64, so the chosen experts are checked bit for bit on every
+token (no near-tie allowance) and the weights to 1e-6; outputs at the usual bars (max-abs 2e-2, relative L2 1e-2);
 losses to 1e-4 relative.
 """
 
@@ -72,15 +72,19 @@ def test_olmoe_shapes(olmoe_layer, T):
     _check(sh, x, *olmoe_layer, out)
 
 
-@pytest.mark.parametrize("T", [1, 8])
-def test_moe_forward_picks_the_fused_path_and_matches_the_layered_one(olmoe_layer, T):
-    """moe_forward without save_for_backward runs the one-kernel layer; with it, the
-    layered kernels. Both choose the same experts; weights and outputs agree."""
+@pytest.mark.parametrize("T", [1, 4, 8])
+def test_fused_and_layered_paths_agree(olmoe_layer, T):
+    """moe_forward without save_for_backward runs the one-kernel layer up to 4
+    tokens (bit-identical to moe_forward_decode there); with save_for_backward
+    it runs the layered kernels. Both choose the same experts; weights and
+    outputs agree."""
     sh = S.LayerShape(T=T)
     x = S.make_tokens(sh, seed=700 + T)
-    fused = _decode(sh, x, *olmoe_layer, explicit=False)
-    explicit = _decode(sh, x, *olmoe_layer, explicit=True)
-    assert torch.equal(fused["y"], explicit["y"]) and np.array_equal(fused["idx"], explicit["idx"])
+    fused = _decode(sh, x, *olmoe_layer, explicit=True)
+    auto = _decode(sh, x, *olmoe_layer, explicit=False)
+    assert np.array_equal(auto["idx"], fused["idx"])
+    if T <= 4:
+        assert torch.equal(auto["y"], fused["y"])
     cfg = M.config(T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff)
     ws = M.workspace(cfg, True)
     dev = [t.cuda() for t in (x, *olmoe_layer)]
