@@ -227,7 +227,7 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
  * summed in fp64 from exact products, so the choice is the exact one (equal
  * logits: the lower expert index). Same arguments and results as moe_forward
  * without save_for_backward (counts are not written). moe_forward takes this
- * path by itself for T <= 4 when nothing is saved for the backward (beyond
+ * path by itself for T <= 6 when nothing is saved for the backward (beyond
  * that the layered tensor-core path is as fast), and moe_stack_forward(_trace)
  * runs each layer of such a batch as one launch of it with the RMSNorm and the
  * residual add fused.

@@ -98,10 +98,11 @@ cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t*
 // is RMSNorm(resid) (unit weight, eps) and the output is added to resid;
 // otherwise x -> y. Forward only (nothing is kept for the backward).
 bool decode_supported(const Shape& s);
-// Batches the layer forward routes to the one-kernel form by itself: up to 4
-// tokens (measured on B200: T=1 57 us against 80 us layered; at T=8 the
-// layered tensor-core path is as fast, 170 against 176 us).
-constexpr int64_t kDecodeAutoTokens = 4;
+// Batches the layer forward routes to the one-kernel form by itself: up to 6
+// tokens (measured on B200, L2 flushed before each call: T=1 57 against 93 us
+// layered, T=4 125 against 159, T=6 152 against 161; at T=8 they tie, and in
+// CUDA-graph replays the layered path is ahead there, 166 against 176 us).
+constexpr int64_t kDecodeAutoTokens = 6;
 cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, float eps, const void* w_router,
                                 const float* bias, const void* w_gate_up, const void* w_down, void* y,
                                 int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,

@@ -1,6 +1,6 @@
 """The one-kernel decode layer (T <= 8) against the oracle.
 
-moe_forward takes this path by itself for batches of up to 4 tokens when
+moe_forward takes this path by itself for batches of up to 6 tokens when
 nothing is saved for the backward, and moe_stack_forward runs each layer of
 such a batch as one launch with the RMSNorm and the residual add fused;
 moe_forward_decode calls it explicitly for up to 8 tokens. Its router sums
@@ -72,9 +72,9 @@ def test_olmoe_shapes(olmoe_layer, T):
     _check(sh, x, *olmoe_layer, out)
 
 
-@pytest.mark.parametrize("T", [1, 4, 8])
+@pytest.mark.parametrize("T", [1, 6, 8])
 def test_fused_and_layered_paths_agree(olmoe_layer, T):
-    """moe_forward without save_for_backward runs the one-kernel layer up to 4
+    """moe_forward without save_for_backward runs the one-kernel layer up to 6
     tokens (bit-identical to moe_forward_decode there); with save_for_backward
     it runs the layered kernels. Both choose the same experts; weights and
     outputs agree."""
@@ -83,7 +83,7 @@ def test_fused_and_layered_paths_agree(olmoe_layer, T):
     fused = _decode(sh, x, *olmoe_layer, explicit=True)
     auto = _decode(sh, x, *olmoe_layer, explicit=False)
     assert np.array_equal(auto["idx"], fused["idx"])
-    if T <= 4:
+    if T <= 6:
         assert torch.equal(auto["y"], fused["y"])
     cfg = M.config(T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff)
     ws = M.workspace(cfg, True)
