@@ -147,6 +147,8 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
+// NT: tokens the phase-1 accumulators are sized for (1, 2, 4 or 8; T <= NT).
+template <int NT>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __nv_bfloat16* act = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // x [T, d], later h [T*k, f]
@@ -312,9 +314,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
     const unsigned tmask = m.tokmask[e];
     const uint4* grow = reinterpret_cast<const uint4*>(a.wgu + (static_cast<int64_t>(e) * 2 * f + i) * d);
     const uint4* urow = grow + static_cast<int64_t>(f) * nvd;
-    float ag[kDecMaxT], au[kDecMaxT];
+    float ag[NT], au[NT];
 #pragma unroll
-    for (int q = 0; q < kDecMaxT; ++q) ag[q] = au[q] = 0.f;
+    for (int q = 0; q < NT; ++q) ag[q] = au[q] = 0.f;
     for (int v0 = 0; v0 < nvd; v0 += 32 * 8) {
       uint4 gq[8], uq[8];
 #pragma unroll
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
           bf16x8(gq[j], gv);
           bf16x8(uq[j], uv);
 #pragma unroll
-          for (int q = 0; q < kDecMaxT; ++q) {
+          for (int q = 0; q < NT; ++q) {
             if ((tmask >> q) & 1u) {
               float xv[8];
               bf16x8(reinterpret_cast<const uint4*>(act + static_cast<int64_t>(q) * d)[v], xv);
@@ -348,7 +350,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
       }
     }
 #pragma unroll
-    for (int q = 0; q < kDecMaxT; ++q) {
+    for (int q = 0; q < NT; ++q) {
       if ((tmask >> q) & 1u) {
         const float g = warp_sum(ag[q]), uu = warp_sum(au[q]);
         if (lane == 0) {
@@ -438,8 +440,15 @@ cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, flo
                                 const float* bias, const void* w_gate_up, const void* w_down, void* y,
                                 int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,
                                 const Workspace& L, cudaStream_t st) {
-  static std::atomic<size_t> set_smem[kMaxDevices];
-  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(decode_layer_kernel), kDecSmem, set_smem);
+  // the accumulator count follows the batch: fewer live registers for small T
+  // keep more of each warp's row loads in flight
+  static std::atomic<size_t> set_smem[4][kMaxDevices];
+  void (*kern)(DecArgs) = s.T <= 1 ? decode_layer_kernel<1>
+                          : s.T <= 2 ? decode_layer_kernel<2>
+                          : s.T <= 4 ? decode_layer_kernel<4>
+                                     : decode_layer_kernel<8>;
+  const int which = s.T <= 1 ? 0 : s.T <= 2 ? 1 : s.T <= 4 ? 2 : 3;
+  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(kern), kDecSmem, set_smem[which]);
   if (e != cudaSuccess) return e;
   DecArgs a{};
   a.T = static_cast<int>(s.T);
@@ -475,7 +484,7 @@ cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, flo
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_layer_kernel, a);
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace moe
