@@ -99,8 +99,8 @@ cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t*
 // otherwise x -> y. Forward only (nothing is kept for the backward).
 bool decode_supported(const Shape& s);
 // Batches the layer forward routes to the one-kernel form by itself: up to 6
-// tokens (measured on B200, L2 flushed before each call: T=1 57 against 93 us
-// layered, T=4 125 against 159, T=6 152 against 161; at T=8 they tie, and in
+// tokens (measured on B200, L2 flushed before each call: T=1 45 against 93 us
+// layered, T=4 97 against 157, T=6 155 against 159; at T=8 they tie, and in
 // CUDA-graph replays the layered path is ahead there, 166 against 176 us).
 constexpr int64_t kDecodeAutoTokens = 6;
 cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, float eps, const void* w_router,
