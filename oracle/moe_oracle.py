@@ -88,6 +88,8 @@ __all__ = [
     "expert_choice",
     "experts_expert_choice",
     "moe_forward_expert_choice",
+    "moe_objective_expert_choice",
+    "moe_backward_expert_choice",
 ]
 
 
@@ -649,3 +651,61 @@ def moe_forward_expert_choice(x, w_router, w_gate_up, w_down, k, router_bias=Non
         "L_lb": 0.0,
         "L_z": router_z_loss(lse),
     }
+
+
+def moe_objective_expert_choice(x, w_router, w_gate_up, w_down, k, dy, beta, router_bias=None, capacity=None):
+    """<dy, y> + beta * L_z for the expert-choice layer (it has no balance loss)."""
+    out = moe_forward_expert_choice(x, w_router, w_gate_up, w_down, k, router_bias, capacity)
+    return float(np.sum(_f64(dy) * out["y"])) + beta * out["L_z"]
+
+
+def moe_backward_expert_choice(x, w_router, w_gate_up, w_down, k, dy, beta, router_bias=None, capacity=None):
+    """Gradients of moe_objective_expert_choice with respect to x and the weights.
+
+    The same chain rule as moe_backward, with the expert's chosen tokens as its
+    rows and p[t, e] as the weight of (t, e); the choice carries no gradient:
+      expert rows   o_te = W_down,e g_te,  g = silu(a) * b,  [a; b] = W_gate_up,e x_t
+      combine       dp_te = <dy_t, o_te> for t chosen by e (zero elsewhere),
+                    do_te = p_te dy_t
+      experts       as in moe_backward
+      softmax       dh_t = p_t * (dp_t - <dp_t, p_t>) + beta * (2 lse_t / T) * p_t
+      router        dW_r = sum_t dh_t x_t^T,   dx_t += W_r^T dh_t
+    Returns dict dx, dw_router, dw_gate_up, dw_down, dp [T,E], and "fwd".
+    """
+    x = _f64(x)
+    dy = _f64(dy)
+    fwd = moe_forward_expert_choice(x, w_router, w_gate_up, w_down, k, router_bias, capacity)
+    sel, p, lse = fwd["sel"], fwd["p"], fwd["lse"]
+    T, d = x.shape
+    n_experts = p.shape[1]
+    f = _f64(w_down[0]).shape[1]
+    dx = np.zeros_like(x)
+    dp = np.zeros((T, n_experts))
+    dw_gate_up = np.zeros((n_experts, 2 * f, d))
+    dw_down = np.zeros((n_experts, d, f))
+    for e in range(n_experts):
+        tok = sel[e]
+        if tok.size == 0:
+            continue
+        wgu = _f64(w_gate_up[e])
+        wd = _f64(w_down[e])
+        xr = x[tok]
+        a = xr @ wgu[:f].T
+        b = xr @ wgu[f:].T
+        with np.errstate(over="ignore"):
+            sig = 1.0 / (1.0 + np.exp(-a))
+        g = a * sig * b
+        o = g @ wd.T
+        dp[tok, e] = np.sum(dy[tok] * o, axis=1)
+        do = p[tok, e][:, None] * dy[tok]
+        dg = do @ wd
+        da = dg * b * (sig * (1.0 + a * (1.0 - sig)))
+        db = dg * (a * sig)
+        dw_down[e] = do.T @ g
+        dw_gate_up[e, :f] = da.T @ xr
+        dw_gate_up[e, f:] = db.T @ xr
+        dx[tok] += da @ wgu[:f] + db @ wgu[f:]
+    dh = p * (dp - np.sum(dp * p, axis=1, keepdims=True))
+    dh += beta * (2.0 * lse / T)[:, None] * p
+    dx += dh @ _f64(w_router)
+    return {"dx": dx, "dw_router": dh.T @ x, "dw_gate_up": dw_gate_up, "dw_down": dw_down, "dp": dp, "fwd": fwd}

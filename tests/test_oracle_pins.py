@@ -528,3 +528,43 @@ def test_expert_choice_dropped_tokens_get_zero_and_z_loss_is_unchanged():
     assert np.all(out["y"][out["fanout"] == 0] == 0.0)
     assert out["L_z"] == O.moe_forward(**L)["L_z"]
     assert out["L_lb"] == 0.0
+
+
+@pytest.mark.parametrize("name", ["x", "w_router", "w_gate_up", "w_down"])
+def test_expert_choice_gradients_by_finite_differences(name):
+    """Central differences of <dy, y> + beta L_z under expert choice, with the
+    choice held fixed inside the step (checked)."""
+    L = _small_layer(31, T=12, d=16, E=6, k=2, f=6, std=0.4)
+    dy = _rng(32).standard_normal((12, 16))
+    beta, eps = 0.3, 1e-6
+    g = O.moe_backward_expert_choice(dy=dy, beta=beta, **L)
+    key = {"x": "dx", "w_router": "dw_router", "w_gate_up": "dw_gate_up", "w_down": "dw_down"}[name]
+    r = _rng(33)
+    for _ in range(3):
+        v = r.standard_normal(L[name].shape)
+        Lp = dict(L)
+        Lp[name] = L[name] + eps * v
+        Lm = dict(L)
+        Lm[name] = L[name] - eps * v
+        assert np.array_equal(O.moe_forward_expert_choice(**Lp)["sel"], O.moe_forward_expert_choice(**Lm)["sel"])
+        fd = (O.moe_objective_expert_choice(dy=dy, beta=beta, **Lp)
+              - O.moe_objective_expert_choice(dy=dy, beta=beta, **Lm)) / (2 * eps)
+        an = float(np.sum(g[key] * v))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_expert_choice_backward_at_full_capacity_is_the_dense_layers():
+    """With C = T every token meets every expert with weight p[t, e], which is
+    token choice with k = E (all experts chosen, weights p): with no loss terms
+    the two objectives are the same function, so every gradient agrees, and
+    dp is <dy_t, Expert_e(x_t)> for every pair."""
+    L = _small_layer(34, T=7, d=12, E=4, k=4, f=5, std=0.4)
+    dy = _rng(35).standard_normal((7, 12))
+    ec = O.moe_backward_expert_choice(dy=dy, beta=0.0, **L)
+    assert ec["fwd"]["capacity"] == 7
+    tc = O.moe_backward(dy=dy, alpha=0.0, beta=0.0, **L)
+    for name in ("dx", "dw_router", "dw_gate_up", "dw_down"):
+        assert np.abs(ec[name] - tc[name]).max() < 1e-12, name
+    for e in range(4):
+        o = O.swiglu_expert(L["x"], L["w_gate_up"][e], L["w_down"][e])
+        assert np.abs(ec["dp"][:, e] - np.sum(dy * o, axis=1)).max() < 1e-12
