@@ -120,3 +120,32 @@ def test_binding_rejects_wrong_tensors_before_calling():
         M.moe_combine(cfg, x, x, x, x)
     with pytest.raises(ValueError):
         B._ptr(torch.zeros(4, 128, dtype=torch.bfloat16), torch.bfloat16, (4, 128), "x")  # host tensor
+
+
+def test_binding_checks_the_new_entry_points_before_calling():
+    """Wrong dtypes, shapes and host tensors are refused in Python, before the
+    library is called (no GPU needed, so each case fails on the first argument
+    the binding examines)."""
+    cfg = M.config(4, 128, 8, 2, 128)
+    C = M.moe_expert_choice_capacity(cfg)  # ceil(4 * 2 / 8) = 1
+    assert C == 1
+    bf = torch.bfloat16
+    x = torch.zeros(4, 128, dtype=bf)
+    wr = torch.zeros(8, 128, dtype=bf)
+    wgu = torch.zeros(8, 256, 128, dtype=bf)
+    wd = torch.zeros(8, 128, 128, dtype=bf)
+    ws = torch.zeros(1024, dtype=torch.uint8)
+    sel = torch.zeros(8, C, dtype=torch.int32)
+    gates = torch.zeros(8, C)
+    with pytest.raises(TypeError, match="x must be torch.bfloat16"):
+        M.moe_forward_decode(cfg, x.float(), wr, None, wgu, wd, x, None, None, None, ws)
+    with pytest.raises(ValueError, match="x must have shape"):
+        M.moe_forward_decode(cfg, x[:3], wr, None, wgu, wd, x, None, None, None, ws)
+    with pytest.raises(ValueError, match="x must be a CUDA tensor"):
+        M.moe_forward_decode(cfg, x, wr, None, wgu, wd, x, None, None, None, ws)
+    with pytest.raises(TypeError, match="x must be torch.bfloat16"):
+        M.moe_route_expert_choice(cfg, x.float(), wr, None, sel, gates, None, None, None, ws)
+    with pytest.raises(ValueError, match="x must be a CUDA tensor"):
+        M.moe_route_expert_choice(cfg, x, wr, None, sel, gates, None, None, None, ws)
+    with pytest.raises(ValueError, match="x must have shape"):
+        M.moe_forward_expert_choice(cfg, torch.zeros(4, 256, dtype=bf), wr, None, wgu, wd, x, None, sel, gates, ws)
