@@ -44,15 +44,19 @@ the design notes):
     that took it in ascending expert order and gets zero when none did; the
     z-loss is unchanged and there is no load-balancing loss (every expert
     holds exactly C tokens).
-  * Storage precision (optional `store` argument of the expert functions,
-    moe_forward and moe_backward): the pages fix no precision for the expert
-    activations. By default nothing is rounded. Given a rounding function,
-    every activation a bf16 implementation keeps between two contractions is
-    passed through it (the SwiGLU output h, the expert output o, and in the
-    backward the saved pre-activations a and b, do = w dy and [da; db]); all
-    arithmetic stays fp64. This states what an implementation with bf16
-    storage computes, so a gradient that sums many such rounded terms can be
-    compared at the bar it should meet.
+  * Operand precision (optional `store` argument of the expert functions,
+    moe_forward and moe_backward). The agreement bar is stated for "bf16
+    inputs with fp32 accumulation": every contraction of the layer takes bf16
+    operands. By default nothing is rounded. Given a rounding function, the
+    operands of the contractions that are not layer inputs already are passed
+    through it: the SwiGLU output h (the down projection's input and dW_down's
+    right factor), do = w dy (the input of dg = do W_down and dW_down's left
+    factor) and [da; db] (the input of the gate/up data gradient and dW_gate_up's
+    left factor). Values no contraction reads (the expert output o, the
+    pre-activations a and b that the SwiGLU derivative uses) are never
+    rounded, and all arithmetic stays fp64. A gradient that sums many
+    products of rounded operands (dW_router sums T terms <dy_t, o_tj> x_t with
+    o computed from a bf16 h) can then be compared at the bar it should meet.
 
 Parity pins for every function live in tests/test_oracle_pins.py.
 """
@@ -263,10 +267,11 @@ def swiglu_expert(x_rows, w_gate_up_e, w_down_e, store=None):
     [OLMoE-Guide] "Top-8 Softmax Routing Formulation": Expert_i(x) =
     (Swish(x W_gate) * (x W_up)) W_down. [MoE-scratch] §2 `Experts` stores the
     gate rows first, then the up rows, in one (2f, d) matrix, and the down
-    projection as (d, f). `store` (see the module notes) rounds h and o.
+    projection as (d, f). `store` (see the module notes) rounds h, the down
+    projection's operand; the output o is not rounded.
     """
     S = _store(store)
-    return S(expert_down(S(swiglu_hidden(x_rows, w_gate_up_e)), w_down_e))
+    return expert_down(S(swiglu_hidden(x_rows, w_gate_up_e)), w_down_e)
 
 
 def experts_grouped(x, idx, w, w_gate_up, w_down, store=None):
@@ -371,7 +376,7 @@ def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias
       router        dW_r = sum_t dh_t x_t^T,   dx_t += W_r^T dh_t
     `experts` optionally restricts which experts' weight gradients are formed
     (the rest are left zero); dx and dW_r always use every expert. `store`
-    (see the module notes) rounds h, o, the saved a and b, do and [da; db].
+    (see the module notes) rounds the contraction operands h, do and [da; db].
     With `renorm` the weights are w_tj = p_tj / s_t (s_t the sum of the chosen
     p), so the chosen probabilities receive dp_ti = (dw_tj - sum_j' dw_tj' w_tj') / s_t
     for i = S_tj instead of dw_tj.
@@ -406,14 +411,10 @@ def moe_backward(x, w_router, w_gate_up, w_down, k, dy, alpha, beta, router_bias
         with np.errstate(over="ignore"):
             sig = 1.0 / (1.0 + np.exp(-a))
         g = S(a * sig * b)
-        o = S(g @ wd.T)
+        o = g @ wd.T
         dw.reshape(-1)[sel] = np.sum(dy[tok] * o, axis=1)
         do = S(w.reshape(-1)[sel][:, None] * dy[tok])
         dg = do @ wd
-        if store is not None:  # the derivative reads the stored pre-activations
-            a, b = S(a), S(b)
-            with np.errstate(over="ignore"):
-                sig = 1.0 / (1.0 + np.exp(-a))
         da = S(dg * b * (sig * (1.0 + a * (1.0 - sig))))
         db = S(dg * (a * sig))
         if e in want:

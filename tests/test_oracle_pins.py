@@ -382,25 +382,56 @@ def test_store_identity_changes_nothing_and_zero_store_removes_the_experts():
 
 
 def test_store_rounding_on_a_two_expert_scalar_layer():
-    """d = f = 1, two experts, k = 1, rounding to multiples of 1/8. By hand:
-    h = [0.3, -0.2] so expert 0 wins with p0 = 1 / (1 + e^-0.5); its hidden
-    silu(0.7) * 1.3 = 0.608 is stored as 0.625, its output 0.8 * 0.625 = 0.5 is
-    exact; y = p0 * 0.5. With dy = 1 and no loss terms, dw = <dy, o> = 0.5, so
-    dh = [0.5 p0 p1, -0.5 p0 p1] and dW_r = dh x with x = 1; do = p0 is stored
-    as 0.625, so dW_down = 0.625 * 0.625."""
+    """d = f = 1, two experts, k = 1, rounding to multiples of 1/8; only the
+    contraction operands h, do and [da; db] are rounded. By hand: logits
+    h = [0.3, -0.2], so expert 0 wins with p0 = 1 / (1 + e^-0.5) = 0.6225; the
+    pre-activations a = 0.7, b = 1.3 stay as they are; the hidden
+    silu(0.7) * 1.3 = 0.4677 * 1.3 = 0.6081 is rounded to 0.625 before the down
+    projection; the output o = 0.9 * 0.625 = 0.5625 is NOT rounded (it would
+    become 0.5), so y = 0.5625 p0. With dy = 1 and no loss terms dw = <dy, o> =
+    0.5625, dh = [0.5625 p0 p1, -0.5625 p0 p1] and dW_r = dh x with x = 1. do =
+    p0 is rounded to 0.625, so dW_down = 0.625 * 0.625 and dg = 0.625 * 0.9 =
+    0.5625; da = dg b silu'(a) = 0.6021 rounds to 0.625 and db = dg silu(a) =
+    0.2631 rounds to 0.25, which are dW_gate_up (x = 1)."""
     R = lambda v: np.round(np.asarray(v) * 8.0) / 8.0
     x = np.array([[1.0]])
     w_router = np.array([[0.3], [-0.2]])
     w_gate_up = np.array([[[0.7], [1.3]], [[0.5], [0.5]]])
-    w_down = np.array([[[0.8]], [[0.5]]])
+    w_down = np.array([[[0.9]], [[0.5]]])
     g = O.moe_backward(x, w_router, w_gate_up, w_down, 1, np.array([[1.0]]), 0.0, 0.0, store=R)
     p0 = 1.0 / (1.0 + math.exp(-0.5))
     p1 = 1.0 - p0
     assert g["fwd"]["idx"][0, 0] == 0
-    assert abs(g["fwd"]["y"][0, 0] - p0 * 0.5) < 1e-15
-    assert abs(g["dw"][0, 0] - 0.5) < 1e-15
-    assert np.allclose(g["dw_router"][:, 0], [0.5 * p0 * p1, -0.5 * p0 * p1], atol=1e-15, rtol=0)
+    assert abs(g["fwd"]["y"][0, 0] - p0 * 0.5625) < 1e-15
+    assert abs(g["dw"][0, 0] - 0.5625) < 1e-15
+    assert np.allclose(g["dw_router"][:, 0], [0.5625 * p0 * p1, -0.5625 * p0 * p1], atol=1e-15, rtol=0)
     assert abs(g["dw_down"][0, 0, 0] - 0.625 * 0.625) < 1e-15
+    assert abs(g["dw_gate_up"][0, 0, 0] - 0.625) < 1e-15 and abs(g["dw_gate_up"][0, 1, 0] - 0.25) < 1e-15
+    assert np.all(g["dw_gate_up"][1] == 0) and np.all(g["dw_down"][1] == 0)
+    # the unrounded values the rounding acted on, by hand
+    s = 1.0 / (1.0 + math.exp(-0.7))
+    assert abs(0.7 * s * 1.3 - 0.6081) < 1e-4
+    assert abs(0.5625 * 1.3 * s * (1.0 + 0.7 * (1.0 - s)) - 0.6021) < 1e-4
+    assert abs(0.5625 * 0.7 * s - 0.2631) < 1e-4
+
+
+def test_operand_rounding_alone_moves_olmoe_router_gradient_past_the_max_abs_bar():
+    """Why weight gradients are compared with the operand-rounded oracle: on a
+    1024-token layer of OLMoE's shapes, rounding only the contraction operands
+    to bf16 (what any bf16-input implementation must do) moves dW_router by
+    more than 2e-2 max-abs from the unrounded fp64 gradient, while its relative
+    L2 change stays near 2e-3 and dx stays far inside both bars."""
+    sh = S.LayerShape(T=1024)
+    inp = S.layer_inputs(sh, seed=4, with_grad=True)
+    f = lambda t: t.to(torch.float64).numpy()
+    args = (f(inp.x), f(inp.w_router), f(inp.w_gate_up), f(inp.w_down), sh.top_k, f(inp.dy), 0.01, 0.001)
+    bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).float().bfloat16().double().numpy()
+    plain = O.moe_backward(*args, experts=[])
+    rounded = O.moe_backward(*args, experts=[], store=bf16)
+    d = rounded["dw_router"] - plain["dw_router"]
+    assert np.abs(d).max() > 2e-2
+    assert np.linalg.norm(d) / np.linalg.norm(plain["dw_router"]) < 5e-3
+    assert np.abs(rounded["dx"] - plain["dx"]).max() < 5e-3
 
 
 # ------------------------------------------------------------------ stack
