@@ -50,7 +50,7 @@ extern "C" {
 struct CUstream_st;
 typedef struct CUstream_st* cudaStream_t;
 
-#define MOE_ABI_VERSION 5
+#define MOE_ABI_VERSION 6
 #define MOE_ROW_ALIGN 128
 
 typedef enum moe_status {
@@ -136,9 +136,13 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
                      int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,
                      size_t ws_bytes, cudaStream_t stream);
 
-/* moe_route without a workspace: the same router, results and output buffers,
+/* moe_route without a workspace: the same routing, outputs and output buffers,
  * but its scratch is a fixed MOE_ROUTE_STATIC_SCRATCH_BYTES array inside the
- * library, so the call allocates nothing and needs no `ws`. The pages have no
+ * library, so the call allocates nothing and needs no `ws`. It always runs the
+ * CUDA-core router (logits summed in fp64): the same experts as moe_route under
+ * the exact-logit tie rule, weights and losses equal within the agreement
+ * tolerances (not bit for bit), and a slower call than moe_route's tensor-core
+ * router for bf16 layers. The pages have no
  * counterpart: this is for callers that cannot provide device memory of their
  * own, such as code whose device memory is planned and owned by a host
  * framework or serving runtime, or a loop that must not call cudaMalloc because
@@ -149,7 +153,8 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
  *     launching anything.
  *   - The first call on a device looks up the array's device address on that
  *     device (it must be the current device); make that first call before any
- *     stream capture.
+ *     stream capture. The address is kept with the context it belongs to and
+ *     looked up again after a device reset or in another context.
  *   - Every device that loads the library keeps the array until the process
  *     exits. All calls share it and find the last call's contents in it; the
  *     part that must start at zero is cleared on `stream` before each launch.
@@ -183,8 +188,10 @@ moe_status moe_dispatch(const moe_config* cfg, const int32_t* topk_idx, const vo
  *   offsets     [device] [E+1]    from moe_dispatch (valid rows per expert)
  *   w_gate_up   [device] [E, 2f, d]  gate rows then up rows per expert
  *   h           [device] [P, f] out, pad rows zero
- *   preact      [device] [P, 2f] out or NULL: the gate and up pre-activations
- *                (kept by moe_forward for the backward). */
+ *   preact      [device] [P, 2f] fp32 out or NULL: the gate and up
+ *                pre-activations, unrounded (moe_forward keeps them for the
+ *                backward's SwiGLU derivative, which is no contraction, so they
+ *                are not rounded to the layer dtype). */
 moe_status moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const int32_t* group_start,
                               const int32_t* offsets, const void* w_gate_up, void* h, void* preact,
                               void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -213,7 +220,10 @@ moe_status moe_combine(const moe_config* cfg, const void* o_perm, const int32_t*
  *   losses   [device] [2] fp32 out {L_lb, L_z}
  *   topk_idx [device] [T, k] int32 out or NULL;  topk_w [device] [T, k] fp32 out or NULL
  *   save_for_backward: 1 keeps what moe_backward needs in ws (which must then be
- *   moe_workspace_bytes(cfg, 1) bytes and stay untouched until moe_backward). */
+ *   moe_workspace_bytes(cfg, 1) bytes and stay untouched until moe_backward);
+ *   the expert outputs and the gate/up pre-activations are then kept in fp32
+ *   (y is summed from the fp32 expert outputs), since no contraction reads
+ *   them: only h, do = w dy and [da; db] enter the GEMMs in the layer dtype. */
 moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router, const float* router_bias,
                        const void* w_gate_up, const void* w_down, void* y, float* losses, int32_t* topk_idx,
                        float* topk_w, int32_t save_for_backward, void* ws, size_t ws_bytes,
@@ -245,6 +255,18 @@ moe_status moe_forward_decode(const moe_config* cfg, const void* x, const void* 
 moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const void* w_router,
                             const float* router_bias, const void* w_gate_up, const void* w_down, void* y_host,
                             float* losses_host, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* moe_forward_host without the final synchronisation: the copy of x_host in,
+ * the layer and the copies of y and the losses out are queued on `stream` and
+ * the call returns; y_host and losses_host hold the results once that work has
+ * completed (synchronise the stream, or wait on an event recorded after the
+ * call). x_host must stay unchanged and y_host unread until then. With pinned
+ * host buffers the copies are asynchronous DMA, so a caller that keeps two
+ * calls in flight on two streams, each with its own workspace and output
+ * buffer, overlaps one call's host transfers with the other's kernels. */
+moe_status moe_forward_host_async(const moe_config* cfg, const void* x_host, const void* w_router,
+                                  const float* router_bias, const void* w_gate_up, const void* w_down, void* y_host,
+                                  float* losses_host, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Backward of <dy, y> + alpha_lb * L_lb + beta_z * L_z for the forward saved in
  * ws (same cfg, inputs and weights). No gradient flows through the expert choice

@@ -28,6 +28,7 @@ from .binding import (  # noqa: F401
     moe_forward_decode,
     moe_forward_expert_choice,
     moe_forward_host,
+    moe_forward_host_async,
     moe_get_device_status,
     moe_padded_rows,
     moe_rmsnorm,

@@ -17,7 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
-ABI_VERSION = 5  # MOE_ABI_VERSION of include/moe.h this binding marshals for
+ABI_VERSION = 6  # MOE_ABI_VERSION of include/moe.h this binding marshals for
 MOE_BF16 = 0
 MOE_FP32 = 1
 MOE_ROUTER_SOFTMAX_TOPK = 0
@@ -39,7 +39,7 @@ EXPORTS = (
     "moe_status_string", "moe_abi_version", "moe_check_config", "moe_padded_rows",
     "moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_route_static", "moe_dispatch",
     "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_forward",
-    "moe_forward_decode", "moe_forward_host", "moe_backward", "moe_rmsnorm", "moe_combine_residual",
+    "moe_forward_decode", "moe_forward_host", "moe_forward_host_async", "moe_backward", "moe_rmsnorm", "moe_combine_residual",
     "moe_stack_forward", "moe_stack_forward_trace", "moe_expert_choice_capacity", "moe_route_expert_choice",
     "moe_forward_expert_choice", "moe_set_stage_events", "moe_get_device_status",
 )
@@ -89,6 +89,7 @@ _SIGS = {
                                    ctypes.c_size_t, _P]),
     "moe_forward_decode": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_forward_host": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_forward_host_async": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_backward": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_rmsnorm": (ctypes.c_int, [_CFG, _P, _P, ctypes.c_float, _P, _P]),
     "moe_combine_residual": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
@@ -267,7 +268,7 @@ def moe_expert_gate_up(cfg, x_perm, group_start, offsets, w_gate_up, h, preact, 
     st = lib().moe_expert_gate_up(
         _cfgp(cfg), _ptr(x_perm, dt, (P, d), "x_perm"), _ptr(group_start, torch.int32, (E + 1,), "group_start"),
         _ptr(offsets, torch.int32, (E + 1,), "offsets"), _ptr(w_gate_up, dt, (E, 2 * f, d), "w_gate_up"),
-        _ptr(h, dt, (P, f), "h"), _ptr(preact, dt, (P, 2 * f), "preact", allow_none=True),
+        _ptr(h, dt, (P, f), "h"), _ptr(preact, torch.float32, (P, 2 * f), "preact", allow_none=True),
         _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
     _check(st, "moe_expert_gate_up")
 
@@ -413,6 +414,22 @@ def moe_forward_host(cfg, x_host, w_router, router_bias, w_gate_up, w_down, y_ho
         _ptr(losses_host, torch.float32, (2,), "losses_host", allow_none=True, device=False),
         _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
     _check(st, "moe_forward_host")
+
+
+def moe_forward_host_async(cfg, x_host, w_router, router_bias, w_gate_up, w_down, y_host, losses_host, ws,
+                           stream=None):
+    """moe_forward_host without the final synchronisation: the results are in
+    y_host / losses_host once `stream`'s queued work has completed."""
+    dt = torch_dtype(cfg)
+    T, d, E, f = cfg.T, cfg.d_model, cfg.n_experts, cfg.d_ff
+    st = lib().moe_forward_host_async(
+        _cfgp(cfg), _ptr(x_host, dt, (T, d), "x_host", device=False), _ptr(w_router, dt, (E, d), "w_router"),
+        _ptr(router_bias, torch.float32, (E,), "router_bias", allow_none=True),
+        _ptr(w_gate_up, dt, (E, 2 * f, d), "w_gate_up"), _ptr(w_down, dt, (E, d, f), "w_down"),
+        _ptr(y_host, dt, (T, d), "y_host", device=False),
+        _ptr(losses_host, torch.float32, (2,), "losses_host", allow_none=True, device=False),
+        _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))
+    _check(st, "moe_forward_host_async")
 
 
 def moe_backward(cfg, dy, x, w_router, w_gate_up, w_down, dx, dw_router, dw_gate_up, dw_down, ws,

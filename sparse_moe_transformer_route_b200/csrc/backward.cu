@@ -4,8 +4,9 @@
 // 4.1.7 for alpha and beta). No gradient flows through the choice of experts or
 // through the counts f_i (a bincount).
 //
-//   combine backward  dw_tj = <dy_t, o_tj>;  dO[r] = w_tj dy_t for the row r of
-//                     pair (t, j), zero on padding rows.       (row-parallel gather)
+//   combine backward  dw_tj = <dy_t, o_tj> with the fp32 expert outputs the
+//                     forward kept; dO[r] = w_tj dy_t for the row r of pair
+//                     (t, j), zero on padding rows.           (row-parallel gather)
 //   router backward   dp_ti = sum_j [S_tj = i] dw_tj + alpha E f_i / T
 //                     dh_t  = p_t * (dp_t - <dp_t, p_t>) + beta (2 lse_t / T) p_t
 //   dx                dx_t = sum_j dX_perm[row(t, j)] + sum_e dh_t,e W_r[e]
@@ -52,12 +53,14 @@ __device__ __forceinline__ void store8(T_* p, const float (&v)[8]) {
   }
 }
 
-// One warp per padded row.
+// One warp per padded row; o_perm holds the fp32 expert outputs.
 template <typename T_>
 __global__ void __launch_bounds__(256)
-    combine_bwd_kernel(const T_* __restrict__ dy, const T_* __restrict__ o_perm, const int32_t* __restrict__ row_pair,
+    combine_bwd_kernel(const T_* __restrict__ dy, const float* __restrict__ o_perm, const int32_t* __restrict__ row_pair,
                        const int32_t* __restrict__ gs, int E, const float* __restrict__ wts, int d, int k,
                        float* __restrict__ dw, T_* __restrict__ dout) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + warp;
   if (r >= gs[E]) return;
@@ -75,7 +78,7 @@ __global__ void __launch_bounds__(256)
   for (int v = lane; v < nv; v += 32) {
     float g[8], o[8], out[8];
     load8<T_>(dy + t * d + v * 8, g);
-    load8<T_>(o_perm + r * d + v * 8, o);
+    load8<float>(o_perm + r * d + v * 8, o);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       dot = fmaf(g[i], o[i], dot);
@@ -93,6 +96,8 @@ __global__ void __launch_bounds__(256)
     router_bwd_kernel(const float* __restrict__ dw, const int32_t* __restrict__ idx, const float* __restrict__ probs,
                       const float* __restrict__ lse, const int32_t* __restrict__ counts, int64_t T, int E, int k,
                       float alpha, float beta, int renorm, float* __restrict__ dh) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp;
   if (t >= T) return;
@@ -180,6 +185,8 @@ template <typename T_>
 __global__ void __launch_bounds__(256)
     dx_kernel(const T_* __restrict__ dx_perm, const int32_t* __restrict__ inv_perm, const float* __restrict__ dh,
               const T_* __restrict__ w_router, int64_t T, int d, int E, int k, T_* __restrict__ dx) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   __shared__ float sdh[kDxRows][kDxE];
   __shared__ __align__(16) float sw[kDxE][kDxCols];
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kDxRows;
@@ -246,6 +253,8 @@ template <typename T_>
 __global__ void __launch_bounds__(256)
     router_wgrad_partial(const float* __restrict__ dh, const T_* __restrict__ x, int64_t T, int d, int E,
                          float* __restrict__ part) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   __shared__ __align__(16) float sdh[kWrTok][64];
   __shared__ __align__(16) float sx[kWrTok][128];
   const int c0 = blockIdx.x * 128;
@@ -301,6 +310,8 @@ __global__ void __launch_bounds__(256)
 
 template <typename T_>
 __global__ void router_wgrad_reduce(const float* __restrict__ part, int64_t n, T_* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
   float s = 0.f;
@@ -318,13 +329,13 @@ cudaError_t launch_combine_backward(const Shape& s, const void* dy, const void* 
                                     const int32_t* row_pair, const float* wts, float* dw, void* dout,
                                     cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((s.P + 7) / 8);
+  const float* o32 = static_cast<const float*>(o_perm);
   if (s.fp32)
-    combine_bwd_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(dy), static_cast<const float*>(o_perm),
-                                                    row_pair, gs, s.E, wts, s.d, s.k, dw, static_cast<float*>(dout));
+    launch_dependent(combine_bwd_kernel<float>, dim3(grid), dim3(256), 0, st, nullptr, 0, static_cast<const float*>(dy), o32, row_pair, gs, s.E, wts, s.d,
+                                                    s.k, dw, static_cast<float*>(dout));
   else
-    combine_bwd_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(o_perm), row_pair, gs, s.E, wts, s.d,
-        s.k, dw, static_cast<__nv_bfloat16*>(dout));
+    launch_dependent(combine_bwd_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, nullptr, 0, static_cast<const __nv_bfloat16*>(dy), o32, row_pair, gs,
+                                                            s.E, wts, s.d, s.k, dw, static_cast<__nv_bfloat16*>(dout));
   return cudaGetLastError();
 }
 
@@ -332,7 +343,7 @@ cudaError_t launch_router_backward(const Shape& s, const float* dw, const int32_
                                    const float* lse, const int32_t* counts, float alpha, float beta, float* dh,
                                    cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((s.T + 7) / 8);
-  router_bwd_kernel<<<grid, 256, 0, st>>>(dw, idx, probs, lse, counts, s.T, s.E, s.k, alpha, beta,
+  launch_dependent(router_bwd_kernel, dim3(grid), dim3(256), 0, st, nullptr, 0, dw, idx, probs, lse, counts, s.T, s.E, s.k, alpha, beta,
                                           s.renorm ? 1 : 0, dh);
   return cudaGetLastError();
 }
@@ -342,11 +353,11 @@ cudaError_t launch_dx_combine(const Shape& s, const void* dx_perm, const int32_t
   const dim3 grid(static_cast<unsigned>((s.T + kDxRows - 1) / kDxRows), static_cast<unsigned>((s.d + kDxCols - 1) / kDxCols));
   const int threads = 256;
   if (s.fp32)
-    dx_kernel<float><<<grid, threads, 0, st>>>(static_cast<const float*>(dx_perm), inv_perm, dh,
+    launch_dependent(dx_kernel<float>, dim3(grid), dim3(threads), 0, st, nullptr, 0, static_cast<const float*>(dx_perm), inv_perm, dh,
                                                static_cast<const float*>(w_router), s.T, s.d, s.E, s.k,
                                                static_cast<float*>(dx));
   else
-    dx_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(static_cast<const __nv_bfloat16*>(dx_perm), inv_perm, dh,
+    launch_dependent(dx_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), 0, st, nullptr, 0, static_cast<const __nv_bfloat16*>(dx_perm), inv_perm, dh,
                                                        static_cast<const __nv_bfloat16*>(w_router), s.T, s.d, s.E, s.k,
                                                        static_cast<__nv_bfloat16*>(dx));
   return cudaGetLastError();
@@ -356,18 +367,18 @@ cudaError_t launch_router_weight_grad(const Shape& s, const float* dh, const voi
                                       cudaStream_t st) {
   dim3 grid((s.d + 127) / 128, kWrSplit, (s.E + 63) / 64);
   if (s.fp32)
-    router_wgrad_partial<float><<<grid, 256, 0, st>>>(dh, static_cast<const float*>(x), s.T, s.d, s.E, part);
+    launch_dependent(router_wgrad_partial<float>, dim3(grid), dim3(256), 0, st, nullptr, 0, dh, static_cast<const float*>(x), s.T, s.d, s.E, part);
   else
-    router_wgrad_partial<__nv_bfloat16><<<grid, 256, 0, st>>>(dh, static_cast<const __nv_bfloat16*>(x), s.T, s.d,
+    launch_dependent(router_wgrad_partial<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, nullptr, 0, dh, static_cast<const __nv_bfloat16*>(x), s.T, s.d,
                                                               s.E, part);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t n = static_cast<int64_t>(s.E) * s.d;
   const unsigned g2 = static_cast<unsigned>((n + 255) / 256);
   if (s.fp32 || s.grad32)
-    router_wgrad_reduce<float><<<g2, 256, 0, st>>>(part, n, static_cast<float*>(dw_router));
+    launch_dependent(router_wgrad_reduce<float>, dim3(g2), dim3(256), 0, st, nullptr, 0, part, n, static_cast<float*>(dw_router));
   else
-    router_wgrad_reduce<__nv_bfloat16><<<g2, 256, 0, st>>>(part, n, static_cast<__nv_bfloat16*>(dw_router));
+    launch_dependent(router_wgrad_reduce<__nv_bfloat16>, dim3(g2), dim3(256), 0, st, nullptr, 0, part, n, static_cast<__nv_bfloat16*>(dw_router));
   return cudaGetLastError();
 }
 

@@ -76,10 +76,14 @@ struct Raw8 {
   }
 };
 
-template <typename T_, bool RESID>
+// OT: element type of the expert rows (the layer dtype, or fp32 when the
+// forward keeps them for the backward); T_: the output's.
+template <typename OT, typename T_, bool RESID>
 __global__ void __launch_bounds__(256)
-    combine_kernel(const T_* __restrict__ o_perm, const int32_t* __restrict__ inv_perm, const float* __restrict__ wts,
+    combine_kernel(const OT* __restrict__ o_perm, const int32_t* __restrict__ inv_perm, const float* __restrict__ wts,
                    int64_t T, int d, int k, T_* __restrict__ y, float* __restrict__ resid) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   __shared__ int32_t rows[kMaxTopK];
   __shared__ float ws_[kMaxTopK];
   const int64_t t = blockIdx.x;
@@ -97,7 +101,7 @@ __global__ void __launch_bounds__(256)
     // re-reads row 0, which always exists, and is then skipped), then the sum
     // runs in slot order.
     for (int j0 = 0; j0 < k; j0 += 8) {
-      Raw8<T_> q[8];
+      Raw8<OT> q[8];
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
         const int j = j0 + jj;
@@ -141,6 +145,8 @@ template <typename T_>
 __global__ void __launch_bounds__(256)
     combine_ec_kernel(const T_* __restrict__ o_perm, const int32_t* __restrict__ slot_row,
                       const float* __restrict__ probs, int64_t T, int d, int E, T_* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   __shared__ int32_t rows[kMaxExperts];
   __shared__ float ws_[kMaxExperts];
   __shared__ int s_n;
@@ -195,29 +201,36 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The normalised value is formed in fp64 (sum of squares, square root and
+// division), then rounded to fp32 and on to the output type: the same value
+// and the same two roundings as an fp64 evaluation of the formula, so the
+// layer input's rounding is decided as an exact computation would decide it.
 template <typename T_>
 __global__ void __launch_bounds__(256)
-    rmsnorm_kernel(const float* __restrict__ resid, const float* __restrict__ weight, float eps, int d,
+    rmsnorm_kernel(const float* __restrict__ resid, const float* __restrict__ weight, double eps, int d,
                    T_* __restrict__ out) {
-  __shared__ float red[8];
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
+  __shared__ double red[8];
   const int64_t t = blockIdx.x;
   const float* r = resid + t * d;
-  float ss = 0.f;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) ss = fmaf(r[i], r[i], ss);
+  double ss = 0.0;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) ss = fma(static_cast<double>(r[i]), static_cast<double>(r[i]), ss);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
   if (threadIdx.x == 0) {
-    float s = 0.f;
+    double s = 0.0;
     for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) s += red[w];
     red[0] = s;
   }
   __syncthreads();
-  const float inv = rsqrtf(red[0] / static_cast<float>(d) + eps);
+  const double den = sqrt(red[0] / static_cast<double>(d) + eps);
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    const float v = r[i] * inv * (weight != nullptr ? weight[i] : 1.0f);
-    out[t * d + i] = from_f32<T_>(v);
+    double v = static_cast<double>(r[i]) / den;
+    if (weight != nullptr) v *= static_cast<double>(weight[i]);
+    out[t * d + i] = from_f32<T_>(static_cast<float>(v));
   }
 }
 
@@ -233,36 +246,36 @@ cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t*
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const Shape& s, const void* o_perm, const int32_t* inv_perm, const float* wts, void* y,
-                           float* resid, cudaStream_t st) {
+namespace {
+template <typename OT, typename T_>
+cudaError_t combine_typed(const Shape& s, const void* o_perm, const int32_t* inv_perm, const float* wts, void* y,
+                          float* resid, cudaStream_t st) {
   const int threads = s.d / 8 < 256 ? s.d / 8 : 256;
   const unsigned grid = static_cast<unsigned>(s.T);
-  if (s.fp32) {
-    if (resid != nullptr)
-      combine_kernel<float, true><<<grid, threads, 0, st>>>(static_cast<const float*>(o_perm), inv_perm, wts, s.T,
-                                                            s.d, s.k, nullptr, resid);
-    else
-      combine_kernel<float, false><<<grid, threads, 0, st>>>(static_cast<const float*>(o_perm), inv_perm, wts, s.T,
-                                                             s.d, s.k, static_cast<float*>(y), nullptr);
-  } else {
-    if (resid != nullptr)
-      combine_kernel<__nv_bfloat16, true><<<grid, threads, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(o_perm), inv_perm, wts, s.T, s.d, s.k, nullptr, resid);
-    else
-      combine_kernel<__nv_bfloat16, false><<<grid, threads, 0, st>>>(static_cast<const __nv_bfloat16*>(o_perm),
-                                                                     inv_perm, wts, s.T, s.d, s.k,
-                                                                     static_cast<__nv_bfloat16*>(y), nullptr);
-  }
+  const OT* o = static_cast<const OT*>(o_perm);
+  if (resid != nullptr)
+    launch_dependent(combine_kernel<OT, T_, true>, dim3(grid), dim3(threads), 0, st, nullptr, 0, o, inv_perm, wts, s.T, s.d, s.k, nullptr, resid);
+  else
+    launch_dependent(combine_kernel<OT, T_, false>, dim3(grid), dim3(threads), 0, st, nullptr, 0, o, inv_perm, wts, s.T, s.d, s.k, static_cast<T_*>(y),
+                                                           nullptr);
   return cudaGetLastError();
 }
+}  // namespace
 
-cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, float eps, void* out,
+cudaError_t launch_combine(const Shape& s, const void* o_perm, bool o32, const int32_t* inv_perm, const float* wts,
+                           void* y, float* resid, cudaStream_t st) {
+  if (s.fp32) return combine_typed<float, float>(s, o_perm, inv_perm, wts, y, resid, st);
+  if (o32) return combine_typed<float, __nv_bfloat16>(s, o_perm, inv_perm, wts, y, resid, st);
+  return combine_typed<__nv_bfloat16, __nv_bfloat16>(s, o_perm, inv_perm, wts, y, resid, st);
+}
+
+cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, double eps, void* out,
                            cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(s.T);
   if (s.fp32)
-    rmsnorm_kernel<float><<<grid, 256, 0, st>>>(resid, weight, eps, s.d, static_cast<float*>(out));
+    launch_dependent(rmsnorm_kernel<float>, dim3(grid), dim3(256), 0, st, nullptr, 0, resid, weight, eps, s.d, static_cast<float*>(out));
   else
-    rmsnorm_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(resid, weight, eps, s.d, static_cast<__nv_bfloat16*>(out));
+    launch_dependent(rmsnorm_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, nullptr, 0, resid, weight, eps, s.d, static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError();
 }
 

@@ -10,16 +10,18 @@
 // Mechanics & Loss Formulations"). Section 6 of the lesson notes that at a
 // batch of one token the layer reads only the k chosen experts' weights, so
 // decoding is bound by streaming those weights; this kernel exists to stream
-// them with nothing else in the way (one launch, two grid barriers).
+// them with nothing else in the way (one launch, one grid barrier).
 //
 // One CTA per SM (grid = SM count, cooperative launch, 16 warps):
 //   prologue  every CTA stages the T input rows in shared memory (with the
 //             RMSNorm applied when the input is the fp32 residual).
-//   phase 0   the T*E router logits, one warp per (token, expert): products of
-//             bf16 values are exact in fp32 and are summed in fp64, so the
-//             logits are exact to ~1e-16 and the top-k matches an exact
-//             computation except for exactly equal logits (lower index wins).
-//   barrier
+//   phase 0   every CTA computes the T*E router logits itself (W_r is read
+//             from L2 by each CTA; no grid barrier): products of bf16 values
+//             are exact in fp32 and are summed in fp32; a token whose k+1
+//             largest logits hold near-equal neighbours has its logits
+//             recomputed as fp64 sums of the exact products, so the top-k
+//             matches an exact computation except for exactly equal logits
+//             (lower index wins). Every CTA takes the same decisions.
 //   phase 0b  every CTA: each expert's rank among a token's logits gives the
 //             top-k at once (no sequential selection); softmax in fp32; the
 //             tokens of each expert as a bit mask; CTA 0 writes the losses,
@@ -56,7 +58,7 @@ constexpr size_t kDecSmem = kDecActBytes + kDecMiscBytes;
 struct DecArgs {
   int T, d, E, k, f;
   int renorm;
-  float eps;
+  double eps;
   const __nv_bfloat16* x;    // [T, d] layer input, or null when `resid` is the input
   float* resid;              // [T, d] fp32 residual (in/out), or null
   const __nv_bfloat16* wr;   // [E, d]
@@ -64,7 +66,6 @@ struct DecArgs {
   const __nv_bfloat16* wgu;  // [E, 2f, d]
   const __nv_bfloat16* wd;   // [E, d, f]
   __nv_bfloat16* y;          // [T, d] out (null with `resid`)
-  double* logits;            // [T, E] workspace
   __nv_bfloat16* h;          // [T*k, f] workspace
   int32_t* idx_out;          // [T, k] or null
   float* w_out;              // [T, k] or null
@@ -84,7 +85,7 @@ struct DecSmem {
   int touched[kDecMaxE];           // experts chosen by some token, ascending
   int n_touched;
   int ok;
-  float inv_rms[kDecMaxT];
+  double rms[kDecMaxT];             // sqrt(mean square + eps) of each input row
   double hd[kDecMaxT][kDecMaxE];   // logits (+ offset)
   float p[kDecMaxT][kDecMaxE];
   float lse[kDecMaxT];
@@ -161,16 +162,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
 
   // ---- prologue: the T input rows, bf16, in shared memory
   if (a.resid != nullptr) {
-    if (warp < T) {  // RMSNorm (unit weight) of token `warp`: mean of squares in a fixed order
+    if (warp < T) {  // RMSNorm (unit weight) of token `warp` in fp64, mean of squares in a fixed order
       const float* r = a.resid + static_cast<int64_t>(warp) * d;
-      float ss = 0.f;
-      for (int i = lane; i < d; i += 32) ss = fmaf(r[i], r[i], ss);
-      ss = warp_sum(ss);
-      if (lane == 0) m.inv_rms[warp] = rsqrtf(ss / static_cast<float>(d) + a.eps);
+      double ss = 0.0;
+      for (int i = lane; i < d; i += 32) ss = fma(static_cast<double>(r[i]), static_cast<double>(r[i]), ss);
+      ss = warp_sum_d(ss);
+      if (lane == 0) m.rms[warp] = sqrt(ss / static_cast<double>(d) + a.eps);
       __syncwarp();
     }
     __syncthreads();
-    for (int i = tid; i < T * d; i += kDecThreads) act[i] = __float2bfloat16_rn(a.resid[i] * m.inv_rms[i / d]);
+    // the fp64 value rounded to fp32, then to bf16 (as the separate RMSNorm kernel does)
+    for (int i = tid; i < T * d; i += kDecThreads)
+      act[i] = __float2bfloat16_rn(static_cast<float>(static_cast<double>(a.resid[i]) / m.rms[i / d]));
   } else {
     const uint4* src = reinterpret_cast<const uint4*>(a.x);
     uint4* dst = reinterpret_cast<uint4*>(act);
@@ -180,12 +183,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
   if (tid < kDecSlots) m.sel_e[tid] = 0;  // defined even if non-finite logits leave a slot unranked
   __syncthreads();
 
-  // ---- phase 0: exact router logits, a warp per (token, expert)
-  for (int pr = gw; pr < T * E; pr += nw) {
-    const int t = pr / E, e = pr - t * E;
+  // ---- phase 0 (every CTA, no grid barrier): the T*E router logits. Warp w
+  //      takes experts w, w + 16, ...; each W_r row is read once into registers
+  //      and meets every token. bf16 x bf16 products are exact in fp32 and are
+  //      summed in fp32 here; every CTA sums in the same order, so every CTA
+  //      holds the same values and takes the same decisions.
+  for (int e = warp; e < E; e += kDecWarps) {
     const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<int64_t>(e) * d);
-    const uint4* xrow = reinterpret_cast<const uint4*>(act + static_cast<int64_t>(t) * d);
-    double acc = 0.0;
+    float acc[NT];
+#pragma unroll
+    for (int q = 0; q < NT; ++q) acc[q] = 0.f;
     for (int v0 = 0; v0 < nvd; v0 += 32 * 8) {
       uint4 wq[8];
 #pragma unroll
@@ -197,29 +204,85 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
       for (int j = 0; j < 8; ++j) {
         const int v = v0 + j * 32 + lane;
         if (v < nvd) {
-          float xv[8], wv[8];
-          bf16x8(xrow[v], xv);
+          float wv[8];
           bf16x8(wq[j], wv);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc += static_cast<double>(xv[i] * wv[i]);  // exact product
+          for (int q = 0; q < NT; ++q) {
+            if (q < T) {
+              float xv[8];
+              bf16x8(reinterpret_cast<const uint4*>(act + static_cast<int64_t>(q) * d)[v], xv);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[q] = fmaf(xv[i], wv[i], acc[q]);
+            }
+          }
         }
       }
     }
-    acc = warp_sum_d(acc);
-    if (lane == 0) a.logits[pr] = acc;
+#pragma unroll
+    for (int q = 0; q < NT; ++q) {
+      if (q < T) {
+        const float h = warp_sum(acc[q]);
+        if (lane == 0) m.hd[q][e] = static_cast<double>(h) + (a.bias != nullptr ? static_cast<double>(a.bias[e]) : 0.0);
+      }
+    }
   }
-  if (!grid_barrier(a.bar, gridDim.x, a.status, &m.ok)) return;
+  __syncthreads();
+  // The choice must be the exact one: a token whose k+1 largest fp32 logits
+  // hold two values closer than 2e-4 * max(1, |h|) (far above the error of a
+  // 2048-term fp32 sum of exact products) has all E logits recomputed exactly
+  // (fp64 sums of the exact products), lane l taking experts l and l + 32.
+  if (warp < T) {
+    const int t = warp;
+    const int e0 = lane, e1 = lane + 32;
+    const double h0 = e0 < E ? m.hd[t][e0] : -INFINITY, h1 = e1 < E ? m.hd[t][e1] : -INFINITY;
+    int r0 = 0, r1 = 0;
+    for (int e = 0; e < E; ++e) {
+      const double v = m.hd[t][e];
+      r0 += (v > h0 || (v == h0 && e < e0)) ? 1 : 0;
+      r1 += (v > h1 || (v == h1 && e < e1)) ? 1 : 0;
+    }
+    bool near = false;
+    for (int e = 0; e < E; ++e) {
+      const double v = m.hd[t][e];
+      const double g = 2e-4 * fmax(1.0, fabs(v));
+      if (e0 < E && e != e0 && r0 <= k && fabs(v - h0) < g) near = true;
+      if (e1 < E && e != e1 && r1 <= k && fabs(v - h1) < g) near = true;
+    }
+    // (a near value may rank below k + 1 itself: then it is within the gap of
+    // a ranked one, which the loop above finds from that ranked lane)
+    if (__any_sync(0xffffffffu, near)) {
+      const uint4* xrow = reinterpret_cast<const uint4*>(act + static_cast<int64_t>(t) * d);
+      double ex[2] = {0.0, 0.0};
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int e = lane + 32 * u;
+        if (e < E) {
+          const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<int64_t>(e) * d);
+          double acc = 0.0;
+          for (int v = 0; v < nvd; ++v) {
+            float xv[8], wv[8];
+            bf16x8(xrow[v], xv);
+            bf16x8(__ldg(wrow + v), wv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc += static_cast<double>(xv[i] * wv[i]);  // exact product
+          }
+          ex[u] = acc + (a.bias != nullptr ? static_cast<double>(a.bias[e]) : 0.0);
+        }
+      }
+      __syncwarp();
+      if (e0 < E) m.hd[t][e0] = ex[0];
+      if (e1 < E) m.hd[t][e1] = ex[1];
+    }
+    __syncwarp();
+  }
+  __syncthreads();
 
   // ---- phase 0b (every CTA): warp t takes token t; lane l holds experts l, l + 32
   if (warp < T) {
     const int t = warp;
     const int e0 = lane, e1 = lane + 32;
-    double h0 = -INFINITY, h1 = -INFINITY;
-    if (e0 < E) h0 = __ldcg(a.logits + t * E + e0) + (a.bias != nullptr ? static_cast<double>(a.bias[e0]) : 0.0);
-    if (e1 < E) h1 = __ldcg(a.logits + t * E + e1) + (a.bias != nullptr ? static_cast<double>(a.bias[e1]) : 0.0);
-    if (e0 < E) m.hd[t][e0] = h0;
-    if (e1 < E) m.hd[t][e1] = h1;
-    __syncwarp();
+    const double h0 = e0 < E ? m.hd[t][e0] : -INFINITY;
+    const double h1 = e1 < E ? m.hd[t][e1] : -INFINITY;
     // rank by (logit descending, index ascending): the experts ranked below k are the choice
     int r0 = 0, r1 = 0;
     for (int e = 0; e < E; ++e) {
@@ -436,7 +499,7 @@ bool decode_supported(const Shape& s) {
   return x_bytes <= kDecActBytes && h_bytes <= kDecActBytes;
 }
 
-cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, float eps, const void* w_router,
+cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, double eps, const void* w_router,
                                 const float* bias, const void* w_gate_up, const void* w_down, void* y,
                                 int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,
                                 const Workspace& L, cudaStream_t st) {
@@ -465,7 +528,6 @@ cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, flo
   a.wgu = static_cast<const __nv_bfloat16*>(w_gate_up);
   a.wd = static_cast<const __nv_bfloat16*>(w_down);
   a.y = static_cast<__nv_bfloat16*>(y);
-  a.logits = at<double>(ws, L.o_perm);
   a.h = at<__nv_bfloat16>(ws, L.h);
   a.idx_out = topk_idx;
   a.w_out = topk_w;

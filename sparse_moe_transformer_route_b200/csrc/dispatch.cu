@@ -31,6 +31,8 @@ __global__ void __launch_bounds__(kDispatchChunk)
                 int32_t* __restrict__ chunk_count, int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets_ws,
                 int32_t* __restrict__ gs_ws, int32_t* __restrict__ offsets_user, int32_t* __restrict__ gs_user,
                 int32_t* __restrict__ ticket, int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   __shared__ uint32_t mask[kMaxExperts * kWords];
   __shared__ int32_t total[kMaxExperts];
   __shared__ int s_last;
@@ -124,6 +126,8 @@ __global__ void __launch_bounds__(256)
                    const int32_t* __restrict__ offsets, const int32_t* __restrict__ gs, int32_t* __restrict__ perm,
                    int32_t* __restrict__ inv_perm, int32_t* __restrict__ row_pair, T_* __restrict__ x_perm,
                    int zero_pads) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp;
   const int nvec = d * static_cast<int>(sizeof(T_)) / 16;
@@ -177,7 +181,7 @@ cudaError_t launch_dispatch_impl(const Shape& s, const int32_t* idx, const void*
   int32_t* ctrl = at<int32_t>(ws, L.ctrl);
   cudaError_t e = cudaSuccess;
   const int nchunks = static_cast<int>(s.chunks());
-  rank_kernel<<<nchunks, kDispatchChunk, 0, st>>>(idx, s.T, s.E, s.k, at<int32_t>(ws, L.local_rank),
+  launch_dependent(rank_kernel, dim3(nchunks), dim3(kDispatchChunk), 0, st, nullptr, 0, idx, s.T, s.E, s.k, at<int32_t>(ws, L.local_rank),
                                                   at<int32_t>(ws, L.chunk_count), at<int32_t>(ws, L.chunk_base),
                                                   at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.group_start), offsets,
                                                   group_start, ctrl + 2, ctrl);
@@ -191,12 +195,12 @@ cudaError_t launch_permute(const Shape& s, const int32_t* idx, const void* x, in
   const int grid = static_cast<int>((s.T + 7) / 8);
   const int grid2 = zero_pads ? (grid > s.E ? grid : s.E) : grid;
   if (s.fp32) {
-    permute_kernel<float><<<grid2, 256, 0, st>>>(
+    launch_dependent(permute_kernel<float>, dim3(grid2), dim3(256), 0, st, nullptr, 0, 
         idx, static_cast<const float*>(x), s.T, s.d, s.E, s.k, at<int32_t>(ws, L.local_rank),
         at<int32_t>(ws, L.chunk_base), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.group_start), perm, inv_perm,
         at<int32_t>(ws, L.row_pair), static_cast<float*>(x_perm), zero_pads ? 1 : 0);
   } else {
-    permute_kernel<__nv_bfloat16><<<grid2, 256, 0, st>>>(
+    launch_dependent(permute_kernel<__nv_bfloat16>, dim3(grid2), dim3(256), 0, st, nullptr, 0, 
         idx, static_cast<const __nv_bfloat16*>(x), s.T, s.d, s.E, s.k, at<int32_t>(ws, L.local_rank),
         at<int32_t>(ws, L.chunk_base), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.group_start), perm, inv_perm,
         at<int32_t>(ws, L.row_pair), static_cast<__nv_bfloat16*>(x_perm), zero_pads ? 1 : 0);

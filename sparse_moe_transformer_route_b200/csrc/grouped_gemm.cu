@@ -45,8 +45,9 @@ enum class Epi { SwigluFwd, Store, SwigluBwd };
 // 64 B per MMA cycle instead of 96, the difference between starving and not
 // on HBM-resident weights. A 256-row tile whose second half lies past its
 // expert's rows issues only the first half.
-// O32: plain-store output in fp32 whatever the operand type (weight gradients
-// kept in fp32 for the caller's optimizer).
+// O32: fp32 output whatever the operand type: the plain store's result (weight
+// gradients kept in fp32 for the caller's optimizer), or the SwiGLU forward's
+// pre-activations (kept for the backward, which reads no rounded copy of them).
 template <bool TF32_, bool A_MN_, bool B_MN_, Group G_, Epi EP_, int BN_, int H_ = 1, bool O32_ = false>
 struct Cfg {
   static constexpr bool TF32 = TF32_;
@@ -91,7 +92,7 @@ struct Cfg {
   static_assert(H == 1 || H == 2, "tile M");
   static_assert(!(H == 2 && TF32), "256-row tiles are bf16 only");
   static_assert(!(EP == Epi::SwigluFwd && B_MN), "gate/up weights are read K-major");
-  static_assert(!O32 || EP == Epi::Store, "fp32 output only for plain stores");
+  static_assert(!O32 || EP != Epi::SwigluBwd, "fp32 output for plain stores and saved pre-activations");
 };
 
 struct Args {
@@ -310,12 +311,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
-    gs[i] = a.group_start[i];
-    off[i] = (a.offsets != nullptr) ? a.offsets[i] : 0;
-  }
-  __syncthreads();
-  if constexpr (C::G == Group::M) tile_starts<C>(a, gs, ts);
+  // prologue that reads nothing an earlier kernel writes, overlapping its tail
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -338,6 +335,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     tmem_relinquish();
   }
   __syncwarp();  // single-lane roles rejoin their warp before the block barrier
+  pdl_wait();
+  for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
+    gs[i] = a.group_start[i];
+    off[i] = (a.offsets != nullptr) ? a.offsets[i] : 0;
+  }
+  __syncthreads();
+  if constexpr (C::G == Group::M) tile_starts<C>(a, gs, ts);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -543,7 +547,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           warp_store_chunk<OutT, C::STG_PITCH>(stg, v, obase + c, a.ld_out, lane);
         }
       } else if constexpr (C::EP == Epi::SwigluFwd) {
-        T* pbase = (a.out2 != nullptr) ? static_cast<T*>(a.out2) + wrow0 * a.ld_out2 + t.n0 + cw : nullptr;
+        T* hbase = static_cast<T*>(a.out) + wrow0 * a.ld_out + t.n0 + cw;  // h has the operand type
+        OutT* pbase = (a.out2 != nullptr) ? static_cast<OutT*>(a.out2) + wrow0 * a.ld_out2 + t.n0 + cw : nullptr;
 #pragma unroll 1
         for (int c = 0; c < WCOLS; c += 32) {
           uint32_t rg[32], ru[32];
@@ -557,7 +562,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const float u = row_ok ? __uint_as_float(ru[i]) : 0.f;
             hv[i] = silu_fast(g) * u;
           }
-          warp_store_chunk<T, C::STG_PITCH>(stg, hv, obase + c, a.ld_out, lane);
+          warp_store_chunk<T, C::STG_PITCH>(stg, hv, hbase + c, a.ld_out, lane);
           if (pbase != nullptr) {
             float g[32], u[32];
 #pragma unroll
@@ -565,12 +570,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
               g[i] = row_ok ? __uint_as_float(rg[i]) : 0.f;
               u[i] = row_ok ? __uint_as_float(ru[i]) : 0.f;
             }
-            warp_store_chunk<T, C::STG_PITCH>(stg, g, pbase + c, a.ld_out2, lane);
-            warp_store_chunk<T, C::STG_PITCH>(stg, u, pbase + a.f_half + c, a.ld_out2, lane);
+            warp_store_chunk<OutT, C::STG_PITCH>(stg, g, pbase + c, a.ld_out2, lane);
+            warp_store_chunk<OutT, C::STG_PITCH>(stg, u, pbase + a.f_half + c, a.ld_out2, lane);
           }
         }
-      } else {  // SwigluBwd: accumulator holds dG for columns [n0, n0+BN)
-        const T* arow = static_cast<const T*>(a.aux) + row * a.ld_aux + t.n0 + cw;
+      } else {  // SwigluBwd: accumulator holds dG for columns [n0, n0+BN); the
+                // saved pre-activations are fp32
+        const float* arow = static_cast<const float*>(a.aux) + row * a.ld_aux + t.n0 + cw;
 #pragma unroll 1
         for (int c = 0; c < WCOLS; c += 32) {
           uint32_t r[32];
@@ -581,8 +587,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           for (int hh = 0; hh < 2; ++hh) {
             if (row_ok) {
               float av[16], bv[16];
-              load16<T>(arow + c + 16 * hh, av);
-              load16<T>(arow + a.f_half + c + 16 * hh, bv);
+              load16<float>(arow + c + 16 * hh, av);
+              load16<float>(arow + a.f_half + c + 16 * hh, bv);
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const float dg = __uint_as_float(r[16 * hh + i]);
@@ -631,9 +637,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // flight. Barriers: TMA bytes of both CTAs land on the leader's `full`; the
 // leader's commits arrive on `empty` and `acc_full` in both CTAs; both CTAs'
 // epilogues arrive on the leader's `acc_empty`.
-template <Epi EP_>
+// O32: the store epilogue writes fp32 (the expert outputs kept for the
+// backward), or the SwiGLU epilogue writes fp32 pre-activations.
+template <Epi EP_, bool O32_ = false>
 struct PairCfg {
   static constexpr Epi EP = EP_;
+  static constexpr bool O32 = O32_;
+  using OutT = std::conditional_t<O32, float, __nv_bfloat16>;  // store output / pre-activations
   static constexpr int BN = 256;                   // accumulator columns per tile
   static constexpr int BK = 64;                    // K per stage (one 128-byte swizzle row)
   static constexpr int UK = 16;                    // K per UMMA
@@ -646,7 +656,7 @@ struct PairCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int STG_PITCH = 32 * 2 + 16;
+  static constexpr int STG_PITCH = 32 * static_cast<int>(sizeof(OutT)) + 16;
   static constexpr int STG_WARP_BYTES = 32 * STG_PITCH;
   static constexpr int STG_BYTES = EPI_WARPS * STG_WARP_BYTES;
   static constexpr int MISC_BYTES = 1024 + 3 * (kMaxExperts + 1) * static_cast<int>(sizeof(int32_t));
@@ -702,7 +712,8 @@ template <class P>
 __global__ void __launch_bounds__(P::THREADS, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const Args a) {
-  using OutT = __nv_bfloat16;
+  using OutT = typename P::OutT;
+  using HT = __nv_bfloat16;  // h, the SwiGLU output
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -726,12 +737,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
   const int cluster = static_cast<int>(blockIdx.x >> 1);
   const int n_clusters = static_cast<int>(gridDim.x >> 1);
 
-  for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
-    gs[i] = a.group_start[i];
-    off[i] = a.offsets[i];
-  }
-  __syncthreads();
-  pair_tile_starts(a.E, gs, pts);
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < P::STAGES; ++s) {
       mbar_init(&full[s], 1);   // the leader's expect_tx arrival (its copy is the one used)
@@ -752,8 +758,18 @@ __global__ void __launch_bounds__(P::THREADS, 1)
     tmem_alloc_pair(tmem_holder, P::TMEM_COLS);
     tmem_relinquish_pair();
   }
+  __syncwarp();
+  // the group layout comes from an earlier kernel
+  pdl_wait();
+  for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
+    gs[i] = a.group_start[i];
+    off[i] = a.offsets[i];
+  }
+  __syncthreads();
+  pair_tile_starts(a.E, gs, pts);
   tc_fence_before();
-  // both CTAs' barriers are initialised before either CTA's copies or commits reach them
+  // both CTAs' barriers are initialised before either CTA's copies or commits
+  // reach them (and the tile starts are visible to every warp)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
@@ -852,7 +868,6 @@ __global__ void __launch_bounds__(P::THREADS, 1)
     const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    OutT* out = static_cast<OutT*>(a.out);
     for (int L = cluster; L < n_tiles; L += n_clusters) {
       const PairTile t = decode_pair_tile<P>(a, gs, off, pts, L, rank);
       if (!mbar_wait(&acc_full[acc], acc_phase)) {
@@ -865,11 +880,11 @@ __global__ void __launch_bounds__(P::THREADS, 1)
         const int64_t wrow0 = static_cast<int64_t>(t.m0) + 128 * static_cast<int>(rank) + q * 32;
         constexpr int WCOLS = P::OUT_N / 2;
         const int cw = csel * WCOLS;
-        OutT* obase = out + wrow0 * a.ld_out + t.n0 + cw;
         unsigned char* stg = stg_base + (warp - 2) * P::STG_WARP_BYTES;
         const uint32_t tbase =
             tmem_base + static_cast<uint32_t>(acc * P::BN + cw) + (static_cast<uint32_t>(q * 32) << 16);
         if constexpr (P::EP == Epi::Store) {
+          OutT* obase = static_cast<OutT*>(a.out) + wrow0 * a.ld_out + t.n0 + cw;
 #pragma unroll 1
           for (int c = 0; c < WCOLS; c += 32) {
             uint32_t r[32];
@@ -881,6 +896,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
             warp_store_chunk<OutT, P::STG_PITCH>(stg, v, obase + c, a.ld_out, lane);
           }
         } else {
+          HT* obase = static_cast<HT*>(a.out) + wrow0 * a.ld_out + t.n0 + cw;
           OutT* pbase =
               (a.out2 != nullptr) ? static_cast<OutT*>(a.out2) + wrow0 * a.ld_out2 + t.n0 + cw : nullptr;
 #pragma unroll 1
@@ -896,7 +912,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
               const float u = row_ok ? __uint_as_float(ru[i]) : 0.f;
               hv[i] = silu_fast(g) * u;
             }
-            warp_store_chunk<OutT, P::STG_PITCH>(stg, hv, obase + c, a.ld_out, lane);
+            warp_store_chunk<HT, P::STG_PITCH>(stg, hv, obase + c, a.ld_out, lane);
             if (pbase != nullptr) {  // the pre-activations, kept for the backward
               float g[32], u[32];
 #pragma unroll
@@ -974,8 +990,8 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtenso
   int grid = device_sm_count();
   if (max_tiles < grid) grid = max_tiles;
   if (grid <= 0) return cudaSuccess;
-  grouped_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(ta, ta32, tb, a);
-  return cudaGetLastError();
+  return launch_dependent(grouped_gemm_kernel<C>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, nullptr, 0, ta,
+                          ta32, tb, a);
 }
 
 template <class P>
@@ -987,19 +1003,13 @@ cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const Args
   int clusters = device_sm_count() / 2;
   if (max_pair_tiles < clusters) clusters = max_pair_tiles;
   if (clusters <= 0) return cudaSuccess;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  cfg.blockDim = dim3(P::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = P::SMEM_BYTES;
-  cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, pair_gemm_kernel<P>, ta, tb, a);
+  return launch_dependent(pair_gemm_kernel<P>, dim3(static_cast<unsigned>(2 * clusters)), dim3(P::THREADS),
+                          P::SMEM_BYTES, st, attr, 1, ta, tb, a);
 }
 
 // Pair tiles of 256 rows are used when the groups are large: a group of R rows
@@ -1070,6 +1080,7 @@ cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* gr
     a.out2 = preact;
     a.ld_out2 = 2 * s.f;
     const int max_pairs = static_cast<int>((s.P / 256 + s.E) * (s.f / 128));
+    if (preact != nullptr) return launch_pair<PairCfg<Epi::SwigluFwd, true>>(ta, tb, a, max_pairs, st);
     return launch_pair<PairCfg<Epi::SwigluFwd>>(ta, tb, a, max_pairs, st);
   }
   // accumulator: BN/2 gate columns and BN/2 up columns of the same outputs
@@ -1090,11 +1101,14 @@ cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* gr
   a.out2 = preact;
   a.ld_out2 = 2 * s.f;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.f / (bn / 2)));
+  if (preact != nullptr)  // pre-activations kept in fp32 for the backward
+    return run_variant<false, false, Group::M, Epi::SwigluFwd, true>(s.fp32, bn, pick_h(s), ta, ta32, tb, a, max_tiles,
+                                                                     st);
   return run_variant<false, false, Group::M, Epi::SwigluFwd>(s.fp32, bn, pick_h(s), ta, ta32, tb, a, max_tiles, st);
 }
 
 cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_start, const int32_t* offsets,
-                        const void* w_down, void* o_perm, int32_t* status, cudaStream_t st) {
+                        const void* w_down, void* o_perm, bool out32, int32_t* status, cudaStream_t st) {
   if (use_pairs(s) && s.d % 256 == 0) {
     CUtensorMap ta, tb;
     if (!make_map(&ta, h, false, s.P, s.f, 64, 128)) return cudaErrorInvalidValue;
@@ -1106,6 +1120,7 @@ cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_star
     a.out = o_perm;
     a.ld_out = s.d;
     const int max_pairs = static_cast<int>((s.P / 256 + s.E) * (s.d / 256));
+    if (out32) return launch_pair<PairCfg<Epi::Store, true>>(ta, tb, a, max_pairs, st);
     return launch_pair<PairCfg<Epi::Store>>(ta, tb, a, max_pairs, st);
   }
   const int bn = few_tiles(s, s.d) ? 128 : pick_bn(s.d);
@@ -1122,6 +1137,8 @@ cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_star
   a.out = o_perm;
   a.ld_out = s.d;
   const int max_tiles = static_cast<int>((s.P / 128) * (s.d / bn));
+  if (out32)
+    return run_variant<false, false, Group::M, Epi::Store, true>(s.fp32, bn, pick_h(s), ta, ta32, tb, a, max_tiles, st);
   return run_variant<false, false, Group::M, Epi::Store>(s.fp32, bn, pick_h(s), ta, ta32, tb, a, max_tiles, st);
 }
 

@@ -118,7 +118,8 @@ Workspace layout(const Shape& s) {
   L.ec_gate = take(P * 4);
   L.ec_slot = take(T * E * 4);
   L.fwd_bytes = o;
-  L.preact = take(P * 2 * s.f * s.esize);
+  L.preact = take(P * 2 * s.f * 4);
+  L.o32 = take(P * s.d * 4);
   L.dw = take(T * k * 4);
   L.dh = take(T * E * 4);
   L.dout = take(P * s.d * s.esize);
@@ -189,7 +190,7 @@ moe_status forward_impl(const Ctx& c, const void* x, const void* w_router, const
   MOE_TRY(marks.mark(0));
   if (!save && resid == nullptr && s.T <= kDecodeAutoTokens && decode_supported(s)) {
     // a decode-sized batch: the whole layer in one kernel (every stage mark after it)
-    MOE_TRY(launch_decode_layer(s, x, nullptr, 0.f, w_router, bias, w_gate_up, w_down, y, topk_idx, topk_w, counts,
+    MOE_TRY(launch_decode_layer(s, x, nullptr, 0.0, w_router, bias, w_gate_up, w_down, y, topk_idx, topk_w, counts,
                                 losses, ws, L, st));
     for (int i = 1; i <= 5; ++i) MOE_TRY(marks.mark(i));
     return MOE_OK;
@@ -209,9 +210,12 @@ moe_status forward_impl(const Ctx& c, const void* x, const void* w_router, const
   MOE_TRY(launch_gate_up(s, x_perm, gs, off, w_gate_up, at<void>(ws, L.h), save ? at<void>(ws, L.preact) : nullptr,
                          status, st));
   MOE_TRY(marks.mark(3));
-  MOE_TRY(launch_down(s, at<void>(ws, L.h), gs, off, w_down, at<void>(ws, L.o_perm), status, st));
+  // Kept for the backward, the expert outputs stay in fp32: the router's
+  // gradient dw = <dy, o> reads them and no contraction does.
+  void* o_rows = save ? at<void>(ws, L.o32) : at<void>(ws, L.o_perm);
+  MOE_TRY(launch_down(s, at<void>(ws, L.h), gs, off, w_down, o_rows, save, status, st));
   MOE_TRY(marks.mark(4));
-  MOE_TRY(launch_combine(s, at<void>(ws, L.o_perm), at<int32_t>(ws, L.inv_perm), wts, y, resid, st));
+  MOE_TRY(launch_combine(s, o_rows, save, at<int32_t>(ws, L.inv_perm), wts, y, resid, st));
   MOE_TRY(marks.mark(5));
   const size_t nk = static_cast<size_t>(s.T) * s.k;
   if (topk_idx != nullptr) MOE_TRY(cudaMemcpyAsync(topk_idx, idx, nk * 4, cudaMemcpyDeviceToDevice, st));
@@ -324,7 +328,7 @@ moe_status moe_expert_down(const moe_config* cfg, const void* h, const int32_t* 
   if (h == nullptr || group_start == nullptr || offsets == nullptr || w_down == nullptr || o_perm == nullptr ||
       !aligned16(h) || !aligned16(w_down) || !aligned16(o_perm))
     return MOE_ERR_INVALID_ARG;
-  MOE_TRY(launch_down(c.s, h, group_start, offsets, w_down, o_perm, at<int32_t>(ws, c.L.ctrl), stream));
+  MOE_TRY(launch_down(c.s, h, group_start, offsets, w_down, o_perm, false, at<int32_t>(ws, c.L.ctrl), stream));
   return MOE_OK;
 }
 
@@ -346,7 +350,7 @@ moe_status moe_combine(const moe_config* cfg, const void* o_perm, const int32_t*
     return MOE_ERR_INVALID_ARG;
   moe_status r = device_ready();
   if (r != MOE_OK) return r;
-  MOE_TRY(launch_combine(s, o_perm, inv_perm, topk_w, y, nullptr, stream));
+  MOE_TRY(launch_combine(s, o_perm, false, inv_perm, topk_w, y, nullptr, stream));
   return MOE_OK;
 }
 
@@ -360,7 +364,7 @@ moe_status moe_combine_residual(const moe_config* cfg, const void* o_perm, const
     return MOE_ERR_INVALID_ARG;
   moe_status r = device_ready();
   if (r != MOE_OK) return r;
-  MOE_TRY(launch_combine(s, o_perm, inv_perm, topk_w, nullptr, resid, stream));
+  MOE_TRY(launch_combine(s, o_perm, false, inv_perm, topk_w, nullptr, resid, stream));
   return MOE_OK;
 }
 
@@ -387,14 +391,14 @@ moe_status moe_forward_decode(const moe_config* cfg, const void* x, const void* 
   if (x == nullptr || w_router == nullptr || w_gate_up == nullptr || w_down == nullptr || y == nullptr ||
       !aligned16(x) || !aligned16(w_router) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y))
     return MOE_ERR_INVALID_ARG;
-  MOE_TRY(launch_decode_layer(c.s, x, nullptr, 0.f, w_router, router_bias, w_gate_up, w_down, y, topk_idx, topk_w,
+  MOE_TRY(launch_decode_layer(c.s, x, nullptr, 0.0, w_router, router_bias, w_gate_up, w_down, y, topk_idx, topk_w,
                               nullptr, losses, ws, c.L, stream));
   return MOE_OK;
 }
 
-moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const void* w_router,
-                            const float* router_bias, const void* w_gate_up, const void* w_down, void* y_host,
-                            float* losses_host, void* ws, size_t ws_bytes, cudaStream_t stream) {
+moe_status moe_forward_host_async(const moe_config* cfg, const void* x_host, const void* w_router,
+                                  const float* router_bias, const void* w_gate_up, const void* w_down, void* y_host,
+                                  float* losses_host, void* ws, size_t ws_bytes, cudaStream_t stream) {
   Ctx c;
   moe_status r = prepare(cfg, ws, ws_bytes, false, &c);
   if (r != MOE_OK) return r;
@@ -412,6 +416,15 @@ moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const voi
   if (losses_host != nullptr)
     MOE_TRY(cudaMemcpyAsync(losses_host, at<float>(ws, c.L.losses), 2 * sizeof(float), cudaMemcpyDeviceToHost,
                             stream));
+  return MOE_OK;
+}
+
+moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const void* w_router,
+                            const float* router_bias, const void* w_gate_up, const void* w_down, void* y_host,
+                            float* losses_host, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const moe_status r = moe_forward_host_async(cfg, x_host, w_router, router_bias, w_gate_up, w_down, y_host,
+                                              losses_host, ws, ws_bytes, stream);
+  if (r != MOE_OK) return r;
   MOE_TRY(cudaStreamSynchronize(stream));
   return MOE_OK;
 }
@@ -435,7 +448,7 @@ moe_status moe_backward(const moe_config* cfg, const void* dy, const void* x, co
   int32_t* off = at<int32_t>(ws, L.offsets);
   float* dw = at<float>(ws, L.dw);
   float* dh = at<float>(ws, L.dh);
-  MOE_TRY(launch_combine_backward(s, dy, at<void>(ws, L.o_perm), gs, at<int32_t>(ws, L.row_pair), at<float>(ws, L.wts),
+  MOE_TRY(launch_combine_backward(s, dy, at<void>(ws, L.o32), gs, at<int32_t>(ws, L.row_pair), at<float>(ws, L.wts),
                                   dw, at<void>(ws, L.dout), stream));
   MOE_TRY(launch_router_backward(s, dw, at<int32_t>(ws, L.idx), at<float>(ws, L.probs), at<float>(ws, L.lse),
                                  at<int32_t>(ws, L.counts), cfg->alpha_lb, cfg->beta_z, dh, stream));
@@ -503,7 +516,7 @@ moe_status moe_forward_expert_choice(const moe_config* cfg, int64_t capacity, co
   MOE_TRY(marks.mark(2));
   MOE_TRY(launch_gate_up(s, x_perm, gs, off, w_gate_up, at<void>(ws, L.h), nullptr, status, stream));
   MOE_TRY(marks.mark(3));
-  MOE_TRY(launch_down(s, at<void>(ws, L.h), gs, off, w_down, at<void>(ws, L.o_perm), status, stream));
+  MOE_TRY(launch_down(s, at<void>(ws, L.h), gs, off, w_down, at<void>(ws, L.o_perm), false, status, stream));
   MOE_TRY(marks.mark(4));
   MOE_TRY(launch_combine_ec(s, at<void>(ws, L.o_perm), at<int32_t>(ws, L.ec_slot), at<float>(ws, L.probs), y, stream));
   MOE_TRY(marks.mark(5));
@@ -543,7 +556,7 @@ moe_status moe_stack_forward_trace(const moe_config* cfg, int32_t n_layers, cons
   if (c.s.T <= kDecodeAutoTokens && decode_supported(c.s)) {  // RMSNorm, layer and residual add in one kernel
     for (int l = 0; l < n_layers; ++l) {
       const float* bias = (router_biases != nullptr) ? router_biases[l] : nullptr;
-      MOE_TRY(launch_decode_layer(c.s, nullptr, resid, 1e-5f, w_router[l], bias, w_gate_up[l], w_down[l], nullptr,
+      MOE_TRY(launch_decode_layer(c.s, nullptr, resid, kStackRmsEps, w_router[l], bias, w_gate_up[l], w_down[l], nullptr,
                                   topk_idx != nullptr ? topk_idx + l * tk : nullptr, nullptr,
                                   counts != nullptr ? counts + static_cast<int64_t>(l) * c.s.E : nullptr,
                                   losses != nullptr ? losses + 2 * l : nullptr, ws, c.L, stream));
@@ -551,7 +564,7 @@ moe_status moe_stack_forward_trace(const moe_config* cfg, int32_t n_layers, cons
     return MOE_OK;
   }
   for (int l = 0; l < n_layers; ++l) {
-    MOE_TRY(launch_rmsnorm(c.s, resid, nullptr, 1e-5f, xn, stream));
+    MOE_TRY(launch_rmsnorm(c.s, resid, nullptr, kStackRmsEps, xn, stream));
     const float* bias = (router_biases != nullptr) ? router_biases[l] : nullptr;
     r = forward_impl(c, xn, w_router[l], bias, w_gate_up[l], w_down[l], nullptr,
                      losses != nullptr ? losses + 2 * l : nullptr, resid,

@@ -43,7 +43,8 @@ struct Workspace {
   size_t local_rank, chunk_count, chunk_base;
   size_t offsets, group_start, perm, inv_perm, row_pair;
   size_t x_perm, h, o_perm;
-  size_t preact;                              // [P, 2f] (training)
+  size_t preact;                              // [P, 2f] fp32 (training)
+  size_t o32;                                 // [P, d] fp32 expert outputs (training)
   size_t dw, dh, dout, dab, dx_perm, wr_part; // backward scratch
   size_t x_dev, y_dev;                        // staging for the host-buffer entry point
   size_t ec_sel, ec_gate, ec_slot;            // expert choice: [E, C] tokens and weights, [T, E] rows
@@ -77,9 +78,13 @@ cudaError_t launch_dispatch(const Shape& s, const int32_t* idx, const void* x, i
 cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* group_start,
                            const int32_t* offsets, const void* w_gate_up, void* h, void* preact, int32_t* status,
                            cudaStream_t st);
+// gate/up: `preact` (or null) receives the pre-activations in fp32.
+// down: o_perm in fp32 when `out32` (the expert outputs kept for the backward),
+// else in the layer dtype.
 cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_start, const int32_t* offsets,
-                        const void* w_down, void* o_perm, int32_t* status, cudaStream_t st);
-cudaError_t launch_combine(const Shape& s, const void* o_perm, const int32_t* inv_perm, const float* wts,
+                        const void* w_down, void* o_perm, bool out32, int32_t* status, cudaStream_t st);
+// `o32`: o_perm holds fp32 rows (the saved expert outputs) instead of the layer dtype.
+cudaError_t launch_combine(const Shape& s, const void* o_perm, bool o32, const int32_t* inv_perm, const float* wts,
                            void* y, float* resid, cudaStream_t st);
 // Expert choice: the router's probabilities and log-normaliser only (no top-k),
 // then each expert's top-C tokens, the row gather and the combine.
@@ -103,14 +108,19 @@ bool decode_supported(const Shape& s);
 // layered, T=4 97 against 157, T=6 155 against 159; at T=8 they tie, and in
 // CUDA-graph replays the layered path is ahead there, 166 against 176 us).
 constexpr int64_t kDecodeAutoTokens = 6;
-cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, float eps, const void* w_router,
+cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, double eps, const void* w_router,
                                 const float* bias, const void* w_gate_up, const void* w_down, void* y,
                                 int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,
                                 const Workspace& L, cudaStream_t st);
-cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, float eps, void* out,
+// RMSNorm of the fp32 residual, evaluated in fp64 and rounded once to fp32
+// and then to the layer dtype.
+cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, double eps, void* out,
                            cudaStream_t st);
+// eps of the stack's pre-norm ("Mixture-of-experts LLMs from scratch with OLMoE",
+// section 3: RMSNorm with the library default 1e-5)
+constexpr double kStackRmsEps = 1e-5;
 
-// backward pieces
+// backward pieces (o32: the fp32 expert outputs saved by the forward)
 cudaError_t launch_dispatch_impl(const Shape& s, const int32_t* idx, const void* x, int32_t* offsets,
                                  int32_t* perm, int32_t* inv_perm, int32_t* group_start, void* x_perm, void* ws,
                                  const Workspace& L, bool zero_pads, cudaStream_t st);
@@ -136,6 +146,28 @@ cudaError_t launch_router_weight_grad(const Shape& s, const float* dh, const voi
 size_t router_wgrad_partial_bytes(const Shape& s);
 
 int device_sm_count();
+
+// Launches `kern` as a programmatic dependent of the previous kernel in the
+// stream: it may be scheduled while that kernel finishes, and calls pdl_wait()
+// (sm100.cuh) before touching memory an earlier kernel writes or reads.
+// `extra` (or null) are further launch attributes (a cluster shape).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             const cudaLaunchAttribute* extra, int n_extra, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[4];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  for (int i = 0; i < n_extra && n < 4; ++i) attr[n++] = extra[i];
+  cfg.attrs = attr;
+  cfg.numAttrs = static_cast<unsigned>(n);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 // Raises `func`'s dynamic shared-memory limit to at least `bytes` on the current
 // device. `cache` (one entry per device id < 64, zero-initialised, owned by the

@@ -35,6 +35,8 @@ __global__ void __launch_bounds__(kThreads) router_kernel(
     float* __restrict__ lse_out, int32_t* __restrict__ counts_part, float* __restrict__ psum_part,
     double* __restrict__ zsum_part, int32_t* __restrict__ counts_ws, int32_t* __restrict__ counts_user,
     float* __restrict__ losses_ws, float* __restrict__ losses_user, int32_t* __restrict__ ticket, int renorm) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
   extern __shared__ __align__(16) unsigned char smem[];
   Tin* xs = reinterpret_cast<Tin*>(smem);                                            // [kTok][d]
   double* logit = reinterpret_cast<double*>(smem + static_cast<size_t>(kTok) * d * sizeof(Tin));  // [kTok][E]
@@ -247,7 +249,7 @@ cudaError_t run(const Shape& s, const void* x, const void* w_router, const float
   // ctrl[1] is zero between calls (moe_workspace_init, then each launch's last CTA)
   int32_t* ctrl = at<int32_t>(ws, L.ctrl);
   const int grid = static_cast<int>(s.router_ctas());
-  router_kernel<Tin><<<grid, kThreads, smem, st>>>(
+  launch_dependent(router_kernel<Tin>, dim3(grid), dim3(kThreads), smem, st, nullptr, 0, 
       static_cast<const Tin*>(x), static_cast<const Tin*>(w_router), bias, s.T, s.d, s.E, s.k, idx, wts,
       at<float>(ws, L.probs), at<float>(ws, L.lse), at<int32_t>(ws, L.counts_part), at<float>(ws, L.psum_part),
       at<double>(ws, L.zsum_part), at<int32_t>(ws, L.counts), counts, at<float>(ws, L.losses), losses, ctrl + 1,
@@ -319,24 +321,52 @@ StaticLayout static_layout(const Shape& s) {
   return L;
 }
 
-constexpr int kMaxDevices = 64;
+// The array's device address belongs to the context it was looked up in; a
+// device reset (or any new primary context) loads the module afresh, so the
+// address is kept together with the context and looked up again when the
+// current context is another one.
+struct ScratchAddr {
+  CUcontext ctx = nullptr;
+  unsigned char* addr = nullptr;
+};
 std::mutex g_scratch_mu;
-unsigned char* g_scratch_addr[kMaxDevices] = {};
+ScratchAddr g_scratch[kMaxDevices];
 
-// Device address of g_route_scratch on the current device (looked up once per device).
+using CtxGetCurrent = CUresult (*)(CUcontext*);
+
+CtxGetCurrent ctx_get_current() {
+  static CtxGetCurrent fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrent>(p);
+    return static_cast<CtxGetCurrent>(nullptr);
+  }();
+  return fn;
+}
+
+// Device address of g_route_scratch in the current device's current context.
 cudaError_t static_scratch(unsigned char** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const CtxGetCurrent get_ctx = ctx_get_current();
+  if (get_ctx == nullptr) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchAddr& c = g_scratch[dev];
+  if (c.addr == nullptr || ctx == nullptr || c.ctx != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    e = cudaGetSymbolAddress(&p, g_route_scratch);  // makes the primary context current if none was
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = static_cast<unsigned char*>(p);
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
+    c.ctx = ctx;
+    c.addr = static_cast<unsigned char*>(p);
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return cudaSuccess;
 }
 
@@ -346,16 +376,16 @@ cudaError_t run_static(const Shape& s, const void* x, const void* w_router, cons
                        cudaStream_t st) {
   const size_t smem = static_cast<size_t>(kTok) * s.d * sizeof(Tin) + static_cast<size_t>(kTok) * s.E * 12 +
                       kTok * 4 + s.E * 4;
+  static std::atomic<size_t> smem_set[moe::kMaxDevices];
   if (smem > 48 * 1024) {
-    cudaError_t e =
-        cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(router_kernel<Tin>), smem, smem_set);
     if (e != cudaSuccess) return e;
   }
   int32_t* ticket = reinterpret_cast<int32_t*>(scratch + L.ticket);
   cudaError_t e = cudaMemsetAsync(ticket, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(s.router_ctas());
-  router_kernel<Tin><<<grid, kThreads, smem, st>>>(
+  launch_dependent(router_kernel<Tin>, dim3(grid), dim3(kThreads), smem, st, nullptr, 0, 
       static_cast<const Tin*>(x), static_cast<const Tin*>(w_router), bias, s.T, s.d, s.E, s.k, idx, wts,
       reinterpret_cast<float*>(scratch + L.probs), reinterpret_cast<float*>(scratch + L.lse),
       reinterpret_cast<int32_t*>(scratch + L.counts_part), reinterpret_cast<float*>(scratch + L.psum_part),

@@ -601,6 +601,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const int nk = a.d / 64;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
 
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -617,6 +618,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_wait();  // x may come from the kernel before (the stack's RMSNorm)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -739,6 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kb_lo = (ks * (a.d / 64)) / a.ksplit;
   const int nk = ((ks + 1) * (a.d / 64)) / a.ksplit - kb_lo;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kLogitTile;
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kLogitStages; ++s) {
       mbar_init(&full[s], 1);
@@ -755,6 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_wait();
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tmx);
@@ -861,8 +865,10 @@ __global__ void __launch_bounds__(128, 2) router_epi_kernel(const RArgs a) {
   int32_t* qn = s_last + 1;
   const int tid = threadIdx.x, lane = tid & 31;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
+  pdl_trigger();
   if (tid < kMaxE) mask[tid] = 0u;
   if (tid == 0) *qn = 0;
+  pdl_wait();
   // this tile's logits: the K-range partials (all loads in flight, then summed
   // in a fixed order), plus the offset
   for (int i = tid; i < kTile * kMaxE; i += 128) {
@@ -945,10 +951,9 @@ cudaError_t router_tc_impl(const Shape& s, const void* x, const void* w_router, 
   // Up to one wave of 32-token tiles: the fused kernel (T=64: 28.7 us against
   // 41.0 us split; T=4096: 40.9 us against 49.2 us). More tiles than SMs: the
   // split form (T=16384: 87-94 us against 102 us fused).
-  if (s.T > 8 && static_cast<int>(grid) <= device_sm_count()) {
-    router_tc_kernel<16, 1><<<grid, kThreads, smem_bytes(16), st>>>(tx, tw, a);
-    return cudaGetLastError();
-  }
+  if (s.T > 8 && static_cast<int>(grid) <= device_sm_count())
+    return launch_dependent(router_tc_kernel<16, 1>, dim3(grid), dim3(kThreads), smem_bytes(16), st, nullptr, 0, tx,
+                            tw, a);
   CUtensorMap tx128;
   if (!make_map(&tx128, x, false, static_cast<uint64_t>(s.T), s.d, 64, kLogitTile)) return cudaErrorInvalidValue;
   const unsigned grid_l = static_cast<unsigned>((s.T + kLogitTile - 1) / kLogitTile);
@@ -959,17 +964,15 @@ cudaError_t router_tc_impl(const Shape& s, const void* x, const void* w_router, 
   while (ks > 1 && s.d / 64 / ks < 2) --ks;
   const size_t cap = static_cast<size_t>(s.P) * s.d * s.esize;
   while (ks > 1 && static_cast<size_t>(ks) * s.T * s.E * 4 > cap) --ks;
-  if (static_cast<size_t>(ks) * s.T * s.E * 4 > cap) {  // tiny layers: the fused kernel
-    router_tc_kernel<16, 1><<<grid, kThreads, smem_bytes(16), st>>>(tx, tw, a);
-    return cudaGetLastError();
-  }
+  if (static_cast<size_t>(ks) * s.T * s.E * 4 > cap)  // tiny layers: the fused kernel
+    return launch_dependent(router_tc_kernel<16, 1>, dim3(grid), dim3(kThreads), smem_bytes(16), st, nullptr, 0, tx,
+                            tw, a);
   a.logit_part = at<float>(ws, L.x_perm);
   a.ksplit = ks;
-  router_logits_kernel<<<dim3(grid_l, static_cast<unsigned>(ks)), kThreads, kLogitSmem, st>>>(tx128, tw, a);
-  e = cudaGetLastError();
+  e = launch_dependent(router_logits_kernel, dim3(grid_l, static_cast<unsigned>(ks)), dim3(kThreads), kLogitSmem, st,
+                       nullptr, 0, tx128, tw, a);
   if (e != cudaSuccess) return e;
-  router_epi_kernel<<<grid, 128, kEpiSmem, st>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(router_epi_kernel, dim3(grid), dim3(128), kEpiSmem, st, nullptr, 0, a);
 }
 }  // namespace
 

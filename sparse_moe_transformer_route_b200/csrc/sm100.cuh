@@ -41,6 +41,17 @@ __device__ __forceinline__ void report(int32_t* status, int32_t code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Kernels of the layer are launched as programmatic dependents of the kernel
+// before them in the stream: each lets its successor be scheduled early
+// (pdl_trigger) and, before it touches global memory that an earlier kernel
+// writes or reads, waits until every earlier kernel has completed and its
+// writes are visible (pdl_wait). Without the launch attribute both are no-ops.
+
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

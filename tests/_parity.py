@@ -21,6 +21,17 @@ def f64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
+def bf16_round(a):
+    """fp64 values rounded to bf16 the way the kernels round an fp32 result: to
+    fp32 first, then to bf16 (both round to nearest even); returned as fp64."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+    return t.to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def f32_round(a):
+    return np.asarray(a, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
 def errors(got, ref):
     got = f64(got)
     ref = np.asarray(ref, dtype=np.float64)

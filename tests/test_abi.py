@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol():
 def test_library_has_no_gpu_only_load_dependencies():
     # static CUDA runtime: the .so must load here, where there is no driver
     lib = M.lib()
-    assert lib.moe_abi_version() == B.ABI_VERSION == 5
+    assert lib.moe_abi_version() == B.ABI_VERSION == 6
 
 
 def test_status_strings():
@@ -110,7 +110,8 @@ def test_workspace_sizes_grow_with_training():
     bwd = M.moe_workspace_bytes(cfg, True)
     P = M.moe_padded_rows(cfg)
     assert fwd >= P * 2048 * 2 * 2 + P * 1024 * 2  # x_perm, o_perm, h
-    assert bwd > fwd + P * 2 * 1024 * 2           # + the saved pre-activations
+    # + the saved fp32 pre-activations and fp32 expert outputs
+    assert bwd > fwd + P * 2 * 1024 * 4 + P * 2048 * 4
 
 
 def test_binding_rejects_wrong_tensors_before_calling():
@@ -149,3 +150,23 @@ def test_binding_checks_the_new_entry_points_before_calling():
         M.moe_route_expert_choice(cfg, x, wr, None, sel, gates, None, None, None, ws)
     with pytest.raises(ValueError, match="x must have shape"):
         M.moe_forward_expert_choice(cfg, torch.zeros(4, 256, dtype=bf), wr, None, wgu, wd, x, None, sel, gates, ws)
+    with pytest.raises(ValueError, match="x_host must be a host tensor"):
+        M.moe_forward_host_async(cfg, x.cuda() if torch.cuda.is_available() else _FakeCuda(x), wr, None, wgu, wd,
+                                 x, None, ws)
+    with pytest.raises(TypeError, match="x_host must be torch.bfloat16"):
+        M.moe_forward_host_async(cfg, x.float(), wr, None, wgu, wd, x, None, ws)
+    with pytest.raises(ValueError, match="w_router must be a CUDA tensor"):
+        M.moe_forward_host_async(cfg, x, wr, None, wgu, wd, x, None, ws)
+
+
+class _FakeCuda(torch.Tensor):
+    """A host tensor that reports itself as a CUDA tensor (for the binding's
+    host-or-device check on a machine without a GPU)."""
+
+    @staticmethod
+    def __new__(cls, t):
+        return torch.Tensor._make_subclass(cls, t)
+
+    @property
+    def is_cuda(self):
+        return True

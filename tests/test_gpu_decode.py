@@ -17,7 +17,7 @@ import sparse_moe_transformer_route_b200 as M
 from oracle import moe_oracle as O
 from sparse_moe_transformer_route_b200 import synthetic as S
 from tests._parity import LazyF64, assert_close, assert_loss_close, f64, require_gpu
-from tests.test_gpu_workloads import _stack_reference
+from tests.test_gpu_workloads import _check_stack_per_layer, _gpu_stack_layers
 
 pytestmark = pytest.mark.gpu
 
@@ -128,31 +128,22 @@ def test_shapes_and_options(T, d, E, k, f, bias, renorm):
 
 def test_stack_of_decode_layers():
     """Four skewed layers at T = 4 (one fused launch per layer, RMSNorm and the
-    residual add inside), every token against the oracle's stack; the trace
-    variant gives the same residual and consistent per-layer counts."""
+    residual add inside): every token of every layer against the oracle fed
+    that layer's input; the whole stack in one call equals its trace variant
+    and its single-layer calls, with consistent per-layer counts."""
     sh = S.LayerShape(T=4, d_model=512, n_experts=64, top_k=8, d_ff=256)
     n = 4
     x0, layers = S.stack_inputs(sh, n, seed=13)
-    cfg = M.config(sh.T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff)
-    ws = M.workspace(cfg, False)
-    dev = [{kk: (v.cuda() if v is not None else None) for kk, v in L.items()} for L in layers]
-    r1 = x0.clone().cuda()
-    M.moe_stack_forward(cfg, dev, r1, ws)
-    r2 = x0.clone().cuda()
-    counts = torch.empty(n, sh.n_experts, dtype=torch.int32, device="cuda")
-    losses = torch.empty(n, 2, device="cuda")
-    idx = torch.empty(n, sh.T, sh.top_k, dtype=torch.int32, device="cuda")
-    M.moe_stack_forward_trace(cfg, dev, r2, ws, counts, losses, idx)
-    torch.cuda.synchronize()
-    assert M.moe_get_device_status(ws) == 0
+    _check_stack_per_layer(sh, x0, layers)
+    r1, _ = _gpu_stack_layers(sh, x0, layers, trace=False)
+    r2, tr = _gpu_stack_layers(sh, x0, layers)
     assert torch.equal(r1, r2)
-    counts, idx = counts.cpu().numpy(), idx.cpu().numpy()
+    r = x0
+    for L in layers:
+        r, _ = _gpu_stack_layers(sh, r, [L], trace=False)
+    assert torch.equal(r1, r)
     for l in range(n):
-        assert np.array_equal(np.bincount(idx[l].reshape(-1), minlength=sh.n_experts), counts[l])
-    ref, tainted = _stack_reference(x0, layers, sh.top_k)
-    ok = torch.from_numpy(~tainted)
-    assert ok.sum() >= 2
-    assert_close(r1.cpu()[ok], ref[~tainted], "stack residual")
+        assert np.array_equal(np.bincount(tr["idx"][l].reshape(-1), minlength=sh.n_experts), tr["counts"][l])
 
 
 def test_deterministic_and_refusals(olmoe_layer):

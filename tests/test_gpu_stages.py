@@ -12,7 +12,7 @@ import torch
 
 import sparse_moe_transformer_route_b200 as M
 from oracle import moe_oracle as O
-from tests._parity import assert_close, f64, padded_group_starts, require_gpu
+from tests._parity import assert_close, bf16_round, f64, padded_group_starts, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -145,7 +145,7 @@ def test_expert_gemms_match_oracle(counts, dtype, d, f):
     w_down = (torch.randn(E, d, f, generator=g) * 0.05).to(dtype)
     dev = lambda t: t.cuda()
     h = torch.full((P, f), float("nan"), dtype=dtype, device="cuda")
-    pre = torch.full((P, 2 * f), float("nan"), dtype=dtype, device="cuda")
+    pre = torch.full((P, 2 * f), float("nan"), dtype=torch.float32, device="cuda")  # kept unrounded
     o = torch.full((P, d), float("nan"), dtype=dtype, device="cuda")
     gs_t = torch.from_numpy(gs.astype(np.int32)).cuda()
     off_t = torch.from_numpy(off.astype(np.int32)).cuda()
@@ -210,4 +210,8 @@ def test_rmsnorm_matches_oracle():
     out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
     M.moe_rmsnorm(cfg, r.cuda(), w.cuda(), 1e-5, out)
     torch.cuda.synchronize()
-    assert_close(out, O.rms_norm(f64(r), f64(w)), "rmsnorm", max_abs=2e-2, rel_l2=4e-3)
+    # the kernel forms the value in fp64 and rounds it (to fp32, then bf16) as the
+    # oracle's value is rounded here, so the two agree bit for bit (eps is the
+    # fp32 value the call passes)
+    ref = bf16_round(O.rms_norm(f64(r), f64(w), eps=float(np.float32(1e-5))))
+    assert np.array_equal(f64(out), ref)
