@@ -348,6 +348,57 @@ def bench_decode(M, S, dev, weights, reps, peaks):
     return out
 
 
+def bench_decode_stack(M, S, dev, reps, peaks):
+    """The 16-layer skewed stack at decode batch sizes (T = 1 and 6): one
+    persistent launch walks all 16 layers (RMSNorm, routing, experts and the
+    residual add of each). The L2 is flushed before each call; bytes are the
+    touched experts' weights of every layer plus the router weights."""
+    import torch
+    out = {}
+    _, layers = S.stack_inputs(S.LayerShape(T=1), S.STACK_LAYERS, seed=8)
+    layers = [{n: (v.to(dev) if v is not None else None) for n, v in L.items()} for L in layers]
+    E, d = layers[0]["w_router"].shape
+    f = layers[0]["w_down"].shape[2]
+    k = S.OLMOE_TOP_K
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for T in (1, 6):
+        sh = S.LayerShape(T=T)
+        x0 = S.make_tokens(sh, seed=90 + T, dtype=torch.float32, normalised=False).to(dev)
+        cfg = M.config(T, d, E, k, f)
+        ws = M.workspace(cfg, False, dev)
+        resid = torch.empty_like(x0)
+        idx = torch.empty(len(layers), T, k, dtype=torch.int32, device=dev)
+        resid.copy_(x0)
+        M.moe_stack_forward_trace(cfg, layers, resid, ws, topk_idx=idx)
+        torch.cuda.synchronize(dev)
+        touched = [int(torch.unique(idx[l]).numel()) for l in range(len(layers))]
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for i in range(reps + 3):
+            resid.copy_(x0)
+            flush.zero_()
+            if i >= 3:
+                evs[i - 3][0].record()
+            M.moe_stack_forward(cfg, layers, resid, ws)
+            if i >= 3:
+                evs[i - 3][1].record()
+        torch.cuda.synchronize(dev)
+        status = M.moe_get_device_status(ws)
+        if status != 0:
+            raise RuntimeError(f"device check failed in the decode stack: 0x{status:x}")
+        us = [a.elapsed_time(b) * 1e3 for a, b in evs]
+        med, p10, p90 = _percentiles(us)
+        nbytes = sum(t * 3 * d * f * 2 for t in touched) + len(layers) * (E * d * 2 + 2 * T * d * 4)
+        gbs = nbytes / (med * 1e-6) / 1e9
+        out[f"T{T}"] = {
+            "us_median": med, "us_p10": p10, "us_p90": p90, "us_per_layer": med / len(layers),
+            "layers": len(layers), "experts_touched_per_layer": touched, "bytes": nbytes, "GB_per_s": gbs,
+            "frac_of_8TBs": gbs / NOMINAL_HBM_GBS, "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
+            "tokens_per_s": T / (med * 1e-6),
+        }
+    out["timing"] = "CUDA events around one moe_stack_forward (one persistent launch), L2 flushed before each"
+    return out
+
+
 def bench_train(M, S, dev, steps, peaks):
     """One training step at T = 16384: moe_forward (saving for backward) and
     moe_backward, with the OLMoE loss weights, an N(0, 1) upstream gradient and
@@ -639,6 +690,10 @@ def run_b200(args, rank, world, local):
             torch.cuda.empty_cache()
         if "decode" in extras:
             line["decode"] = bench_decode(M, S, dev, (wr, wgu, wd), 200, peaks)
+            torch.cuda.empty_cache()
+        if "decode_stack" in extras:
+            line["decode_stack"] = bench_decode_stack(M, S, dev, 50, peaks)
+            torch.cuda.empty_cache()
         del x, wr, wgu, wd, ws, y
         torch.cuda.empty_cache()
         if "train" in extras:
@@ -669,8 +724,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the expert-choice, decode, training-step and 16-layer stack workloads (N=1 only)")
-    ap.add_argument("--extras", default="ec,decode,train,stack",
-                    help="comma list of the extra workloads to run at N=1 (ec, decode, train, stack)")
+    ap.add_argument("--extras", default="ec,decode,decode_stack,train,stack",
+                    help="comma list of the extra workloads to run at N=1 (ec, decode, decode_stack, train, stack)")
     ap.add_argument("--routing", choices=("token", "expert"), default="token",
                     help="token choice (OLMoE, the benchmarked layer) or expert choice (for profiling)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")

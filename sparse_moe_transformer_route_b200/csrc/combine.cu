@@ -201,10 +201,11 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// The normalised value is formed in fp64 (sum of squares, square root and
-// division), then rounded to fp32 and on to the output type: the same value
-// and the same two roundings as an fp64 evaluation of the formula, so the
-// layer input's rounding is decided as an exact computation would decide it.
+// The normalised value is formed in fp64 (sum of squares, square root, one
+// reciprocal per row and a product per element), then rounded to fp32 and on
+// to the output type: within an ulp of fp64 of an fp64 evaluation of the
+// formula, so the layer input's rounding is decided as an exact computation
+// decides it (short of values within ~1e-16 of a rounding boundary).
 template <typename T_>
 __global__ void __launch_bounds__(256)
     rmsnorm_kernel(const float* __restrict__ resid, const float* __restrict__ weight, double eps, int d,
@@ -226,9 +227,9 @@ __global__ void __launch_bounds__(256)
     red[0] = s;
   }
   __syncthreads();
-  const double den = sqrt(red[0] / static_cast<double>(d) + eps);
+  const double inv = 1.0 / sqrt(red[0] / static_cast<double>(d) + eps);
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    double v = static_cast<double>(r[i]) / den;
+    double v = static_cast<double>(r[i]) * inv;
     if (weight != nullptr) v *= static_cast<double>(weight[i]);
     out[t * d + i] = from_f32<T_>(static_cast<float>(v));
   }

@@ -1,6 +1,9 @@
 // The whole MoE layer for a decode-sized batch (T <= 8 tokens) in one
 // persistent cooperative kernel: router, gate/up + SwiGLU, down and combine,
-// optionally with the block's RMSNorm in front and the residual add behind.
+// optionally with the block's RMSNorm in front and the residual add behind;
+// and a stack of such blocks (up to 16 per launch) in the same kernel, which
+// walks the layers with a grid barrier between one layer's residual update
+// and the next layer's RMSNorm.
 //
 // Method: the layer of "Mixture-of-experts LLMs from scratch with OLMoE",
 // section 2 (softmax over all experts, top-k without renormalisation, each
@@ -54,24 +57,31 @@ constexpr int kDecSlots = kDecMaxT * kMaxTopK;            // (token, slot) pairs
 constexpr size_t kDecActBytes = 160 * 1024;               // staged x, then h
 constexpr size_t kDecMiscBytes = 28 * 1024;
 constexpr size_t kDecSmem = kDecActBytes + kDecMiscBytes;
+constexpr int kDecMaxLayers = 16;                          // layers of a stack per launch
+
+// One layer's weights.
+struct DecLayer {
+  const __nv_bfloat16* wr;   // [E, d]
+  const float* bias;         // [E] or null
+  const __nv_bfloat16* wgu;  // [E, 2f, d]
+  const __nv_bfloat16* wd;   // [E, d, f]
+};
 
 struct DecArgs {
   int T, d, E, k, f;
   int renorm;
   double eps;
+  int n_layers;              // 1, or up to kDecMaxLayers blocks of a stack (with `resid`)
+  DecLayer layer[kDecMaxLayers];
   const __nv_bfloat16* x;    // [T, d] layer input, or null when `resid` is the input
   float* resid;              // [T, d] fp32 residual (in/out), or null
-  const __nv_bfloat16* wr;   // [E, d]
-  const float* bias;         // [E] or null
-  const __nv_bfloat16* wgu;  // [E, 2f, d]
-  const __nv_bfloat16* wd;   // [E, d, f]
   __nv_bfloat16* y;          // [T, d] out (null with `resid`)
   __nv_bfloat16* h;          // [T*k, f] workspace
-  int32_t* idx_out;          // [T, k] or null
-  float* w_out;              // [T, k] or null
-  int32_t* counts;           // [E] or null
-  float* losses;             // [2] or null
-  float* losses_ws;          // [2] workspace copy
+  int32_t* idx_out;          // [n_layers, T, k] or null
+  float* w_out;              // [T, k] or null (single layer)
+  int32_t* counts;           // [n_layers, E] or null
+  float* losses;             // [n_layers, 2] or null
+  float* losses_ws;          // [2] workspace copy (of the last layer)
   unsigned* bar;             // [2] arrival count, generation
   int32_t* status;
 };
@@ -85,10 +95,11 @@ struct DecSmem {
   int touched[kDecMaxE];           // experts chosen by some token, ascending
   int n_touched;
   int ok;
-  double rms[kDecMaxT];             // sqrt(mean square + eps) of each input row
+  double rms[kDecMaxT];             // 1 / sqrt(mean square + eps) of each input row
   double hd[kDecMaxT][kDecMaxE];   // logits (+ offset)
   float p[kDecMaxT][kDecMaxE];
   float lse[kDecMaxT];
+  DecLayer layers[kDecMaxLayers];  // the launch's layer table
 };
 static_assert(sizeof(DecSmem) <= kDecMiscBytes, "decode bookkeeping fits");
 
@@ -149,8 +160,11 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 }
 
 // NT: tokens the phase-1 accumulators are sized for (1, 2, 4 or 8; T <= NT).
-template <int NT>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecArgs a) {
+// STACK: walks a.n_layers layers of a stack; otherwise exactly one layer (a
+// loop whose trip count the compiler knows keeps the kernel free of register
+// spills; the stack's runtime layer loop costs some).
+template <int NT, bool STACK>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __grid_constant__ DecArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __nv_bfloat16* act = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // x [T, d], later h [T*k, f]
   DecSmem& m = *reinterpret_cast<DecSmem*>(smem_raw + kDecActBytes);
@@ -159,6 +173,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
   const int nvd = d / 8, nvf = f / 8;  // 16-byte vectors per row
   const int gw = blockIdx.x * kDecWarps + warp;
   const int nw = gridDim.x * kDecWarps;
+  // the layer table in shared memory (indexed by layer below; kernel parameters
+  // are only read at fixed offsets)
+#pragma unroll
+  for (int l = 0; l < kDecMaxLayers; ++l)
+    if (tid == l) m.layers[l] = a.layer[l];
+  __syncthreads();
+
+  const int n_layers = STACK ? a.n_layers : 1;
+#pragma unroll 1
+  for (int l = 0; l < n_layers; ++l) {
+  // a layer of a stack reads the residual the previous layer completed
+  if (l > 0 && !grid_barrier(a.bar, gridDim.x, a.status, &m.ok)) return;
+  const DecLayer Ly = m.layers[l];
+  int32_t* const idx_out = a.idx_out != nullptr ? a.idx_out + static_cast<int64_t>(l) * T * k : nullptr;
+  int32_t* const counts = a.counts != nullptr ? a.counts + static_cast<int64_t>(l) * E : nullptr;
+  float* const losses = a.losses != nullptr ? a.losses + 2 * l : nullptr;
 
   // ---- prologue: the T input rows, bf16, in shared memory
   if (a.resid != nullptr) {
@@ -167,13 +197,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
       double ss = 0.0;
       for (int i = lane; i < d; i += 32) ss = fma(static_cast<double>(r[i]), static_cast<double>(r[i]), ss);
       ss = warp_sum_d(ss);
-      if (lane == 0) m.rms[warp] = sqrt(ss / static_cast<double>(d) + a.eps);
+      if (lane == 0) m.rms[warp] = 1.0 / sqrt(ss / static_cast<double>(d) + a.eps);
       __syncwarp();
     }
     __syncthreads();
     // the fp64 value rounded to fp32, then to bf16 (as the separate RMSNorm kernel does)
     for (int i = tid; i < T * d; i += kDecThreads)
-      act[i] = __float2bfloat16_rn(static_cast<float>(static_cast<double>(a.resid[i]) / m.rms[i / d]));
+      act[i] = __float2bfloat16_rn(static_cast<float>(static_cast<double>(a.resid[i]) * m.rms[i / d]));
   } else {
     const uint4* src = reinterpret_cast<const uint4*>(a.x);
     uint4* dst = reinterpret_cast<uint4*>(act);
@@ -189,7 +219,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
   //      summed in fp32 here; every CTA sums in the same order, so every CTA
   //      holds the same values and takes the same decisions.
   for (int e = warp; e < E; e += kDecWarps) {
-    const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<int64_t>(e) * d);
+    const uint4* wrow = reinterpret_cast<const uint4*>(Ly.wr + static_cast<int64_t>(e) * d);
     float acc[NT];
 #pragma unroll
     for (int q = 0; q < NT; ++q) acc[q] = 0.f;
@@ -222,7 +252,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
     for (int q = 0; q < NT; ++q) {
       if (q < T) {
         const float h = warp_sum(acc[q]);
-        if (lane == 0) m.hd[q][e] = static_cast<double>(h) + (a.bias != nullptr ? static_cast<double>(a.bias[e]) : 0.0);
+        if (lane == 0) m.hd[q][e] = static_cast<double>(h) + (Ly.bias != nullptr ? static_cast<double>(Ly.bias[e]) : 0.0);
       }
     }
   }
@@ -257,7 +287,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
       for (int u = 0; u < 2; ++u) {
         const int e = lane + 32 * u;
         if (e < E) {
-          const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<int64_t>(e) * d);
+          const uint4* wrow = reinterpret_cast<const uint4*>(Ly.wr + static_cast<int64_t>(e) * d);
           double acc = 0.0;
           for (int v = 0; v < nvd; ++v) {
             float xv[8], wv[8];
@@ -266,7 +296,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc += static_cast<double>(xv[i] * wv[i]);  // exact product
           }
-          ex[u] = acc + (a.bias != nullptr ? static_cast<double>(a.bias[e]) : 0.0);
+          ex[u] = acc + (Ly.bias != nullptr ? static_cast<double>(Ly.bias[e]) : 0.0);
         }
       }
       __syncwarp();
@@ -323,7 +353,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
         const float w = a.renorm ? m.p[t][e] / den : m.p[t][e];
         m.sel_w[t * k + j] = w;
         if (blockIdx.x == 0) {
-          if (a.idx_out != nullptr) a.idx_out[t * k + j] = e;
+          if (idx_out != nullptr) idx_out[t * k + j] = e;
           if (a.w_out != nullptr) a.w_out[t * k + j] = w;
         }
       }
@@ -345,7 +375,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
         double pe = 0.0;
         for (int t = 0; t < T; ++t) pe += m.p[t][e];
         lb += static_cast<double>(ce) * pe;
-        if (a.counts != nullptr) a.counts[e] = ce;
+        if (counts != nullptr) counts[e] = ce;
       }
     }
     if (lane == 0) m.n_touched = base;
@@ -358,9 +388,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
         const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(z / Td);
         a.losses_ws[0] = l0;
         a.losses_ws[1] = l1;
-        if (a.losses != nullptr) {
-          a.losses[0] = l0;
-          a.losses[1] = l1;
+        if (losses != nullptr) {
+          losses[0] = l0;
+          losses[1] = l1;
         }
       }
     }
@@ -375,7 +405,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
     const int u = item / f, i = item - u * f;
     const int e = m.touched[u];
     const unsigned tmask = m.tokmask[e];
-    const uint4* grow = reinterpret_cast<const uint4*>(a.wgu + (static_cast<int64_t>(e) * 2 * f + i) * d);
+    const uint4* grow = reinterpret_cast<const uint4*>(Ly.wgu + (static_cast<int64_t>(e) * 2 * f + i) * d);
     const uint4* urow = grow + static_cast<int64_t>(f) * nvd;
     float ag[NT], au[NT];
 #pragma unroll
@@ -440,7 +470,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
         for (int uu = 0; uu < 4; ++uu) {
           if (u0 + uu < nt) {
             const uint4* row =
-                reinterpret_cast<const uint4*>(a.wd + (static_cast<int64_t>(m.touched[u0 + uu]) * d + c) * f);
+                reinterpret_cast<const uint4*>(Ly.wd + (static_cast<int64_t>(m.touched[u0 + uu]) * d + c) * f);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int v = v0 + j * 32 + lane;
@@ -489,6 +519,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const DecA
     }
     __syncwarp();
   }
+  }  // layers
 }
 
 }  // namespace
@@ -499,20 +530,24 @@ bool decode_supported(const Shape& s) {
   return x_bytes <= kDecActBytes && h_bytes <= kDecActBytes;
 }
 
-cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, double eps, const void* w_router,
-                                const float* bias, const void* w_gate_up, const void* w_down, void* y,
-                                int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,
-                                const Workspace& L, cudaStream_t st) {
+namespace {
+// One cooperative launch over `n` (<= kDecMaxLayers) layers.
+cudaError_t launch_decode(const Shape& s, const void* x, float* resid, double eps, int n,
+                          const void* const* w_router, const float* const* biases, const void* const* w_gate_up,
+                          const void* const* w_down, void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                          float* losses, void* ws, const Workspace& L, cudaStream_t st) {
   // the accumulator count follows the batch: fewer live registers for small T
   // keep more of each warp's row loads in flight
-  static std::atomic<size_t> set_smem[4][kMaxDevices];
-  void (*kern)(DecArgs) = s.T <= 1 ? decode_layer_kernel<1>
-                          : s.T <= 2 ? decode_layer_kernel<2>
-                          : s.T <= 4 ? decode_layer_kernel<4>
-                                     : decode_layer_kernel<8>;
-  const int which = s.T <= 1 ? 0 : s.T <= 2 ? 1 : s.T <= 4 ? 2 : 3;
+  static std::atomic<size_t> set_smem[8][kMaxDevices];
+  const bool stack = n > 1;
+  void (*kern)(DecArgs) = s.T <= 1 ? (stack ? decode_layer_kernel<1, true> : decode_layer_kernel<1, false>)
+                          : s.T <= 2 ? (stack ? decode_layer_kernel<2, true> : decode_layer_kernel<2, false>)
+                          : s.T <= 4 ? (stack ? decode_layer_kernel<4, true> : decode_layer_kernel<4, false>)
+                                     : (stack ? decode_layer_kernel<8, true> : decode_layer_kernel<8, false>);
+  const int which = (s.T <= 1 ? 0 : s.T <= 2 ? 1 : s.T <= 4 ? 2 : 3) + (stack ? 4 : 0);
   cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(kern), kDecSmem, set_smem[which]);
   if (e != cudaSuccess) return e;
+  if (n < 1 || n > kDecMaxLayers) return cudaErrorInvalidValue;
   DecArgs a{};
   a.T = static_cast<int>(s.T);
   a.d = s.d;
@@ -521,12 +556,15 @@ cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, dou
   a.f = s.f;
   a.renorm = s.renorm ? 1 : 0;
   a.eps = eps;
+  a.n_layers = n;
+  for (int l = 0; l < n; ++l) {
+    a.layer[l].wr = static_cast<const __nv_bfloat16*>(w_router[l]);
+    a.layer[l].bias = biases != nullptr ? biases[l] : nullptr;
+    a.layer[l].wgu = static_cast<const __nv_bfloat16*>(w_gate_up[l]);
+    a.layer[l].wd = static_cast<const __nv_bfloat16*>(w_down[l]);
+  }
   a.x = static_cast<const __nv_bfloat16*>(x);
   a.resid = resid;
-  a.wr = static_cast<const __nv_bfloat16*>(w_router);
-  a.bias = bias;
-  a.wgu = static_cast<const __nv_bfloat16*>(w_gate_up);
-  a.wd = static_cast<const __nv_bfloat16*>(w_down);
   a.y = static_cast<__nv_bfloat16*>(y);
   a.h = at<__nv_bfloat16>(ws, L.h);
   a.idx_out = topk_idx;
@@ -547,6 +585,31 @@ cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, dou
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
+}
+}  // namespace
+
+cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, double eps, const void* w_router,
+                                const float* bias, const void* w_gate_up, const void* w_down, void* y,
+                                int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,
+                                const Workspace& L, cudaStream_t st) {
+  return launch_decode(s, x, resid, eps, 1, &w_router, &bias, &w_gate_up, &w_down, y, topk_idx, topk_w, counts, losses,
+                       ws, L, st);
+}
+
+cudaError_t launch_decode_stack(const Shape& s, float* resid, double eps, int n_layers, const void* const* w_router,
+                                const float* const* biases, const void* const* w_gate_up, const void* const* w_down,
+                                int32_t* topk_idx, int32_t* counts, float* losses, void* ws, const Workspace& L,
+                                cudaStream_t st) {
+  for (int l0 = 0; l0 < n_layers; l0 += kDecMaxLayers) {
+    const int n = n_layers - l0 < kDecMaxLayers ? n_layers - l0 : kDecMaxLayers;
+    const cudaError_t e = launch_decode(
+        s, nullptr, resid, eps, n, w_router + l0, biases != nullptr ? biases + l0 : nullptr, w_gate_up + l0,
+        w_down + l0, nullptr, topk_idx != nullptr ? topk_idx + static_cast<int64_t>(l0) * s.T * s.k : nullptr,
+        nullptr, counts != nullptr ? counts + static_cast<int64_t>(l0) * s.E : nullptr,
+        losses != nullptr ? losses + 2 * l0 : nullptr, ws, L, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace moe

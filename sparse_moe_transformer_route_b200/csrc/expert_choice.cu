@@ -13,13 +13,20 @@
 // order and is zero when no expert took it.
 //
 // Kernels:
-//   ec_select_kernel   one CTA per expert: an exact radix select (four 8-bit
-//                      passes over the fp32 bit patterns, which order like the
-//                      values since p >= 0) finds the C-th largest p[:, e] and
-//                      how many of the tokens equal to it fit; then one pass in
-//                      token order writes the chosen tokens, their weights, and
-//                      for every token its row in the expert's group (or -1).
-//                      One more CTA sums the z-loss and writes the group table.
+//   ec_select_kernel   one CTA per expert: a radix select (four 8-bit passes
+//                      over the fp32 bit patterns, which order like the values
+//                      since p >= 0) finds the C-th largest fp32 p[:, e]. Tokens
+//                      whose fp32 p lies within 4e-4 (relative) of it, a band
+//                      wider than any error of the fp32 probabilities (the
+//                      token-choice router's 2e-4 bound on each logit, twice),
+//                      are then ranked by their exact key h[t, e] - lse_t, the
+//                      logits summed in fp64 from exact bf16 products (equal
+//                      keys: the lower token index), and the ones above the
+//                      band are taken outright; so the choice is the one an
+//                      exact computation makes. One pass in token order then
+//                      writes the chosen tokens, their weights, and for every
+//                      token its row in the expert's group (or -1). One more
+//                      CTA sums the z-loss and writes the group table.
 //   ec_gather_kernel   x_perm[group_start[e] + i] = x[sel[e, i]], a warp per row.
 // The expert GEMMs are the token-choice ones (every group holds C rows), and
 // the combine is combine_ec_kernel in combine.cu.
@@ -35,9 +42,17 @@ constexpr int kEcWarps = kEcThreads / 32;
 // ones are read from the probabilities in L2 on every pass.
 constexpr int64_t kEcSmemTokens = 40960;
 
+// Tokens near the C-th value that one CTA re-ranks exactly; more (only when
+// that many probabilities tie within the band) fall back to the fp32 order.
+constexpr int kEcMaxCand = 256;
+
 struct EcArgs {
   const float* probs;  // [T, E]
   const float* lse;    // [T]
+  const __nv_bfloat16* x;   // [T, d] tokens (for the exact keys)
+  const __nv_bfloat16* wr;  // [E, d] router weight
+  const float* bias;        // [E] or null
+  int d;
   int64_t T;
   int E, C, Cpad;
   int32_t* sel;          // [E, C] chosen tokens, ascending
@@ -78,9 +93,52 @@ __device__ __forceinline__ int block_warp_scan(int* cnt, int* tot_s, int warp, i
   return cnt[warp];
 }
 
+// The exact logit <x_t, W_r[ee]> (+ bias) by one warp: lane l takes 8-element
+// pieces l, l + 32, ... (coalesced), every load in flight before the
+// arithmetic, exact bf16 products summed in fp64, then a fixed shuffle tree.
+__device__ __forceinline__ double exact_logit(const EcArgs& a, int64_t t, int ee, int lane) {
+  constexpr int kPieces = 4;  // 16-byte pieces per lane in flight (a 1024-thread CTA has 64 registers)
+  const uint4* xrow = reinterpret_cast<const uint4*>(a.x + t * a.d);
+  const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<int64_t>(ee) * a.d);
+  const int nv = a.d / 8;
+  double acc = 0.0;
+  for (int v0 = 0; v0 < nv; v0 += 32 * kPieces) {
+    uint4 xq[kPieces], wq[kPieces];
+#pragma unroll
+    for (int j = 0; j < kPieces; ++j) {
+      const int v = v0 + lane + 32 * j;
+      if (v < nv) {
+        xq[j] = __ldg(xrow + v);
+        wq[j] = __ldg(wrow + v);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kPieces; ++j) {
+      if (v0 + lane + 32 * j < nv) {
+        const uint32_t xa[4] = {xq[j].x, xq[j].y, xq[j].z, xq[j].w}, wa[4] = {wq[j].x, wq[j].y, wq[j].z, wq[j].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xa[c]));
+          const float2 wf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[c]));
+          acc += static_cast<double>(xf.x * wf.x);  // exact products
+          acc += static_cast<double>(xf.y * wf.y);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc + (a.bias != nullptr ? static_cast<double>(a.bias[ee]) : 0.0);
+}
+
 __global__ void __launch_bounds__(kEcThreads, 1) ec_select_kernel(const EcArgs a) {
   extern __shared__ uint32_t keys_s[];  // [min(T, kEcSmemTokens)]
   __shared__ int hist[256];
+  __shared__ int64_t cand_t[kEcMaxCand];
+  __shared__ double cand_x[kEcMaxCand];
+  __shared__ unsigned char cand_take[kEcMaxCand];
+  __shared__ double cand_h[kMaxExperts];
+  __shared__ int s_ncand, s_nhi;
   __shared__ int wcnt[kEcWarps];
   __shared__ int s_tot;
   __shared__ int s_digit, s_above;
@@ -180,7 +238,63 @@ __global__ void __launch_bounds__(kEcThreads, 1) ec_select_kernel(const EcArgs a
     pmask |= 255u << shift;
     __syncthreads();
   }
-  const uint32_t kstar = prefix;  // the C-th largest key; `need` of its equals are taken
+  const uint32_t kstar = prefix;  // the C-th largest fp32 key; `need` of its equals are taken
+
+  // ---- exact decision inside the band [lo, hi] around the C-th value
+  const float vstar = __uint_as_float(kstar);
+  const uint32_t lo_key = __float_as_uint(vstar * (1.0f - 4e-4f));
+  const uint32_t hi_key = __float_as_uint(vstar * (1.0f + 4e-4f));
+  if (tid == 0) {
+    s_ncand = 0;
+    s_nhi = 0;
+  }
+  __syncthreads();
+  {
+    int nhi = 0;
+    for (int64_t t = tid; t < T; t += kEcThreads) {
+      const uint32_t k = key(t);
+      if (k > hi_key) {
+        ++nhi;
+      } else if (k >= lo_key) {
+        const int slot = atomicAdd(&s_ncand, 1);
+        if (slot < kEcMaxCand) cand_t[slot] = t;
+      }
+    }
+    atomicAdd(&s_nhi, nhi);
+  }
+  __syncthreads();
+  const int ncand = s_ncand;
+  const bool exact = ncand <= kEcMaxCand;  // else: the fp32 order decides (many equal values)
+  if (exact) {
+    // each candidate's exact key h[t, e] - lse_t: its E exact logits by the
+    // CTA's warps, then lse in fp64 (max, sum of exponentials, in expert order)
+    for (int i = 0; i < ncand; ++i) {
+      for (int ee = warp; ee < E; ee += kEcWarps) {
+        const double hv = exact_logit(a, cand_t[i], ee, lane);
+        if (lane == 0) cand_h[ee] = hv;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const double h0 = lane < E ? cand_h[lane] : -INFINITY, h1 = lane + 32 < E ? cand_h[lane + 32] : -INFINITY;
+        double mx = fmax(h0, h1);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        double sum = (lane < E ? exp(h0 - mx) : 0.0) + (lane + 32 < E ? exp(h1 - mx) : 0.0);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) cand_x[i] = cand_h[e] - (mx + log(sum));
+      }
+      __syncthreads();
+    }
+    const int need_c = a.C - s_nhi;  // taken from the band
+    for (int i = tid; i < ncand; i += kEcThreads) {
+      int rank = 0;
+      for (int j = 0; j < ncand; ++j)
+        rank += (cand_x[j] > cand_x[i] || (cand_x[j] == cand_x[i] && cand_t[j] < cand_t[i])) ? 1 : 0;
+      cand_take[i] = rank < need_c ? 1 : 0;
+    }
+    __syncthreads();
+  }
 
   // ---- one pass in token order: ranks among the equals, then positions
   const int gs_e = e * a.Cpad;
@@ -189,8 +303,16 @@ __global__ void __launch_bounds__(kEcThreads, 1) ec_select_kernel(const EcArgs a
     const int64_t t = c0 + tid;
     const bool valid = t < T;
     const uint32_t k = valid ? key(t) : 0u;
-    const bool gt = valid && k > kstar;
-    const bool eq = valid && k == kstar;
+    bool gt = valid && k > kstar;
+    bool eq = valid && k == kstar;
+    if (exact) {  // above the band: taken; inside it: the exact decision; below: not
+      bool tk = valid && k > hi_key;
+      if (valid && k >= lo_key && k <= hi_key)
+        for (int i = 0; i < ncand; ++i)
+          if (cand_t[i] == t) tk = cand_take[i] != 0;
+      gt = tk;
+      eq = false;
+    }
     const unsigned beq = __ballot_sync(0xffffffffu, eq);
     if (lane == 0) wcnt[warp] = __popc(beq);
     int eq_tot;
@@ -263,11 +385,15 @@ bool ec_capacity_ok(const Shape& s, int64_t C) {
   return static_cast<int64_t>(s.E) * cpad <= s.P;
 }
 
-cudaError_t launch_ec_select(const Shape& s, int64_t C, int32_t* counts, float* losses, void* ws, const Workspace& L,
-                             cudaStream_t st) {
+cudaError_t launch_ec_select(const Shape& s, int64_t C, const void* x, const void* w_router, const float* bias,
+                             int32_t* counts, float* losses, void* ws, const Workspace& L, cudaStream_t st) {
   EcArgs a{};
   a.probs = at<float>(ws, L.probs);
   a.lse = at<float>(ws, L.lse);
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.wr = static_cast<const __nv_bfloat16*>(w_router);
+  a.bias = bias;
+  a.d = s.d;
   a.T = s.T;
   a.E = s.E;
   a.C = static_cast<int>(C);

@@ -78,7 +78,9 @@ struct Cfg {
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   // Each epilogue warp stages a 32 x 32 output chunk in shared memory (rows
   // padded by 16 bytes against bank conflicts) and writes it back as whole rows.
-  static constexpr int STG_PITCH = 32 * static_cast<int>(sizeof(OutT)) + 16;
+  // staging rows sized for the operand type (fp32 output of bf16 operands
+  // leaves in two passes), so fp32 output costs no ring stage
+  static constexpr int STG_PITCH = 32 * static_cast<int>(sizeof(T)) + 16;
   static constexpr int STG_WARP_BYTES = 32 * STG_PITCH;
   static constexpr int STG_BYTES = EPI_WARPS * STG_WARP_BYTES;
   static constexpr int MISC_BYTES = 1024 + 3 * (kMaxExperts + 1) * static_cast<int>(sizeof(int32_t));
@@ -249,38 +251,47 @@ __device__ __forceinline__ void load16(const T* src, float (&v)[16]) {
 // in v: the rows go to shared memory first, then leave as whole rows (each
 // store instruction covers several complete rows), instead of 32 scattered
 // 16-byte pieces per instruction. `g` points at (the warp's first row, the
-// chunk's first column); `ld` is the row stride in elements.
+// chunk's first column); `ld` is the row stride in elements. A staging row of
+// PITCH bytes holds up to (PITCH - 16) bytes of values; wider rows (fp32 output
+// through a buffer sized for bf16) go out in two passes of 16 columns.
 template <typename T, int PITCH>
 __device__ __forceinline__ void warp_store_chunk(unsigned char* stg, const float (&v)[32], T* g, int64_t ld,
                                                  int lane) {
-  constexpr int RB = 32 * static_cast<int>(sizeof(T));  // bytes of one row of the chunk
-  constexpr int LPR = RB / 16;                           // lanes per row on the way out
-  constexpr int RPI = 32 / LPR;                          // rows per store instruction
+  constexpr int CPP = ((PITCH - 16) / static_cast<int>(sizeof(T))) < 32 ? 16 : 32;  // columns per pass
+  constexpr int RB = CPP * static_cast<int>(sizeof(T));  // bytes of one row of a pass
+  constexpr int LPR = RB / 16;                            // lanes per row on the way out
+  constexpr int RPI = 32 / LPR;                           // rows per store instruction
+  static_assert(RB + 16 <= PITCH || CPP == 16, "staging row");
   unsigned char* mine = stg + lane * PITCH;
-  if constexpr (std::is_same_v<T, float>) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      *reinterpret_cast<float4*>(mine + 16 * i) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-  } else {
+  for (int p = 0; p < 32 / CPP; ++p) {
+    if constexpr (std::is_same_v<T, float>) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint4 w;
-      w.x = pack_bf16x2(v[8 * i], v[8 * i + 1]);
-      w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
-      w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
-      w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
-      *reinterpret_cast<uint4*>(mine + 16 * i) = w;
+      for (int i = 0; i < CPP / 4; ++i)
+        *reinterpret_cast<float4*>(mine + 16 * i) =
+            make_float4(v[p * CPP + 4 * i], v[p * CPP + 4 * i + 1], v[p * CPP + 4 * i + 2], v[p * CPP + 4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < CPP / 8; ++i) {
+        const int b = p * CPP + 8 * i;
+        uint4 w;
+        w.x = pack_bf16x2(v[b], v[b + 1]);
+        w.y = pack_bf16x2(v[b + 2], v[b + 3]);
+        w.z = pack_bf16x2(v[b + 4], v[b + 5]);
+        w.w = pack_bf16x2(v[b + 6], v[b + 7]);
+        *reinterpret_cast<uint4*>(mine + 16 * i) = w;
+      }
     }
-  }
-  __syncwarp();
+    __syncwarp();
 #pragma unroll
-  for (int it = 0; it < 32 / RPI; ++it) {
-    const int r = it * RPI + lane / LPR;
-    const int seg = lane % LPR;
-    const uint4 val = *reinterpret_cast<const uint4*>(stg + r * PITCH + seg * 16);
-    *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(g + r * ld) + seg * 16) = val;
+    for (int it = 0; it < 32 / RPI; ++it) {
+      const int r = it * RPI + lane / LPR;
+      const int seg = lane % LPR;
+      const uint4 val = *reinterpret_cast<const uint4*>(stg + r * PITCH + seg * 16);
+      *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(g + r * ld + p * CPP) + seg * 16) = val;
+    }
+    __syncwarp();
   }
-  __syncwarp();
 }
 
 // -------------------------------------------------------------- the kernel
@@ -656,7 +667,7 @@ struct PairCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int STG_PITCH = 32 * static_cast<int>(sizeof(OutT)) + 16;
+  static constexpr int STG_PITCH = 32 * 2 + 16;  // bf16-sized rows; fp32 output leaves in two passes
   static constexpr int STG_WARP_BYTES = 32 * STG_PITCH;
   static constexpr int STG_BYTES = EPI_WARPS * STG_WARP_BYTES;
   static constexpr int MISC_BYTES = 1024 + 3 * (kMaxExperts + 1) * static_cast<int>(sizeof(int32_t));

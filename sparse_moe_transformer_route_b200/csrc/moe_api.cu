@@ -480,7 +480,7 @@ moe_status moe_route_expert_choice(const moe_config* cfg, int64_t capacity, cons
       !aligned16(w_router))
     return MOE_ERR_INVALID_ARG;
   MOE_TRY(launch_router_probs(c.s, x, w_router, router_bias, ws, c.L, stream));
-  MOE_TRY(launch_ec_select(c.s, C, counts, losses, ws, c.L, stream));
+  MOE_TRY(launch_ec_select(c.s, C, x, w_router, router_bias, counts, losses, ws, c.L, stream));
   const size_t n = static_cast<size_t>(c.s.E) * static_cast<size_t>(C);
   MOE_TRY(cudaMemcpyAsync(sel, at<int32_t>(ws, c.L.ec_sel), n * 4, cudaMemcpyDeviceToDevice, stream));
   MOE_TRY(cudaMemcpyAsync(gates, at<float>(ws, c.L.ec_gate), n * 4, cudaMemcpyDeviceToDevice, stream));
@@ -511,7 +511,7 @@ moe_status moe_forward_expert_choice(const moe_config* cfg, int64_t capacity, co
   MOE_TRY(marks.mark(0));
   MOE_TRY(launch_router_probs(s, x, w_router, router_bias, ws, L, stream));
   MOE_TRY(marks.mark(1));
-  MOE_TRY(launch_ec_select(s, C, nullptr, losses, ws, L, stream));
+  MOE_TRY(launch_ec_select(s, C, x, w_router, router_bias, nullptr, losses, ws, L, stream));
   MOE_TRY(launch_ec_gather(s, C, x, ws, L, stream));
   MOE_TRY(marks.mark(2));
   MOE_TRY(launch_gate_up(s, x_perm, gs, off, w_gate_up, at<void>(ws, L.h), nullptr, status, stream));
@@ -553,14 +553,10 @@ moe_status moe_stack_forward_trace(const moe_config* cfg, int32_t n_layers, cons
     if (w_router[l] == nullptr || w_gate_up[l] == nullptr || w_down[l] == nullptr) return MOE_ERR_INVALID_ARG;
   void* xn = at<void>(ws, c.L.x_dev);
   const int64_t tk = c.s.T * c.s.k;
-  if (c.s.T <= kDecodeAutoTokens && decode_supported(c.s)) {  // RMSNorm, layer and residual add in one kernel
-    for (int l = 0; l < n_layers; ++l) {
-      const float* bias = (router_biases != nullptr) ? router_biases[l] : nullptr;
-      MOE_TRY(launch_decode_layer(c.s, nullptr, resid, kStackRmsEps, w_router[l], bias, w_gate_up[l], w_down[l], nullptr,
-                                  topk_idx != nullptr ? topk_idx + l * tk : nullptr, nullptr,
-                                  counts != nullptr ? counts + static_cast<int64_t>(l) * c.s.E : nullptr,
-                                  losses != nullptr ? losses + 2 * l : nullptr, ws, c.L, stream));
-    }
+  if (c.s.T <= kDecodeAutoTokens && decode_supported(c.s)) {
+    // the whole stack in one persistent kernel (RMSNorm, layer and residual add of every layer)
+    MOE_TRY(launch_decode_stack(c.s, resid, kStackRmsEps, n_layers, w_router, router_biases, w_gate_up, w_down, topk_idx,
+                                counts, losses, ws, c.L, stream));
     return MOE_OK;
   }
   for (int l = 0; l < n_layers; ++l) {

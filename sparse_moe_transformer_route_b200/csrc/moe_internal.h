@@ -92,8 +92,9 @@ cudaError_t launch_router_probs(const Shape& s, const void* x, const void* w_rou
                                 const Workspace& L, cudaStream_t st);
 int64_t ec_default_capacity(const Shape& s);
 bool ec_capacity_ok(const Shape& s, int64_t C);
-cudaError_t launch_ec_select(const Shape& s, int64_t C, int32_t* counts, float* losses, void* ws, const Workspace& L,
-                             cudaStream_t st);
+// x, w_router, bias: the router's inputs, for the exact re-ranking near the C-th value
+cudaError_t launch_ec_select(const Shape& s, int64_t C, const void* x, const void* w_router, const float* bias,
+                             int32_t* counts, float* losses, void* ws, const Workspace& L, cudaStream_t st);
 cudaError_t launch_ec_gather(const Shape& s, int64_t C, const void* x, void* ws, const Workspace& L,
                              cudaStream_t st);
 cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t* slot_row, const float* probs,
@@ -114,6 +115,12 @@ cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, dou
                                 const Workspace& L, cudaStream_t st);
 // RMSNorm of the fp32 residual, evaluated in fp64 and rounded once to fp32
 // and then to the layer dtype.
+// A stack of n_layers decode blocks, resid <- resid + MoE_l(RMSNorm(resid)),
+// in one launch per 16 layers (per-layer outputs may be null).
+cudaError_t launch_decode_stack(const Shape& s, float* resid, double eps, int n_layers, const void* const* w_router,
+                                const float* const* biases, const void* const* w_gate_up, const void* const* w_down,
+                                int32_t* topk_idx, int32_t* counts, float* losses, void* ws, const Workspace& L,
+                                cudaStream_t st);
 cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, double eps, void* out,
                            cudaStream_t st);
 // eps of the stack's pre-norm ("Mixture-of-experts LLMs from scratch with OLMoE",

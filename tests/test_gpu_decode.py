@@ -156,3 +156,28 @@ def test_deterministic_and_refusals(olmoe_layer):
     with pytest.raises(M.MoeError) as e:
         _decode(big, S.make_tokens(big, seed=801), *olmoe_layer)
     assert e.value.status == 2
+
+
+@pytest.fixture(scope="module")
+def olmoe_stack_weights():
+    """Sixteen OLMoE-shape layers (the skewed stack's weights and Zipf offset)."""
+    _, layers = S.stack_inputs(S.LayerShape(T=1), S.STACK_LAYERS, seed=8)
+    return layers
+
+
+@pytest.mark.parametrize("T", [1, 6])
+def test_sixteen_layer_decode_stack_in_one_launch(olmoe_stack_weights, T):
+    """The whole 16-layer stack of decode blocks as one persistent launch: every
+    layer on the oracle's residual at its depth, and the one-launch stack equal
+    bit for bit to its sixteen single-layer launches."""
+    sh = S.LayerShape(T=T)
+    x0 = S.make_tokens(sh, seed=90 + T, dtype=torch.float32, normalised=False)
+    layers = olmoe_stack_weights
+    _check_stack_per_layer(sh, x0, layers)
+    one, tr = _gpu_stack_layers(sh, x0, layers)
+    r = x0
+    for L in layers:
+        r, _ = _gpu_stack_layers(sh, r, [L], trace=False)
+    assert torch.equal(one, r)
+    for l in range(len(layers)):
+        assert np.array_equal(np.bincount(tr["idx"][l].reshape(-1), minlength=sh.n_experts), tr["counts"][l])

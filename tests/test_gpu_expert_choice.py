@@ -2,13 +2,10 @@
 
 Each expert keeps the C tokens with the largest router probability for it
 ("OLMoE: Open Mixture-of-Experts Language Models", section 4.1.4, read as the
-oracle's module notes state). The choice is an order statistic of floating-
-point values, so it is checked two ways:
-  * bit-exact: the kernel's chosen tokens equal the oracle's expert_choice run
-    on the kernel's own fp32 probabilities (the decision taken in the kernel's
-    precision on both sides, ties to the lower token index included);
-  * against the oracle's fp64 probabilities: a token chosen by one side only
-    must sit within 1e-5 (relative) of the expert's C-th value.
+oracle's module notes state). The kernel re-ranks the tokens near each
+expert's C-th value by exact keys, so its choice is compared directly with the
+oracle's choice on fp64 probabilities: a token chosen by one side only must
+sit within 1e-6 (relative) of the expert's C-th value (a near-tie, counted).
 The probabilities themselves, the z-loss and the layer output are compared with
 the oracle at the usual bars.
 """
@@ -24,7 +21,7 @@ from tests._parity import LazyF64, assert_close, assert_loss_close, f64, require
 
 pytestmark = pytest.mark.gpu
 
-BOUNDARY_REL = 1e-5
+BOUNDARY_REL = 1e-6
 
 
 @pytest.fixture(autouse=True, scope="module")
@@ -78,14 +75,11 @@ def _check_routing(inp, r):
         assert C == O.ec_capacity(inp.shape.T, inp.shape.top_k, E)
     # probabilities (fp32 from fp32 tensor-core logits)
     assert_close(r["probs"], p, "probabilities", max_abs=1e-5, rel_l2=1e-5)
-    # the decision in the kernel's precision: bit-exact, ties included
+    # the weights are the kernel's probabilities of its chosen tokens, bit for bit
     kp = f64(r["probs"])
-    ref_sel, _ = O.expert_choice(kp, C)
-    assert np.array_equal(r["sel"], ref_sel), "selection differs from the oracle's on the kernel's probabilities"
-    # weights are the kernel's probabilities of the chosen tokens, bit for bit
     want = torch.from_numpy(np.take_along_axis(kp.T, r["sel"].astype(np.int64), axis=1)).float()
     assert torch.equal(r["gates"], want)
-    # against fp64: only boundary tokens may differ
+    # the choice against the oracle's on fp64 probabilities: only near-ties may differ
     sel64, _ = O.expert_choice(p, C)
     n_boundary = 0
     for e in range(E):
@@ -191,6 +185,24 @@ def test_exact_ties_go_to_the_lower_token():
             assert r["sel"][e].tolist() == [best, best + 4, best + 8, best + 12]
     out = _forward(inp)
     _check_output(inp, out, p)
+
+
+def test_exact_ties_across_router_tiles_go_to_the_lower_token():
+    """Repeated rows spread over four 32-token router tiles: their fp32
+    probabilities may differ in the last bits between tiles, but their exact
+    keys are equal, so each expert takes the lowest-index copies of its best
+    row (32 copies, C = 16 of them: the first 16)."""
+    sh = S.LayerShape(T=128, d_model=256, n_experts=16, top_k=2, d_ff=128)
+    inp = S.layer_inputs(sh, seed=48)
+    inp.x = inp.x[:4].clone().repeat(32, 1)
+    r = _route(inp)
+    assert r["C"] == 16
+    p, _ = _check_routing(inp, r)
+    for e in range(sh.n_experts):
+        vals = p[:4, e]
+        best = int(np.argmax(vals))
+        if np.sum(vals == vals[best]) == 1:
+            assert r["sel"][e].tolist() == [best + 4 * i for i in range(16)]
 
 
 @pytest.mark.parametrize("capacity", [1, 37, 200])
