@@ -660,10 +660,12 @@ struct PairCfg {
   static constexpr int UK = 16;                    // K per UMMA
   static constexpr int KSTEPS = BK / UK;
   static constexpr int A_BYTES = 128 * 128;        // this CTA's 128 rows of A
+  static constexpr int A_TAIL_BYTES = 64 * 128;    // its 64 rows of A in a tail tile
   static constexpr int B_BYTES = 128 * 128;        // this CTA's 128 rows of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int ACC_BUFS = 2;
   static constexpr uint32_t IDESC = make_idesc(false, false, false, 256, BN);
+  static constexpr uint32_t IDESC_TAIL = make_idesc(false, false, false, 128, BN);  // 64 rows per CTA
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
@@ -679,14 +681,22 @@ struct PairCfg {
   static_assert(EP == Epi::SwigluFwd || EP == Epi::Store, "forward epilogues");
 };
 
+// A tile is 256 rows (128 per CTA, M = 256 MMAs), except an expert group's
+// last tile when only 128 of its rows remain: that tail tile is 128 rows (64
+// per CTA, M = 128 MMAs), so no MMA work is spent on the next group's rows.
+// In an M = 128 pair MMA each CTA's accumulator holds its 64 rows twice over:
+// TMEM lanes 0..63 carry output columns 0..127 and lanes 64..127 columns
+// 128..255, both at TMEM columns 0..127 (lane 64 + r is row r again; checked
+// on B200 by passing each row's and column's index through the MMA).
 struct PairTile {
   int e, m0, n0;
-  int valid;  // valid rows of this CTA's half (may be 0)
-  int mine;   // rows of this CTA's half inside the expert's group (0 or 128)
+  int tail;   // 1: a 128-row tail tile
+  int valid;  // valid rows of this CTA's share (may be 0)
+  int share;  // rows per CTA: 128, or 64 in a tail tile
 };
 
 // pts[e]: first pair tile of expert e; a group of R rows (R a multiple of 128)
-// spans ceil(R / 256) pair tiles.
+// spans ceil(R / 256) pair tiles, the last one a tail tile when R / 128 is odd.
 __device__ __forceinline__ void pair_tile_starts(int E, const int32_t* gs, int32_t* pts) {
   if (threadIdx.x == 0) {
     int acc = 0;
@@ -713,15 +723,17 @@ __device__ __forceinline__ PairTile decode_pair_tile(const Args& a, const int32_
   t.e = lo;
   t.m0 = gs[lo] + (mt - pts[lo]) * 256;
   t.n0 = nt * P::OUT_N;
-  const int my0 = t.m0 + 128 * static_cast<int>(rank);
-  t.valid = max(0, min(128, gs[lo] + (off[lo + 1] - off[lo]) - my0));
-  t.mine = (my0 < gs[lo + 1]) ? 128 : 0;
+  t.tail = (gs[lo + 1] - t.m0 == 128) ? 1 : 0;
+  t.share = t.tail ? 64 : 128;
+  const int my0 = t.m0 + t.share * static_cast<int>(rank);
+  t.valid = max(0, min(t.share, gs[lo] + (off[lo + 1] - off[lo]) - my0));
   return t;
 }
 
 template <class P>
 __global__ void __launch_bounds__(P::THREADS, 1)
-    pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA64,
+                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB64,
                      const Args a) {
   using OutT = typename P::OutT;
   using HT = __nv_bfloat16;  // h, the SwiGLU output
@@ -763,7 +775,9 @@ __global__ void __launch_bounds__(P::THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmA64);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmB64);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, P::TMEM_COLS);
@@ -794,12 +808,22 @@ __global__ void __launch_bounds__(P::THREADS, 1)
       bool ok = true;
       for (int L = cluster; L < n_tiles && ok; L += n_clusters) {
         const PairTile t = decode_pair_tile<P>(a, gs, off, pts, L, rank);
-        const int arow = t.m0 + 128 * static_cast<int>(rank);
-        int brow;
-        if constexpr (P::EP == Epi::SwigluFwd)
-          brow = t.e * a.b_rows_per_expert + t.n0 + (leader ? 0 : a.f_half);
-        else
+        const int arow = t.m0 + t.share * static_cast<int>(rank);
+        // B rows: gate/up, full tile: the leader the 128 gate rows, the peer the
+        // matching up rows; tail tile: each CTA 64 gate rows and the matching 64
+        // up rows (so that a TMEM lane holds both halves of its outputs). Down:
+        // each CTA one 128-row half of the output columns.
+        int brow, brow2 = 0;
+        if constexpr (P::EP == Epi::SwigluFwd) {
+          if (t.tail) {
+            brow = t.e * a.b_rows_per_expert + t.n0 + 64 * static_cast<int>(rank);
+            brow2 = brow + a.f_half;
+          } else {
+            brow = t.e * a.b_rows_per_expert + t.n0 + (leader ? 0 : a.f_half);
+          }
+        } else {
           brow = t.e * a.b_rows_per_expert + t.n0 + 128 * static_cast<int>(rank);
+        }
         for (int kb = 0; kb < a.K_total / P::BK; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u)) {
             report(a.status, DEV_WAIT_TIMEOUT_PRODUCER);
@@ -807,9 +831,15 @@ __global__ void __launch_bounds__(P::THREADS, 1)
             break;
           }
           unsigned char* sa = stage_base + static_cast<size_t>(stage) * P::STAGE_BYTES;
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * P::STAGE_BYTES);
-          tma_load_2d_pair(&tmA, &full[stage], sa, kb * P::BK, arow);
-          tma_load_2d_pair(&tmB, &full[stage], sa + P::A_BYTES, kb * P::BK, brow);
+          if (leader)
+            mbar_arrive_expect_tx(&full[stage], t.tail ? 2 * (P::A_TAIL_BYTES + P::B_BYTES) : 2 * P::STAGE_BYTES);
+          tma_load_2d_pair(t.tail ? &tmA64 : &tmA, &full[stage], sa, kb * P::BK, arow);
+          if (P::EP == Epi::SwigluFwd && t.tail) {
+            tma_load_2d_pair(&tmB64, &full[stage], sa + P::A_BYTES, kb * P::BK, brow);
+            tma_load_2d_pair(&tmB64, &full[stage], sa + P::A_BYTES + 64 * 128, kb * P::BK, brow2);
+          } else {
+            tma_load_2d_pair(&tmB, &full[stage], sa + P::A_BYTES, kb * P::BK, brow);
+          }
           if (++stage == P::STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -827,6 +857,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
       bool ok = true;
       const int nk = a.K_total / P::BK;
       for (int L = cluster; L < n_tiles && ok; L += n_clusters) {
+        const uint32_t idesc = decode_pair_tile<P>(a, gs, off, pts, L, rank).tail ? P::IDESC_TAIL : P::IDESC;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u)) {
           report(a.status, DEV_WAIT_TIMEOUT_MMA);
           break;
@@ -845,7 +876,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < P::KSTEPS; ++kk)
             umma_bf16_pair(d_tmem, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024),
-                           P::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+                           idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           umma_commit_pair(&empty[stage], 0x3);  // frees the slot in both CTAs
           if (++stage == P::STAGES) {
             stage = 0;
@@ -874,8 +905,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
   } else {
     // ------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
-    const int csel = (warp - 2) >> 2;  // which half of the tile's output columns
-    const int r_local = q * 32 + lane;
+    const int csel = (warp - 2) >> 2;  // which half of the warp's output columns
     const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -886,18 +916,23 @@ __global__ void __launch_bounds__(P::THREADS, 1)
         break;
       }
       tc_fence_after();
-      if (t.mine != 0) {  // rows of the next expert's group are not ours to write
-        const bool row_ok = r_local < t.valid;
-        const int64_t wrow0 = static_cast<int64_t>(t.m0) + 128 * static_cast<int>(rank) + q * 32;
-        constexpr int WCOLS = P::OUT_N / 2;
-        const int cw = csel * WCOLS;
+      {
+        // this warp's 32 rows of the CTA's share, and the accumulator columns
+        // its lane quadrant holds (a tail tile's quadrants 2 and 3 hold the
+        // second half of the columns for the same rows as quadrants 0 and 1)
+        const int rq = t.tail ? (q & 1) : q;
+        const int half = t.tail ? (q >> 1) : 0;
+        const bool row_ok = rq * 32 + lane < t.valid;
+        const int64_t wrow0 = static_cast<int64_t>(t.m0) + t.share * static_cast<int>(rank) + rq * 32;
         unsigned char* stg = stg_base + (warp - 2) * P::STG_WARP_BYTES;
-        const uint32_t tbase =
-            tmem_base + static_cast<uint32_t>(acc * P::BN + cw) + (static_cast<uint32_t>(q * 32) << 16);
+        const uint32_t tq = tmem_base + static_cast<uint32_t>(acc * P::BN) + (static_cast<uint32_t>(q * 32) << 16);
         if constexpr (P::EP == Epi::Store) {
-          OutT* obase = static_cast<OutT*>(a.out) + wrow0 * a.ld_out + t.n0 + cw;
+          // output columns: full tile 128 per warp; tail tile 64 of its quadrant's half
+          const int wc = t.tail ? 64 : 128;
+          OutT* obase = static_cast<OutT*>(a.out) + wrow0 * a.ld_out + t.n0 + half * 128 + csel * wc;
+          const uint32_t tbase = tq + static_cast<uint32_t>(csel * wc);
 #pragma unroll 1
-          for (int c = 0; c < WCOLS; c += 32) {
+          for (int c = 0; c < wc; c += 32) {
             uint32_t r[32];
             tmem_ld32(tbase + c, r);
             tmem_ld_wait();
@@ -907,14 +942,19 @@ __global__ void __launch_bounds__(P::THREADS, 1)
             warp_store_chunk<OutT, P::STG_PITCH>(stg, v, obase + c, a.ld_out, lane);
           }
         } else {
-          HT* obase = static_cast<HT*>(a.out) + wrow0 * a.ld_out + t.n0 + cw;
-          OutT* pbase =
-              (a.out2 != nullptr) ? static_cast<OutT*>(a.out2) + wrow0 * a.ld_out2 + t.n0 + cw : nullptr;
+          // h columns: full tile 64 per warp (gate at accumulator column j, up at
+          // 128 + j); tail tile 32 of its quadrant's 64 (gate at j, up at 64 + j)
+          const int wc = t.tail ? 32 : 64;
+          const int up_off = t.tail ? 64 : P::BN / 2;
+          const int64_t ocol = t.n0 + half * 64 + csel * wc;
+          HT* obase = static_cast<HT*>(a.out) + wrow0 * a.ld_out + ocol;
+          OutT* pbase = (a.out2 != nullptr) ? static_cast<OutT*>(a.out2) + wrow0 * a.ld_out2 + ocol : nullptr;
+          const uint32_t tbase = tq + static_cast<uint32_t>(csel * wc);
 #pragma unroll 1
-          for (int c = 0; c < WCOLS; c += 32) {
+          for (int c = 0; c < wc; c += 32) {
             uint32_t rg[32], ru[32];
             tmem_ld32(tbase + c, rg);
-            tmem_ld32(tbase + P::BN / 2 + c, ru);
+            tmem_ld32(tbase + up_off + c, ru);
             tmem_ld_wait();
             float hv[32];
 #pragma unroll
@@ -1006,8 +1046,8 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtenso
 }
 
 template <class P>
-cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const Args& a, int max_pair_tiles,
-                        cudaStream_t st) {
+cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& ta64, const CUtensorMap& tb,
+                        const CUtensorMap& tb64, const Args& a, int max_pair_tiles, cudaStream_t st) {
   static std::atomic<size_t> smem_set[kMaxDevices];
   cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(pair_gemm_kernel<P>), P::SMEM_BYTES, smem_set);
   if (e != cudaSuccess) return e;
@@ -1020,7 +1060,7 @@ cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const Args
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   return launch_dependent(pair_gemm_kernel<P>, dim3(static_cast<unsigned>(2 * clusters)), dim3(P::THREADS),
-                          P::SMEM_BYTES, st, attr, 1, ta, tb, a);
+                          P::SMEM_BYTES, st, attr, 1, ta, ta64, tb, tb64, a);
 }
 
 // Pair tiles of 256 rows are used when the groups are large: a group of R rows
@@ -1077,9 +1117,12 @@ cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* gr
                            const int32_t* offsets, const void* w_gate_up, void* h, void* preact, int32_t* status,
                            cudaStream_t st) {
   if (use_pairs(s)) {
-    CUtensorMap ta, tb;
+    CUtensorMap ta, ta64, tb, tb64;
     if (!make_map(&ta, x_perm, false, s.P, s.d, 64, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&ta64, x_perm, false, s.P, s.d, 64, 64)) return cudaErrorInvalidValue;
     if (!make_map(&tb, w_gate_up, false, static_cast<uint64_t>(s.E) * 2 * s.f, s.d, 64, 128))
+      return cudaErrorInvalidValue;
+    if (!make_map(&tb64, w_gate_up, false, static_cast<uint64_t>(s.E) * 2 * s.f, s.d, 64, 64))
       return cudaErrorInvalidValue;
     Args a = base_args(s, group_start, offsets, status);
     a.N_total = s.f;
@@ -1091,8 +1134,8 @@ cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* gr
     a.out2 = preact;
     a.ld_out2 = 2 * s.f;
     const int max_pairs = static_cast<int>((s.P / 256 + s.E) * (s.f / 128));
-    if (preact != nullptr) return launch_pair<PairCfg<Epi::SwigluFwd, true>>(ta, tb, a, max_pairs, st);
-    return launch_pair<PairCfg<Epi::SwigluFwd>>(ta, tb, a, max_pairs, st);
+    if (preact != nullptr) return launch_pair<PairCfg<Epi::SwigluFwd, true>>(ta, ta64, tb, tb64, a, max_pairs, st);
+    return launch_pair<PairCfg<Epi::SwigluFwd>>(ta, ta64, tb, tb64, a, max_pairs, st);
   }
   // accumulator: BN/2 gate columns and BN/2 up columns of the same outputs
   const int bn = few_tiles(s, 2 * s.f) ? 128 : 256;
@@ -1121,8 +1164,9 @@ cudaError_t launch_gate_up(const Shape& s, const void* x_perm, const int32_t* gr
 cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_start, const int32_t* offsets,
                         const void* w_down, void* o_perm, bool out32, int32_t* status, cudaStream_t st) {
   if (use_pairs(s) && s.d % 256 == 0) {
-    CUtensorMap ta, tb;
+    CUtensorMap ta, ta64, tb;
     if (!make_map(&ta, h, false, s.P, s.f, 64, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&ta64, h, false, s.P, s.f, 64, 64)) return cudaErrorInvalidValue;
     if (!make_map(&tb, w_down, false, static_cast<uint64_t>(s.E) * s.d, s.f, 64, 128)) return cudaErrorInvalidValue;
     Args a = base_args(s, group_start, offsets, status);
     a.N_total = s.d;
@@ -1131,8 +1175,8 @@ cudaError_t launch_down(const Shape& s, const void* h, const int32_t* group_star
     a.out = o_perm;
     a.ld_out = s.d;
     const int max_pairs = static_cast<int>((s.P / 256 + s.E) * (s.d / 256));
-    if (out32) return launch_pair<PairCfg<Epi::Store, true>>(ta, tb, a, max_pairs, st);
-    return launch_pair<PairCfg<Epi::Store>>(ta, tb, a, max_pairs, st);
+    if (out32) return launch_pair<PairCfg<Epi::Store, true>>(ta, ta64, tb, tb, a, max_pairs, st);
+    return launch_pair<PairCfg<Epi::Store>>(ta, ta64, tb, tb, a, max_pairs, st);
   }
   const int bn = few_tiles(s, s.d) ? 128 : pick_bn(s.d);
   const int kcols = ch_elems(s.fp32);
