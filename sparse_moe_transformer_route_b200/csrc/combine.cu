@@ -235,6 +235,78 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+__device__ __forceinline__ void store4(float* p, const float (&o)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, const __nv_bfloat16 (&o)[4]) {
+  __nv_bfloat162 lo, hi;
+  lo.x = o[0];
+  lo.y = o[1];
+  hi.x = o[2];
+  hi.y = o[3];
+  uint2 u;
+  u.x = *reinterpret_cast<const uint32_t*>(&lo);
+  u.y = *reinterpret_cast<const uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+// The same values for rows of up to 2048 elements, 64 threads per row: thread
+// p holds elements 4p + 256j (j < 8) in registers, so the row is read once
+// with 16-byte loads. The sum of squares runs over each thread's elements in
+// order, then a fixed butterfly within each warp, then warp 0's sum plus warp
+// 1's.
+constexpr int kNormRowsPerCta = 4;
+
+template <typename T_>
+__global__ void __launch_bounds__(64 * kNormRowsPerCta)
+    rmsnorm_rows_kernel(const float* __restrict__ resid, const float* __restrict__ weight, double eps, int d,
+                        int64_t T, T_* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();  // reads and writes buffers an earlier kernel of the layer uses
+  constexpr int kV = 8;  // float4 per thread: d <= 256 * kV
+  __shared__ double part[kNormRowsPerCta][2];
+  const int p = threadIdx.x & 63, row = threadIdx.x >> 6;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kNormRowsPerCta + row;
+  const bool live = t < T;
+  const float4* r = reinterpret_cast<const float4*>(resid + t * d);
+  const int nv = d / 4;
+  float4 v[kV];
+#pragma unroll
+  for (int j = 0; j < kV; ++j)
+    if (live && p + 64 * j < nv) v[j] = __ldg(r + p + 64 * j);
+  double ss = 0.0;
+#pragma unroll
+  for (int j = 0; j < kV; ++j) {
+    if (live && p + 64 * j < nv) {
+      ss = fma(static_cast<double>(v[j].x), static_cast<double>(v[j].x), ss);
+      ss = fma(static_cast<double>(v[j].y), static_cast<double>(v[j].y), ss);
+      ss = fma(static_cast<double>(v[j].z), static_cast<double>(v[j].z), ss);
+      ss = fma(static_cast<double>(v[j].w), static_cast<double>(v[j].w), ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((p & 31) == 0) part[row][p >> 5] = ss;
+  __syncthreads();
+  if (!live) return;
+  const double inv = 1.0 / sqrt((part[row][0] + part[row][1]) / static_cast<double>(d) + eps);
+#pragma unroll
+  for (int j = 0; j < kV; ++j) {
+    const int i = 4 * (p + 64 * j);
+    if (i < d) {
+      const float a[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      T_ o[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        double x = static_cast<double>(a[c]) * inv;
+        if (weight != nullptr) x *= static_cast<double>(weight[i + c]);
+        o[c] = from_f32<T_>(static_cast<float>(x));
+      }
+      store4(out + t * d + i, o);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t* slot_row, const float* probs,
@@ -272,6 +344,16 @@ cudaError_t launch_combine(const Shape& s, const void* o_perm, bool o32, const i
 
 cudaError_t launch_rmsnorm(const Shape& s, const float* resid, const float* weight, double eps, void* out,
                            cudaStream_t st) {
+  if (s.d <= 2048) {  // 64 threads per row, the row in registers
+    const unsigned grid = static_cast<unsigned>((s.T + kNormRowsPerCta - 1) / kNormRowsPerCta);
+    if (s.fp32)
+      launch_dependent(rmsnorm_rows_kernel<float>, dim3(grid), dim3(64 * kNormRowsPerCta), 0, st, nullptr, 0, resid,
+                       weight, eps, s.d, s.T, static_cast<float*>(out));
+    else
+      launch_dependent(rmsnorm_rows_kernel<__nv_bfloat16>, dim3(grid), dim3(64 * kNormRowsPerCta), 0, st, nullptr, 0,
+                       resid, weight, eps, s.d, s.T, static_cast<__nv_bfloat16*>(out));
+    return cudaGetLastError();
+  }
   const unsigned grid = static_cast<unsigned>(s.T);
   if (s.fp32)
     launch_dependent(rmsnorm_kernel<float>, dim3(grid), dim3(256), 0, st, nullptr, 0, resid, weight, eps, s.d, static_cast<float*>(out));

@@ -43,7 +43,8 @@ namespace moe {
 namespace {
 
 constexpr int kTile = kDispatchChunk;  // 32 tokens
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;          // logits kernel: TMA warp, MMA warp, 4 epilogue warps
+constexpr int kFusedThreads = 512;     // fused kernel: 16 warps; warps 0 and 1 also load and issue the MMAs
 constexpr int kMaxE = 64;
 constexpr int kMaxSel = kMaxTopK + 3;
 constexpr int kAload = kTile * 128;                      // bytes of A loaded per stage
@@ -51,11 +52,9 @@ constexpr int kStageMax = kAload + kMaxE * 128;          // 12 KB
 // ring bytes for S stages, plus the over-read of the last stage's A
 constexpr int ring_bytes(int S) { return S * kStageMax + 16 * 1024; }
 constexpr int kLogitStride = kMaxE + 1;
-constexpr int kScanBlock = 128;                          // chunks scanned per pass in the last CTA
 constexpr size_t kMiscBytes = 4096;
 constexpr size_t smem_bytes(int S) { return 1024 + static_cast<size_t>(ring_bytes(S)) + kMiscBytes; }
 static_assert(kTile == 32, "one mask word per expert");
-static_assert(kScanBlock * kMaxE * 8 <= ring_bytes(7), "scan block fits in the smallest ring");
 
 struct RArgs {
   int64_t T;
@@ -86,36 +85,70 @@ struct RArgs {
   int probs_only;     // stop after p and lse (expert choice selects from p afterwards)
 };
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// The router's work once the tile's 32 logit rows are in shared memory (S),
+// shared by the fused kernel and the epilogue-only kernel. kEpiThreads
+// threads (tid 0..511, 16 warps) synchronise on named barrier 1; a half-warp
+// takes a token and each of its 16 threads four experts (e = sub + 16 i).
+//   softmax      half-warp max and sum, probabilities and lse in fp32;
+//   ranks        each expert's rank among the token's fp32 logits (larger
+//                first, equal values to the lower index) and the distance to
+//                the nearest other logit, in one pass over the row;
+//   exact ranks  a token whose k+1 largest logits hold two values closer than
+//                2e-4 * max(1, |h|) (far above the error of a 2048-term fp32
+//                sum of exact bf16 products) has every run of such neighbours
+//                that reaches its top k recomputed exactly (fp64 sums of the
+//                exact products, a warp per logit) and re-ranked; a run that
+//                reaches past rank k+3 has all E logits recomputed;
+//   outputs      the k best experts in slot order with their weights, a bit
+//                mask per expert of the tile's tokens that chose it (each
+//                pair's rank inside the chunk), the per-chunk counts and the
+//                loss partials.
+// The last CTA to finish scans the per-chunk counts into chunk bases (each
+// expert's chunks cut into 8 segments, one thread each), the bincount
+// offsets and the padded group starts, and reduces the loss partials. Every
+// sum runs in a fixed order, so the results are deterministic.
+constexpr int kEpiThreads = 512;
+constexpr int kEpiWarps = kEpiThreads / 32;
+constexpr int kScanSeg = kEpiThreads / kMaxE;   // segments per expert in the scan
+constexpr int kScanBlock = 64;                  // chunks per pass of the scan
+constexpr int kWin = kMaxSel + 1;               // sorted window of a token: ranks 0 .. k+3
+// byte offsets inside the free ring (after the accumulator is complete)
+constexpr int kOffS = 0;                                        // float [kTile][kLogitStride]
+constexpr int kOffP = kOffS + kTile * kLogitStride * 4;         // float [kTile][kMaxE]
+constexpr int kOffRk = kOffP + kTile * kMaxE * 4;               // uint8 [kTile][kMaxE]
+constexpr int kOffSv = kOffRk + kTile * kMaxE;                  // float [kTile][kWin]
+constexpr int kOffSe = kOffSv + kTile * kWin * 4;               // int   [kTile][kWin]
+constexpr int kOffQ = kOffSe + kTile * kWin * 4;                // uint32 [kTile * kMaxE]
+constexpr int kOffX = (kOffQ + kTile * kMaxE * 4 + 7) / 8 * 8;  // double [kTile * kMaxE]
+constexpr int kOffQb = kOffX + kTile * kMaxE * 8;               // int [kTile] first slot, count, all-E flag
+constexpr int kOffSegI = kOffQb + 3 * kTile * 4;                // int [kScanSeg][kMaxE]
+constexpr int kOffSegD = kOffSegI + kScanSeg * kMaxE * 4;       // double [kScanSeg][kMaxE]
+constexpr int kOffZ = kOffSegD + kScanSeg * kMaxE * 8;          // double [kEpiThreads]
+constexpr int kOffScan = kOffZ + kEpiThreads * 8;               // int + float [kScanBlock][kMaxE]
+constexpr int kEpiScratch = kOffScan + kScanBlock * kMaxE * 8;
+static_assert(kOffX % 8 == 0 && kOffSegD % 8 == 0 && kOffZ % 8 == 0 && kOffScan % 16 == 0, "alignment");
+
+struct EpiSmem {
+  unsigned char* ring;  // kEpiScratch bytes
+  uint32_t* mask;       // [kMaxE]
+  float* lse_s;         // [kTile]
+  int32_t* s_last;
+  int32_t* qn;
+  int32_t* tot;         // [kMaxE]
+  double* tot_p;        // [kMaxE]
+};
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
 __device__ __forceinline__ float near_gap(float v) { return 2e-4f * fmaxf(1.0f, fabsf(v)); }
 
-// Arg-max across the 4 threads of a quad: larger value wins, equal values go to the lower index.
-// Quads may diverge (near-ties, the ragged last tile), so every quad shuffle
-// names only its own four lanes.
-__device__ __forceinline__ unsigned quad_mask() { return 0xFu << ((threadIdx.x & 31) & 28); }
-
-template <typename V>
-__device__ __forceinline__ void quad_argmax(V& v, int& i) {
-  const unsigned qm = quad_mask();
-#pragma unroll
-  for (int o = 1; o <= 2; o <<= 1) {
-    const V ov = __shfl_xor_sync(qm, v, o);
-    const int oi = __shfl_xor_sync(qm, i, o);
-    if (ov > v || (ov == v && oi < i)) {
-      v = ov;
-      i = oi;
-    }
-  }
-}
-
 // <x_t, W_r[e]> from exact products of bf16 inputs, summed in fp64 by a whole
-// warp: lane l takes elements 8l + 256i; the loads of up to 16 steps are issued
-// before any arithmetic so the row pair costs about one memory round trip. The
+// warp: lane l takes elements 8l + 256i; the loads of 4 steps are issued before
+// their arithmetic, so a row pair of d = 2048 costs two memory round trips. The
 // lane sums are combined by a fixed shuffle tree (every lane gets the result).
 __device__ __forceinline__ double exact_logit_warp(const __nv_bfloat16* xr, const __nv_bfloat16* wr, int d,
                                                    int lane) {
-  constexpr int kBatch = 16;
+  constexpr int kBatch = 4;
   double acc = 0.0;
   for (int base = lane * 8; base < d; base += 256 * kBatch) {
     uint4 xv[kBatch], wv[kBatch];
@@ -146,175 +179,130 @@ __device__ __forceinline__ double exact_logit_warp(const __nv_bfloat16* xr, cons
   return acc;
 }
 
-// The router's work once the tile's 32 logit rows are in shared memory (S),
-// shared by the fused kernel and the epilogue-only kernel. 128 threads
-// (tid 0..127, lane = tid % 32) synchronise on named barrier 1; the last CTA
-// of the grid also scans the per-chunk counts through `ring` (kScanBlock*E*8 bytes).
-struct EpiSmem {
-  float* S;
-  float* P;
-  int32_t* chosen;
-  uint32_t* queue;
-  double* exact;
-  int32_t* qn;
-  uint32_t* mask;
-  float* lse_s;
-  int32_t* s_last;
-  int32_t* tot;
-  double* tot_p;
-  double* zred;
-  unsigned char* ring;
-};
-
 __device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& sm, int64_t t0, int tid, int lane) {
-  float* S = sm.S;
-  float* P = sm.P;
-  int32_t* chosen = sm.chosen;
-  uint32_t* queue = sm.queue;
-  double* exact = sm.exact;
-  int32_t* qn = sm.qn;
-  uint32_t* mask = sm.mask;
-  float* lse_s = sm.lse_s;
-  int32_t* s_last = sm.s_last;
-  int32_t* tot = sm.tot;
-  double* tot_p = sm.tot_p;
-  double* zred = sm.zred;
-  unsigned char* ring = sm.ring;
+  unsigned char* R = sm.ring;
+  float* S = reinterpret_cast<float*>(R + kOffS);
+  float* P = reinterpret_cast<float*>(R + kOffP);
+  uint8_t* rk = R + kOffRk;
+  float* sv = reinterpret_cast<float*>(R + kOffSv);
+  int32_t* se = reinterpret_cast<int32_t*>(R + kOffSe);
+  uint32_t* queue = reinterpret_cast<uint32_t*>(R + kOffQ);
+  double* exact = reinterpret_cast<double*>(R + kOffX);
+  int32_t* qb = reinterpret_cast<int32_t*>(R + kOffQb);  // [kTile] first slot, [kTile] count, [kTile] all-E
   const int E = a.E, k = a.k;
-  // ---- a quad per token: thread qp holds experts 16*qp .. 16*qp+15
-  const int r = tid >> 2, qp = tid & 3;
+  const int r = tid >> 4, sub = tid & 15;
+  const unsigned hm = 0xFFFFu << (lane & 16);
   const int64_t t = t0 + r;
-  const bool valid = t < a.T;  // the whole quad agrees
-  const int eb = qp * 16;
-  float h[16];
+  const bool valid = t < a.T;  // the whole half-warp agrees
+  // ---- softmax over the token's E logits
+  float h[4], ex[4];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) h[i] = S[r * kLogitStride + eb + i];
-  float m = -INFINITY;
+  for (int i = 0; i < 4; ++i) {
+    const int e = sub + 16 * i;
+    h[i] = e < E ? S[r * kLogitStride + e] : -INFINITY;
+  }
+  float m = fmaxf(fmaxf(h[0], h[1]), fmaxf(h[2], h[3]));
 #pragma unroll
-  for (int i = 0; i < 16; ++i) m = fmaxf(m, h[i]);
-  const unsigned qm = quad_mask();
-  m = fmaxf(m, __shfl_xor_sync(qm, m, 1));
-  m = fmaxf(m, __shfl_xor_sync(qm, m, 2));
-  float ex[16];  // exp(h - m), computed once for the sum and the probabilities
+  for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(hm, m, o));
   float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    ex[i] = (eb + i < E) ? expf(h[i] - m) : 0.f;
+  for (int i = 0; i < 4; ++i) {
+    ex[i] = (sub + 16 * i < E) ? expf(h[i] - m) : 0.f;
     s += ex[i];
   }
-  s += __shfl_xor_sync(qm, s, 1);
-  s += __shfl_xor_sync(qm, s, 2);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(hm, s, o);
   const float lse = m + logf(s);
-  {
-    float pv[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) pv[i] = valid ? ex[i] / s : 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) P[r * kMaxE + eb + i] = pv[i];
-    if (valid && eb < E) {
-      float* dst = a.probs + t * E + eb;
-      if (eb + 16 <= E) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          reinterpret_cast<float4*>(dst)[i] = make_float4(pv[4 * i], pv[4 * i + 1], pv[4 * i + 2], pv[4 * i + 3]);
-      } else {
-        for (int i = 0; i < E - eb; ++i) dst[i] = pv[i];
-      }
-    }
+  for (int i = 0; i < 4; ++i) {
+    const int e = sub + 16 * i;
+    const float p = valid ? ex[i] / s : 0.f;
+    P[r * kMaxE + e] = p;
+    if (valid && e < E) a.probs[t * E + e] = p;
   }
-  if (qp == 0) {
-    lse_s[r] = valid ? lse : 0.f;
+  if (sub == 0) {
+    sm.lse_s[r] = valid ? lse : 0.f;
     if (valid) a.lse_out[t] = lse;
   }
   if (a.probs_only) return;  // uniform over the CTA
 
-  // ---- top (k+3) in fp32 by quad arg-max (uniform within the quad); nearm bit j
-  //      marks ranks j and j+1 as closer than the fp32 uncertainty
-  const int nsel = min(k + 3, E);
-  int ord[kMaxSel];
-  float val[kMaxSel];
-  uint32_t taken = 0;  // bit i: expert eb + i chosen
-  uint32_t nearm = 0;
+  // ---- ranks among the fp32 logits and the nearest other logit
+  int rank[4] = {0, 0, 0, 0};
+  float gap[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+  for (int e2 = 0; e2 < E; ++e2) {
+    const float v = S[r * kLogitStride + e2];
 #pragma unroll
-  for (int j = 0; j < kMaxSel; ++j) {
-    if (j < nsel) {
-      float v = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        if (eb + i < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || h[i] > v)) {
-          v = h[i];
-          bi = eb + i;
-        }
+    for (int i = 0; i < 4; ++i) {
+      const int e = sub + 16 * i;
+      if (e2 != e) {
+        rank[i] += (v > h[i] || (v == h[i] && e2 < e)) ? 1 : 0;
+        gap[i] = fminf(gap[i], fabsf(v - h[i]));
       }
-      quad_argmax(v, bi);
-      if (bi - eb >= 0 && bi - eb < 16) taken |= 1u << (bi - eb);
-      ord[j] = bi;
-      val[j] = v;
-      if (j > 0 && val[j - 1] - v < near_gap(val[j - 1])) nearm |= 1u << (j - 1);
     }
   }
-  float hv[kMaxSel];  // fp32 logit of ord[j], kept for the weights
+  bool nearv = false;
 #pragma unroll
-  for (int j = 0; j < kMaxSel; ++j) hv[j] = val[j];
-  // Slow path (rare): some run of near-equal neighbours decides a slot order or
-  // the k-th choice. It works on local copies so the common path stays in registers.
-  const bool slow = valid && (nearm & ((1u << k) - 1u)) != 0;
-  bool fallback = false;
-  int run_a[kMaxSel], run_b[kMaxSel];
-  int nrun = 0;
-  int oloc[kMaxSel];
-  float hloc[kMaxSel];
-  if (slow) {
-#pragma unroll
-    for (int j = 0; j < kMaxSel; ++j) {
-      oloc[j] = ord[j];
-      hloc[j] = hv[j];
+  for (int i = 0; i < 4; ++i) {
+    const int e = sub + 16 * i;
+    if (e < E) {
+      rk[r * kMaxE + e] = static_cast<uint8_t>(rank[i]);
+      if (rank[i] <= k && gap[i] < near_gap(h[i])) nearv = true;
+      if (rank[i] < kWin) {  // the sorted window of the first k+4 ranks
+        sv[r * kWin + rank[i]] = h[i];
+        se[r * kWin + rank[i]] = e;
+      }
     }
-    int jj = 0;
-    while (jj < nsel - 1) {
-      if ((nearm >> jj) & 1u) {
-        int b = jj + 1;
-        while (b < nsel - 1 && ((nearm >> b) & 1u)) ++b;
-        if (jj <= k - 1) {
-          if (b == nsel - 1 && nsel < E) {
-            fallback = true;
-            break;
+  }
+  const bool near = valid && __any_sync(hm, nearv);
+  if (tid == 0) *sm.qn = 0;
+  epi_sync();
+  // ---- queue the logits to recompute exactly: runs of near neighbours in the
+  //      sorted window that reach into the top k (rare; one thread per token)
+  if (sub == 0) {
+    int cnt = 0, base = 0;
+    bool fallback = false;
+    if (near) {
+      const int win = min(k + 4, E);
+      // run bounds [ra, rb] with consecutive gaps under the bar
+      int ra = 0;
+      for (int j = 1; j <= win; ++j) {
+        const bool link = j < win && (sv[r * kWin + j - 1] - sv[r * kWin + j] < near_gap(sv[r * kWin + j - 1]));
+        if (!link) {
+          if (j - 1 > ra && ra <= k - 1) {  // a run of length >= 2 reaching into the top k
+            if (j == win && win < E) fallback = true;  // it may continue past the window
+            cnt += j - ra;
           }
-          run_a[nrun] = jj;
-          run_b[nrun] = b;
-          ++nrun;
+          ra = j;
         }
-        jj = b;
+      }
+      if (fallback) cnt = E;
+      base = atomicAdd(sm.qn, cnt);
+      if (fallback) {
+        for (int e = 0; e < E; ++e) queue[base + e] = (static_cast<uint32_t>(r) << 8) | static_cast<uint32_t>(e);
       } else {
-        ++jj;
+        int p = base;
+        ra = 0;
+        for (int j = 1; j <= win; ++j) {
+          const bool link = j < win && (sv[r * kWin + j - 1] - sv[r * kWin + j] < near_gap(sv[r * kWin + j - 1]));
+          if (!link) {
+            if (j - 1 > ra && ra <= k - 1)
+              for (int y = ra; y < j; ++y)
+                queue[p++] = (static_cast<uint32_t>(r) << 8) | static_cast<uint32_t>(se[r * kWin + y]);
+            ra = j;
+          }
+        }
       }
     }
-  }
-  // queue the (token, expert) pairs whose exact logits are needed
-  int nitems = 0;
-  if (fallback) {
-    nitems = E;
-  } else {
-    for (int i = 0; i < nrun; ++i) nitems += run_b[i] - run_a[i] + 1;
-  }
-  int qbase = 0;
-  if (qp == 0 && nitems > 0) qbase = atomicAdd(qn, nitems);
-  qbase = __shfl_sync(qm, qbase, lane & ~3);
-  if (fallback) {
-    for (int e = qp; e < E; e += 4) queue[qbase + e] = (static_cast<uint32_t>(r) << 8) | static_cast<uint32_t>(e);
-  } else if (nrun > 0) {
-    int p = 0;
-    for (int i = 0; i < nrun; ++i)
-      for (int y = run_a[i]; y <= run_b[i]; ++y, ++p)
-        if ((p & 3) == qp) queue[qbase + p] = (static_cast<uint32_t>(r) << 8) | static_cast<uint32_t>(oloc[y]);
+    qb[r] = base;
+    qb[kTile + r] = cnt;
+    qb[2 * kTile + r] = fallback ? 1 : 0;
   }
   epi_sync();
-  // ---- exact logits of the queued pairs: a warp per pair, all loads in flight together
+  // ---- exact logits of the queued pairs: a warp per pair
   {
-    const int nq = *qn;
-    const int ew = tid >> 5;
-    for (int it = ew; it < nq; it += 4) {
+    const int nq = *sm.qn;
+    const int w = tid >> 5;
+    for (int it = w; it < nq; it += kEpiWarps) {
       const uint32_t code = queue[it];
       const int rr = static_cast<int>(code >> 8), e = static_cast<int>(code & 255u);
       const double v = exact_logit_warp(a.x + (t0 + rr) * a.d, a.w + static_cast<int64_t>(e) * a.d, a.d, lane);
@@ -322,246 +310,221 @@ __device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& s
     }
   }
   epi_sync();
-  if (slow) {
-    if (!fallback) {  // re-rank each run by its exact logits (ties: lower expert index)
-      int p = qbase;
-      for (int i = 0; i < nrun; ++i) {
-        const int ra = run_a[i], rb = run_b[i];
-        double ex[kMaxSel];
-        for (int y = ra; y <= rb; ++y) ex[y] = exact[p++];
-        for (int x1 = ra + 1; x1 <= rb; ++x1) {
-          const double ve = ex[x1];
-          const int oe = oloc[x1];
-          const float he = hloc[x1];
-          int y = x1 - 1;
-          while (y >= ra && (ex[y] < ve || (ex[y] == ve && oloc[y] > oe))) {
-            ex[y + 1] = ex[y];
-            oloc[y + 1] = oloc[y];
-            hloc[y + 1] = hloc[y];
-            --y;
-          }
-          ex[y + 1] = ve;
-          oloc[y + 1] = oe;
-          hloc[y + 1] = he;
+  // ---- re-rank the queued experts of each such token by their exact logits
+  if (sub == 0 && qb[kTile + r] > 0) {
+    const int base = qb[r], cnt = qb[kTile + r];
+    if (qb[2 * kTile + r] != 0) {  // every expert (queued in expert order): ranks from the exact values
+      for (int i = 0; i < E; ++i) {
+        const double vi = exact[base + i];
+        int rr = 0;
+        for (int j = 0; j < E; ++j) {
+          const double vj = exact[base + j];
+          rr += (vj > vi || (vj == vi && j < i)) ? 1 : 0;
         }
+        rk[r * kMaxE + i] = static_cast<uint8_t>(rr);  // queue order is expert order
       }
-    } else {  // a run reaches past rank k+3: rank every expert by its exact logit
-      double xe[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) xe[i] = (eb + i < E) ? exact[qbase + eb + i] : -INFINITY;
-      uint32_t tk = 0;
-      for (int j = 0; j < k; ++j) {
-        double v = -INFINITY;
-        int bi = 0x7fffffff;
-        float hb = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (eb + i < E && !((tk >> i) & 1u) && (bi == 0x7fffffff || xe[i] > v)) {
-            v = xe[i];
-            bi = eb + i;
-            hb = h[i];
+    } else {
+      // each queued run occupies consecutive ranks; sort every run by the exact
+      // values (equal values: the lower expert) and hand its ranks back in order
+      int i0 = 0;
+      while (i0 < cnt) {
+        const int first_rank = rk[r * kMaxE + (queue[base + i0] & 255u)];
+        int i1 = i0 + 1;
+        while (i1 < cnt && rk[r * kMaxE + (queue[base + i1] & 255u)] == first_rank + (i1 - i0)) ++i1;
+        for (int i = i0; i < i1; ++i) {
+          const int ei = static_cast<int>(queue[base + i] & 255u);
+          const double vi = exact[base + i];
+          int rr = 0;
+          for (int j = i0; j < i1; ++j) {
+            const int ej = static_cast<int>(queue[base + j] & 255u);
+            const double vj = exact[base + j];
+            rr += (vj > vi || (vj == vi && ej < ei)) ? 1 : 0;
           }
+          rk[r * kMaxE + ei] = static_cast<uint8_t>(first_rank + rr);
         }
-        quad_argmax(v, bi);
-        if (bi - eb >= 0 && bi - eb < 16) tk |= 1u << (bi - eb);
-        oloc[j] = bi;
-        // the fp32 logit of the winner, from the thread that holds it
-        const int owner = (lane & ~3) | ((bi >> 4) & 3);
-        hloc[j] = __shfl_sync(qm, (bi >= eb && bi < eb + 16) ? hb : 0.f, owner);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kMaxSel; ++j) {
-      ord[j] = oloc[j];
-      hv[j] = hloc[j];
-    }
-  }
-  // ---- outputs: thread qp writes slots qp, qp+4, ...
-  if (valid) {
-    // the weights' denominator: all experts' exponentials, or (renormalised)
-    // the k chosen ones summed in slot order
-    float den = s;
-    if (a.renorm) {
-      den = 0.f;
-#pragma unroll
-      for (int j = 0; j < kMaxTopK; ++j)
-        if (j < k) den += expf(hv[j] - m);
-    }
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < k && (j & 3) == qp) {
-        const int e = ord[j];
-        a.idx_out[t * k + j] = e;
-        a.w_out[t * k + j] = expf(hv[j] - m) / den;
-        chosen[r * kMaxTopK + j] = e;
-        atomicOr(&mask[e], 1u << r);
+        i0 = i1;
       }
     }
   }
   epi_sync();
-  // ---- ranks inside the chunk and per-CTA partials
+  // ---- outputs: the experts ranked below k, slot = rank
+  float chosen_ex = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = sub + 16 * i;
+    rank[i] = e < E ? static_cast<int>(rk[r * kMaxE + e]) : E;
+    if (rank[i] < k) chosen_ex += ex[i];
+  }
+  float den = s;
+  if (a.renorm) {  // the weights' denominator: the k chosen exponentials
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) chosen_ex += __shfl_xor_sync(hm, chosen_ex, o);
+    den = chosen_ex;
+  }
   if (valid) {
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < k && (j & 3) == qp) {
-        const int e = ord[j];
-        a.local_rank[t * k + j] = __popc(mask[e] & ((1u << r) - 1u));
+    for (int i = 0; i < 4; ++i) {
+      const int e = sub + 16 * i;
+      if (rank[i] < k) {
+        a.idx_out[t * k + rank[i]] = e;
+        a.w_out[t * k + rank[i]] = ex[i] / den;
+        atomicOr(&sm.mask[e], 1u << r);
       }
+    }
+  }
+  epi_sync();
+  // ---- ranks inside the chunk and the per-CTA partials
+  if (valid) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = sub + 16 * i;
+      if (rank[i] < k) a.local_rank[t * k + rank[i]] = __popc(sm.mask[e] & ((1u << r) - 1u));
     }
   }
   const int cta = blockIdx.x;
   if (tid < E) {
-    a.chunk_count[static_cast<size_t>(cta) * E + tid] = __popc(mask[tid]);
+    a.chunk_count[static_cast<size_t>(cta) * E + tid] = __popc(sm.mask[tid]);
     float ps = 0.f;
     for (int rr = 0; rr < kTile; ++rr) ps += P[rr * kMaxE + tid];
     a.psum_part[static_cast<size_t>(cta) * E + tid] = ps;
   }
-  if (tid == 0) {
+  if (tid == kMaxE) {
     double z = 0.0;
-    for (int rr = 0; rr < kTile; ++rr) z += static_cast<double>(lse_s[rr]) * lse_s[rr];
+    for (int rr = 0; rr < kTile; ++rr) z += static_cast<double>(sm.lse_s[rr]) * sm.lse_s[rr];
     a.zsum_part[cta] = z;
   }
   __threadfence();
   epi_sync();
-  if (tid == 0) *s_last = (atomicAdd(a.ticket, 1) == static_cast<int>(gridDim.x) - 1);
+  if (tid == 0) *sm.s_last = (atomicAdd(a.ticket, 1) == static_cast<int>(gridDim.x) - 1);
   epi_sync();
-  if (*s_last) {
-    __threadfence();
-    const int nb = gridDim.x;
-    int32_t* cnt_s = reinterpret_cast<int32_t*>(ring);                     // [kScanBlock][E]
-    float* ps_s = reinterpret_cast<float*>(ring + kScanBlock * kMaxE * 4);  // [kScanBlock][E]
-    int run = 0;       // thread tid < E: running total of expert tid
-    double pe = 0.0;
-    for (int c0 = 0; c0 < nb; c0 += kScanBlock) {
-      const int nc = min(kScanBlock, nb - c0);
-      // the block's counts and probability sums, read with all 128 threads as
-      // 16-byte loads, eight in flight per thread (c0 * E is a multiple of 4)
-      {
-        const int n = nc * E;
-        const int32_t* gc = a.chunk_count + static_cast<size_t>(c0) * E;
-        const float* gp = a.psum_part + static_cast<size_t>(c0) * E;
-        for (int i0 = tid * 4; i0 < (n & ~3); i0 += 128 * 4 * 8) {
-          int4 cv[8];
-          float4 pv[8];
-#pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            const int i = i0 + b * 512;
-            if (i < (n & ~3)) {
-              cv[b] = __ldcg(reinterpret_cast<const int4*>(gc + i));
-              pv[b] = __ldcg(reinterpret_cast<const float4*>(gp + i));
-            }
-          }
-#pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            const int i = i0 + b * 512;
-            if (i < (n & ~3)) {
-              *reinterpret_cast<int4*>(cnt_s + i) = cv[b];
-              *reinterpret_cast<float4*>(ps_s + i) = pv[b];
-            }
-          }
-        }
-        for (int i = (n & ~3) + tid; i < n; i += 128) {
-          cnt_s[i] = __ldcg(gc + i);
-          ps_s[i] = __ldcg(gp + i);
-        }
+  if (!*sm.s_last) return;
+
+  // ---- the last CTA: scan of the per-chunk counts, losses
+  __threadfence();
+  const int nb = gridDim.x;
+  int32_t* seg_i = reinterpret_cast<int32_t*>(R + kOffSegI);
+  double* seg_d = reinterpret_cast<double*>(R + kOffSegD);
+  double* zred = reinterpret_cast<double*>(R + kOffZ);
+  int32_t* cnt_s = reinterpret_cast<int32_t*>(R + kOffScan);               // [kScanBlock][E]
+  float* ps_s = reinterpret_cast<float*>(R + kOffScan + kScanBlock * kMaxE * 4);  // [kScanBlock][E]
+  const int e = tid & (kMaxE - 1), g = tid / kMaxE;  // expert, segment
+  constexpr int kSegLen = kScanBlock / kScanSeg;
+  int run = 0;
+  double pe = 0.0;
+  for (int c0 = 0; c0 < nb; c0 += kScanBlock) {
+    const int nc = min(kScanBlock, nb - c0);
+    {  // the block's counts and probability sums, 16-byte loads (c0 * E is a multiple of 4)
+      const int n = nc * E;
+      const int32_t* gc = a.chunk_count + static_cast<size_t>(c0) * E;
+      const float* gp = a.psum_part + static_cast<size_t>(c0) * E;
+      for (int i = tid * 4; i < (n & ~3); i += kEpiThreads * 4) {
+        *reinterpret_cast<int4*>(cnt_s + i) = __ldcg(reinterpret_cast<const int4*>(gc + i));
+        *reinterpret_cast<float4*>(ps_s + i) = __ldcg(reinterpret_cast<const float4*>(gp + i));
       }
-      epi_sync();
-      if (tid < E) {  // eight chunks' loads in flight, then the running sums in order
-        int c = 0;
-        for (; c + 8 <= nc; c += 8) {
-          int v[8];
-          float q[8];
-#pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            v[b] = cnt_s[(c + b) * E + tid];
-            q[b] = ps_s[(c + b) * E + tid];
-          }
-#pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            cnt_s[(c + b) * E + tid] = run;  // becomes the chunk base
-            run += v[b];
-            pe += static_cast<double>(q[b]);
-          }
-        }
-        for (; c < nc; ++c) {
-          const int v = cnt_s[c * E + tid];
-          cnt_s[c * E + tid] = run;
-          run += v;
-          pe += static_cast<double>(ps_s[c * E + tid]);
-        }
+      for (int i = (n & ~3) + tid; i < n; i += kEpiThreads) {
+        cnt_s[i] = __ldcg(gc + i);
+        ps_s[i] = __ldcg(gp + i);
       }
-      epi_sync();
-      for (int i = tid; i < nc * E; i += 128) a.chunk_base[static_cast<size_t>(c0) * E + i] = cnt_s[i];
-      epi_sync();
-    }
-    if (tid < E) {
-      tot[tid] = run;
-      tot_p[tid] = pe;
-      a.counts_ws[tid] = run;
-      if (a.counts_user != nullptr) a.counts_user[tid] = run;
-    }
-    // sum of lse^2 partials: 128 contiguous slices in order, then the slices in order
-    {
-      const int per = (nb + 127) / 128;
-      double z = 0.0;
-      for (int c = tid * per; c < min(nb, (tid + 1) * per); ++c) z += __ldcg(&a.zsum_part[c]);
-      zred[tid] = z;
     }
     epi_sync();
-    if (tid < 32) {
-      // warp-wide finalisation (E <= 64): lane holds experts lane and lane + 32.
-      // Group starts and offsets are exclusive prefix sums; the two loss sums use a
-      // fixed butterfly order, so every lane ends with the same bits on every run.
-      const int e0 = lane, e1 = lane + 32;
-      const int c0v = e0 < E ? tot[e0] : 0, c1v = e1 < E ? tot[e1] : 0;
-      const int g0v = (c0v + kRowAlign - 1) / kRowAlign * kRowAlign;
-      const int g1v = (c1v + kRowAlign - 1) / kRowAlign * kRowAlign;
-      int ic0 = c0v, ig0 = g0v, ic1 = c1v, ig1 = g1v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u0 = __shfl_up_sync(0xffffffffu, ic0, o), w0 = __shfl_up_sync(0xffffffffu, ig0, o);
-        const int u1 = __shfl_up_sync(0xffffffffu, ic1, o), w1 = __shfl_up_sync(0xffffffffu, ig1, o);
-        if (lane >= o) {
-          ic0 += u0;
-          ig0 += w0;
-          ic1 += u1;
-          ig1 += w1;
+    int sc = 0;
+    double sp = 0.0;
+    if (e < E) {
+      for (int j = 0; j < kSegLen; ++j) {
+        const int c = g * kSegLen + j;
+        if (c < nc) {
+          sc += cnt_s[c * E + e];
+          sp += static_cast<double>(ps_s[c * E + e]);
         }
       }
-      const int tc0 = __shfl_sync(0xffffffffu, ic0, 31), tg0 = __shfl_sync(0xffffffffu, ig0, 31);
-      const int tc1 = __shfl_sync(0xffffffffu, ic1, 31), tg1 = __shfl_sync(0xffffffffu, ig1, 31);
-      if (e0 < E) {
-        a.offsets_ws[e0] = ic0 - c0v;
-        a.gs_ws[e0] = ig0 - g0v;
-      }
-      if (e1 < E) {
-        a.offsets_ws[e1] = tc0 + ic1 - c1v;
-        a.gs_ws[e1] = tg0 + ig1 - g1v;
-      }
-      // load balance: E * sum_e (c_e / (T k)) (P_e / T) = E * sum_e c_e P_e / (T^2 k)
-      double lb = (e0 < E ? static_cast<double>(c0v) * tot_p[e0] : 0.0) +
-                  (e1 < E ? static_cast<double>(c1v) * tot_p[e1] : 0.0);
-      double zt = ((zred[4 * lane] + zred[4 * lane + 1]) + zred[4 * lane + 2]) + zred[4 * lane + 3];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        lb += __shfl_xor_sync(0xffffffffu, lb, o);
-        zt += __shfl_xor_sync(0xffffffffu, zt, o);
-      }
-      if (lane == 0) {
-        const int off = tc0 + tc1;
-        a.offsets_ws[E] = off;
-        a.gs_ws[E] = tg0 + tg1;
-        const double Td = static_cast<double>(a.T);
-        const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(zt / Td);
-        a.losses_ws[0] = l0;
-        a.losses_ws[1] = l1;
-        if (a.losses_user != nullptr) {
-          a.losses_user[0] = l0;
-          a.losses_user[1] = l1;
+    }
+    seg_i[g * kMaxE + e] = sc;
+    seg_d[g * kMaxE + e] = sp;
+    epi_sync();
+    if (e < E) {
+      int base = run;
+      for (int g2 = 0; g2 < g; ++g2) base += seg_i[g2 * kMaxE + e];
+      for (int j = 0; j < kSegLen; ++j) {
+        const int c = g * kSegLen + j;
+        if (c < nc) {
+          a.chunk_base[static_cast<size_t>(c0 + c) * E + e] = base;
+          base += cnt_s[c * E + e];
         }
-        if (static_cast<int64_t>(off) != a.T * k) report(a.status, DEV_COUNT_MISMATCH);
-        *a.ticket = 0;
       }
+      for (int g2 = 0; g2 < kScanSeg; ++g2) {
+        run += seg_i[g2 * kMaxE + e];
+        pe += seg_d[g2 * kMaxE + e];
+      }
+    }
+    epi_sync();  // the block's scratch is reused by the next pass
+  }
+  if (g == 0 && e < E) {
+    sm.tot[e] = run;
+    sm.tot_p[e] = pe;
+    a.counts_ws[e] = run;
+    if (a.counts_user != nullptr) a.counts_user[e] = run;
+  }
+  {  // sum of lse^2 partials: contiguous slices in order, then the slices in order
+    const int per = (nb + kEpiThreads - 1) / kEpiThreads;
+    double z = 0.0;
+    for (int c = tid * per; c < min(nb, (tid + 1) * per); ++c) z += __ldcg(&a.zsum_part[c]);
+    zred[tid] = z;
+  }
+  epi_sync();
+  if (tid < 32) {
+    // warp-wide finalisation (E <= 64): lane holds experts lane and lane + 32.
+    // Group starts and offsets are exclusive prefix sums; the two loss sums use a
+    // fixed butterfly order, so every lane ends with the same bits on every run.
+    const int e0 = lane, e1 = lane + 32;
+    const int c0v = e0 < E ? sm.tot[e0] : 0, c1v = e1 < E ? sm.tot[e1] : 0;
+    const int g0v = (c0v + kRowAlign - 1) / kRowAlign * kRowAlign;
+    const int g1v = (c1v + kRowAlign - 1) / kRowAlign * kRowAlign;
+    int ic0 = c0v, ig0 = g0v, ic1 = c1v, ig1 = g1v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u0 = __shfl_up_sync(0xffffffffu, ic0, o), w0 = __shfl_up_sync(0xffffffffu, ig0, o);
+      const int u1 = __shfl_up_sync(0xffffffffu, ic1, o), w1 = __shfl_up_sync(0xffffffffu, ig1, o);
+      if (lane >= o) {
+        ic0 += u0;
+        ig0 += w0;
+        ic1 += u1;
+        ig1 += w1;
+      }
+    }
+    const int tc0 = __shfl_sync(0xffffffffu, ic0, 31), tg0 = __shfl_sync(0xffffffffu, ig0, 31);
+    const int tc1 = __shfl_sync(0xffffffffu, ic1, 31), tg1 = __shfl_sync(0xffffffffu, ig1, 31);
+    if (e0 < E) {
+      a.offsets_ws[e0] = ic0 - c0v;
+      a.gs_ws[e0] = ig0 - g0v;
+    }
+    if (e1 < E) {
+      a.offsets_ws[e1] = tc0 + ic1 - c1v;
+      a.gs_ws[e1] = tg0 + ig1 - g1v;
+    }
+    // load balance: E * sum_e (c_e / (T k)) (P_e / T) = E * sum_e c_e P_e / (T^2 k)
+    double lb = (e0 < E ? static_cast<double>(c0v) * sm.tot_p[e0] : 0.0) +
+                (e1 < E ? static_cast<double>(c1v) * sm.tot_p[e1] : 0.0);
+    double zt = 0.0;
+    for (int j = 0; j < kEpiThreads / 32; ++j) zt += zred[lane * (kEpiThreads / 32) + j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lb += __shfl_xor_sync(0xffffffffu, lb, o);
+      zt += __shfl_xor_sync(0xffffffffu, zt, o);
+    }
+    if (lane == 0) {
+      const int off = tc0 + tc1;
+      a.offsets_ws[E] = off;
+      a.gs_ws[E] = tg0 + tg1;
+      const double Td = static_cast<double>(a.T);
+      const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(zt / Td);
+      a.losses_ws[0] = l0;
+      a.losses_ws[1] = l1;
+      if (a.losses_user != nullptr) {
+        a.losses_user[0] = l0;
+        a.losses_user[1] = l1;
+      }
+      if (static_cast<int64_t>(off) != a.T * k) report(a.status, DEV_COUNT_MISMATCH);
+      *a.ticket = 0;
     }
   }
 }
@@ -570,7 +533,7 @@ __device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& s
 // tiles fit on the SMs at once, two with 7-deep rings (one's epilogue then
 // overlaps the other's loads) when there are more tiles than SMs.
 template <int STAGES, int MINB>
-__global__ void __launch_bounds__(kThreads, MINB)
+__global__ void __launch_bounds__(kFusedThreads, MINB)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                      const RArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -586,16 +549,11 @@ __global__ void __launch_bounds__(kThreads, MINB)
   uint32_t* mask = tmem_holder + 4;                          // [kMaxE]
   float* lse_s = reinterpret_cast<float*>(mask + kMaxE);      // [kTile]
   int32_t* s_last = reinterpret_cast<int32_t*>(lse_s + kTile);
+  int32_t* qn = s_last + 1;                                   // queued pairs
   int32_t* tot = s_last + 4;                                  // [kMaxE]
   double* tot_p = reinterpret_cast<double*>(tot + kMaxE);     // [kMaxE]
-  double* zred = tot_p + kMaxE;                               // [128]
-  // once the accumulator is complete the ring is free
-  float* S = reinterpret_cast<float*>(ring);                          // [kTile][kLogitStride] logits
-  float* P = S + kTile * kLogitStride;                                 // [kTile][kMaxE] probabilities
-  int32_t* chosen = reinterpret_cast<int32_t*>(P + kTile * kMaxE);     // [kTile][kMaxTopK]
-  uint32_t* queue = reinterpret_cast<uint32_t*>(ring + 20480);         // [kTile * kMaxE] (token << 8) | expert
-  double* exact = reinterpret_cast<double*>(ring + 20480 + kTile * kMaxE * 4);  // [kTile * kMaxE]
-  int32_t* qn = s_last + 1;                                            // queued pairs
+  // once the accumulator is complete the ring is free: the logits go to its start
+  float* S = reinterpret_cast<float*>(ring + kOffS);          // [kTile][kLogitStride]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = a.d / 64;
@@ -669,9 +627,11 @@ __global__ void __launch_bounds__(kThreads, MINB)
       }
       if (ok) umma_commit(acc_full);
     }
-  } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
-    const int tid = threadIdx.x - 64;  // 0..127
+  }
+  __syncwarp();  // the single-lane roles rejoin their warps
+  {
+    // ------------------------------------------------------------ epilogue (all 16 warps)
+    const int tid = threadIdx.x;
     const int E = a.E, k = a.k;
     if (tid < kMaxE) mask[tid] = 0u;
     if (tid == 0) *qn = 0;
@@ -695,10 +655,10 @@ __global__ void __launch_bounds__(kThreads, MINB)
     tc_fence_before();
     epi_sync();
 
-    const EpiSmem sm{S, P, chosen, queue, exact, qn, mask, lse_s, s_last, tot, tot_p, zred, ring};
+    const EpiSmem sm{ring, mask, lse_s, s_last, qn, tot, tot_p};
     router_epilogue(a, sm, t0, tid, lane);
   }
-  __syncwarp();  // single-lane roles rejoin their warp before the block barrier
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -719,10 +679,9 @@ constexpr int kLogitTile = 128;
 constexpr int kLogitStages = 8;
 constexpr int kLogitStage = kLogitTile * 128 + kMaxE * 128;  // x rows, then W_r rows (per 64-wide K step)
 constexpr size_t kLogitSmem = 1024 + static_cast<size_t>(kLogitStages) * kLogitStage + 1024;
-constexpr int kEpiRing = 64 * 1024;  // shared-memory scratch of the epilogue (and of the last CTA's scan)
+constexpr int kEpiRing = (kEpiScratch + 1023) / 1024 * 1024;  // scratch of the epilogue and the last CTA's scan
 constexpr size_t kEpiSmem = 1024 + kEpiRing + kMiscBytes;
-static_assert(kScanBlock * kMaxE * 8 <= kEpiRing, "scan block fits in the epilogue scratch");
-static_assert(20480 + kTile * kMaxE * 12 <= kEpiRing, "epilogue tiles fit in the scratch");
+static_assert(kEpiScratch <= ring_bytes(16), "the fused kernel's ring holds the epilogue scratch");
 
 __global__ void __launch_bounds__(kThreads, 1)
     router_logits_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
@@ -846,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-__global__ void __launch_bounds__(128, 2) router_epi_kernel(const RArgs a) {
+__global__ void __launch_bounds__(kEpiThreads, 2) router_epi_kernel(const RArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* ring = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -854,15 +813,10 @@ __global__ void __launch_bounds__(128, 2) router_epi_kernel(const RArgs a) {
   uint32_t* mask = reinterpret_cast<uint32_t*>(misc);          // [kMaxE]
   float* lse_s = reinterpret_cast<float*>(mask + kMaxE);      // [kTile]
   int32_t* s_last = reinterpret_cast<int32_t*>(lse_s + kTile);
+  int32_t* qn = s_last + 1;
   int32_t* tot = s_last + 4;                                  // [kMaxE]
   double* tot_p = reinterpret_cast<double*>(tot + kMaxE);     // [kMaxE]
-  double* zred = tot_p + kMaxE;                               // [128]
-  float* S = reinterpret_cast<float*>(ring);
-  float* P = S + kTile * kLogitStride;
-  int32_t* chosen = reinterpret_cast<int32_t*>(P + kTile * kMaxE);
-  uint32_t* queue = reinterpret_cast<uint32_t*>(ring + 20480);
-  double* exact = reinterpret_cast<double*>(ring + 20480 + kTile * kMaxE * 4);
-  int32_t* qn = s_last + 1;
+  float* S = reinterpret_cast<float*>(ring + kOffS);
   const int tid = threadIdx.x, lane = tid & 31;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
   pdl_trigger();
@@ -871,7 +825,7 @@ __global__ void __launch_bounds__(128, 2) router_epi_kernel(const RArgs a) {
   pdl_wait();
   // this tile's logits: the K-range partials (all loads in flight, then summed
   // in a fixed order), plus the offset
-  for (int i = tid; i < kTile * kMaxE; i += 128) {
+  for (int i = tid; i < kTile * kMaxE; i += kEpiThreads) {
     const int r = i / kMaxE, e = i - r * kMaxE;
     float h = -INFINITY;
     if (t0 + r < a.T && e < a.E) {
@@ -889,7 +843,7 @@ __global__ void __launch_bounds__(128, 2) router_epi_kernel(const RArgs a) {
     S[r * kLogitStride + e] = h;
   }
   epi_sync();
-  const EpiSmem sm{S, P, chosen, queue, exact, qn, mask, lse_s, s_last, tot, tot_p, zred, ring};
+  const EpiSmem sm{ring, mask, lse_s, s_last, qn, tot, tot_p};
   router_epilogue(a, sm, t0, tid, lane);
 }
 
@@ -952,7 +906,7 @@ cudaError_t router_tc_impl(const Shape& s, const void* x, const void* w_router, 
   // 41.0 us split; T=4096: 40.9 us against 49.2 us). More tiles than SMs: the
   // split form (T=16384: 87-94 us against 102 us fused).
   if (s.T > 8 && static_cast<int>(grid) <= device_sm_count())
-    return launch_dependent(router_tc_kernel<16, 1>, dim3(grid), dim3(kThreads), smem_bytes(16), st, nullptr, 0, tx,
+    return launch_dependent(router_tc_kernel<16, 1>, dim3(grid), dim3(kFusedThreads), smem_bytes(16), st, nullptr, 0, tx,
                             tw, a);
   CUtensorMap tx128;
   if (!make_map(&tx128, x, false, static_cast<uint64_t>(s.T), s.d, 64, kLogitTile)) return cudaErrorInvalidValue;
@@ -965,14 +919,14 @@ cudaError_t router_tc_impl(const Shape& s, const void* x, const void* w_router, 
   const size_t cap = static_cast<size_t>(s.P) * s.d * s.esize;
   while (ks > 1 && static_cast<size_t>(ks) * s.T * s.E * 4 > cap) --ks;
   if (static_cast<size_t>(ks) * s.T * s.E * 4 > cap)  // tiny layers: the fused kernel
-    return launch_dependent(router_tc_kernel<16, 1>, dim3(grid), dim3(kThreads), smem_bytes(16), st, nullptr, 0, tx,
+    return launch_dependent(router_tc_kernel<16, 1>, dim3(grid), dim3(kFusedThreads), smem_bytes(16), st, nullptr, 0, tx,
                             tw, a);
   a.logit_part = at<float>(ws, L.x_perm);
   a.ksplit = ks;
   e = launch_dependent(router_logits_kernel, dim3(grid_l, static_cast<unsigned>(ks)), dim3(kThreads), kLogitSmem, st,
                        nullptr, 0, tx128, tw, a);
   if (e != cudaSuccess) return e;
-  return launch_dependent(router_epi_kernel, dim3(grid), dim3(128), kEpiSmem, st, nullptr, 0, a);
+  return launch_dependent(router_epi_kernel, dim3(grid), dim3(kEpiThreads), kEpiSmem, st, nullptr, 0, a);
 }
 }  // namespace
 
