@@ -237,12 +237,15 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
  * summed in fp64 from exact products, so the choice is the exact one (equal
  * logits: the lower expert index). Same arguments and results as moe_forward
  * without save_for_backward (counts are not written). moe_forward takes this
- * path by itself for T <= 6 when nothing is saved for the backward (beyond
- * that the layered tensor-core path is as fast), and moe_stack_forward(_trace)
+ * path by itself for T <= 4 when nothing is saved for the backward (beyond
+ * that the layered tensor-core path is faster), and moe_stack_forward(_trace)
  * runs each layer of such a batch as one launch of it with the RMSNorm and the
  * residual add fused.
- * Supported: bf16, T <= 8, E <= 64, T*d*2 and T*k*f*2 bytes each at most
- * 160 KiB; otherwise MOE_ERR_UNSUPPORTED_SHAPE. */
+ * Supported: bf16, T <= 8, E <= 64, d_ff <= 2 d_model, and
+ * max(T*d, T*k*f)*2 + 8*d bytes at most 192 KiB (the staged rows and two
+ * weight stages in shared memory); otherwise MOE_ERR_UNSUPPORTED_SHAPE. The
+ * kernel does nothing when the workspace status word is already set (see
+ * moe_get_device_status). */
 moe_status moe_forward_decode(const moe_config* cfg, const void* x, const void* w_router, const float* router_bias,
                               const void* w_gate_up, const void* w_down, void* y, float* losses, int32_t* topk_idx,
                               float* topk_w, void* ws, size_t ws_bytes, cudaStream_t stream);

@@ -1,9 +1,7 @@
 // The whole MoE layer for a decode-sized batch (T <= 8 tokens) in one
 // persistent cooperative kernel: router, gate/up + SwiGLU, down and combine,
 // optionally with the block's RMSNorm in front and the residual add behind;
-// and a stack of such blocks (up to 16 per launch) in the same kernel, which
-// walks the layers with a grid barrier between one layer's residual update
-// and the next layer's RMSNorm.
+// and a stack of such blocks (up to 16 per launch) in the same kernel.
 //
 // Method: the layer of "Mixture-of-experts LLMs from scratch with OLMoE",
 // section 2 (softmax over all experts, top-k without renormalisation, each
@@ -12,37 +10,43 @@
 // Guide", "Top-8 Softmax Routing Formulation", and its losses ("Router
 // Mechanics & Loss Formulations"). Section 6 of the lesson notes that at a
 // batch of one token the layer reads only the k chosen experts' weights, so
-// decoding is bound by streaming those weights; this kernel exists to stream
-// them with nothing else in the way (one launch, one grid barrier).
+// decoding is bound by streaming those weights; this kernel is built to keep
+// that stream running.
 //
-// One CTA per SM (grid = SM count, cooperative launch, 16 warps):
-//   prologue  every CTA stages the T input rows in shared memory (with the
-//             RMSNorm applied when the input is the fp32 residual).
-//   phase 0   every CTA computes the T*E router logits itself (W_r is read
-//             from L2 by each CTA; no grid barrier): products of bf16 values
-//             are exact in fp32 and are summed in fp32; a token whose k+1
-//             largest logits hold near-equal neighbours has its logits
-//             recomputed as fp64 sums of the exact products, so the top-k
-//             matches an exact computation except for exactly equal logits
-//             (lower index wins). Every CTA takes the same decisions.
-//   phase 0b  every CTA: each expert's rank among a token's logits gives the
-//             top-k at once (no sequential selection); softmax in fp32; the
+// One CTA per SM (grid = SM count, cooperative launch, 16 warps). Per layer:
+//   prologue  every CTA stages the T input rows in shared memory (RMSNorm of
+//             the fp32 residual in fp64 when the input is the residual).
+//   logits    the T*E router logits are spread over the grid, one warp per
+//             (expert, token): fp64 sums of the exact bf16 x bf16 products,
+//             written to the workspace. Grid barrier.
+//   routing   every CTA reads the T*E logits and takes the same decisions:
+//             each expert's rank among a token's logits gives the top-k at
+//             once (equal logits: lower index first); softmax in fp32; the
 //             tokens of each expert as a bit mask; CTA 0 writes the losses,
 //             counts and the optional top-k outputs.
-//   phase 1   one warp per (touched expert, hidden row i): the gate row i and
-//             the up row i stream once from HBM (all of the pair's loads in
-//             flight before any arithmetic) and meet every token that chose
-//             the expert; h = SiLU(g) * u is stored in bf16 (as the grouped
-//             GEMM stores it).
-//   barrier
-//   phase 2   every CTA stages h; one warp per output column c: row c of each
-//             touched expert's down matrix streams once, its dot products with
-//             the tokens' h rows are summed per token in slot order in fp32,
-//             weighted, and written once (bf16 y, or added to the residual).
-// The grid barrier is an arrival counter and a generation word in the
-// workspace; each wait gives up after about a second, records a status and
-// lets the kernel finish. Every single-lane section rejoins its warp
-// (__syncwarp) before a block-wide barrier.
+//   phase 1   this CTA's share of the touched experts' (expert, hidden row)
+//             list, one gate/up row pair per job: the pair meets every token
+//             that chose the expert; h = SiLU(g) * u is stored in bf16 (as the
+//             grouped GEMM stores it). Grid barrier; every CTA copies h of all
+//             slots into shared memory.
+//   phase 2   this CTA's share of the output columns: the down-matrix rows of
+//             each column's touched experts, a few rows per job; their dot
+//             products with the h rows of the expert's tokens; then each
+//             token's slot-ordered weighted sum is written once (bf16 y, or
+//             added to the residual, whose columns this CTA owns).
+// The streaming warps each own two job buffers in shared memory and fetch
+// their jobs with 16-byte asynchronous copies, the next job's bytes in flight
+// while the current one is computed; so no register holds data in flight, and
+// the copies of a warp's first phase-2 jobs go out before the grid barrier.
+// Shares are dealt round-robin by rows (pairs, columns): every SM streams
+// within one row of the same number of bytes, and at any moment the grid
+// reads one contiguous stretch of each weight matrix (per-CTA contiguous
+// ranges, read in lockstep, streamed at about half the rate on B200). The
+// grid barrier is an arrival counter that the launch counts up (barrier j
+// completes at j * grid) and that the last CTA to finish puts back to zero;
+// every wait gives up after about a second, records a status and lets the
+// kernel finish; a launch that finds the status word set does nothing
+// (moe_get_device_status clears it and the counters).
 #include "moe_internal.h"
 #include "sm100.cuh"
 
@@ -53,11 +57,10 @@ constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kDecMaxT = 8;
 constexpr int kDecMaxE = 64;
-constexpr int kDecSlots = kDecMaxT * kMaxTopK;            // (token, slot) pairs
-constexpr size_t kDecActBytes = 160 * 1024;               // staged x, then h
-constexpr size_t kDecMiscBytes = 28 * 1024;
-constexpr size_t kDecSmem = kDecActBytes + kDecMiscBytes;
-constexpr int kDecMaxLayers = 16;                          // layers of a stack per launch
+constexpr int kDecSlots = kDecMaxT * kMaxTopK;  // (token, slot) pairs
+constexpr int kDecMaxLayers = 16;               // layers of a stack per launch
+constexpr size_t kDecSmemCap = 227 * 1024;      // dynamic shared memory of one CTA
+constexpr int kMaxStreamWarps = kDecWarps;     // warps that fetch and compute jobs
 
 // One layer's weights.
 struct DecLayer {
@@ -77,73 +80,85 @@ struct DecArgs {
   float* resid;              // [T, d] fp32 residual (in/out), or null
   __nv_bfloat16* y;          // [T, d] out (null with `resid`)
   __nv_bfloat16* h;          // [T*k, f] workspace
+  double* logits;            // [T, E] workspace
   int32_t* idx_out;          // [n_layers, T, k] or null
   float* w_out;              // [T, k] or null (single layer)
   int32_t* counts;           // [n_layers, E] or null
   float* losses;             // [n_layers, 2] or null
   float* losses_ws;          // [2] workspace copy (of the last layer)
-  unsigned* bar;             // [2] arrival count, generation
+  unsigned* bar;             // [0] grid-barrier arrivals, [1] CTAs finished
   int32_t* status;
+  // shared-memory plan (byte offsets from the start of dynamic shared memory)
+  uint32_t act_off, ps_off, buf_off;
+  uint32_t job_bytes;        // one job buffer: a gate/up row pair, or rows_per_job down rows
+  int rows_per_job;
+  int n_stream;              // streaming warps (0 .. n_stream-1), two job buffers each
 };
 
 struct DecSmem {
   int sel_e[kDecSlots];
   float sel_w[kDecSlots];
-  float ps[kDecWarps][kDecSlots];  // per-warp dot products of one output column
   unsigned tokmask[kDecMaxE];      // bit t: token t chose the expert
   int slot_of[kDecMaxT][kDecMaxE]; // slot of expert e among token t's choices, or -1
   int touched[kDecMaxE];           // experts chosen by some token, ascending
   int n_touched;
-  int ok;
-  double rms[kDecMaxT];             // 1 / sqrt(mean square + eps) of each input row
+  int ok;                          // result of the last grid barrier
+  int abort;                       // a failure is recorded: do nothing
+  unsigned bars;                   // grid barriers passed in this launch
+  double rms[kDecMaxT];            // 1 / sqrt(mean square + eps) of each input row
   double hd[kDecMaxT][kDecMaxE];   // logits (+ offset)
   float p[kDecMaxT][kDecMaxE];
   float lse[kDecMaxT];
   DecLayer layers[kDecMaxLayers];  // the launch's layer table
 };
-static_assert(sizeof(DecSmem) <= kDecMiscBytes, "decode bookkeeping fits");
 
-// Grid-wide barrier (all CTAs co-resident: cooperative launch). Returns false
-// when the wait gave up; the failure is recorded and every CTA then unwinds.
-__device__ bool grid_barrier(unsigned* bar, unsigned n, int32_t* status, int* ok_s) {
-  __syncwarp();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    volatile unsigned* gen = bar + 1;
-    const unsigned g = *gen;
-    __threadfence();
-    int ok = 1;
-    if (atomicAdd(bar, 1u) == n - 1) {
-      atomicExch(bar, 0u);
-      __threadfence();
-      atomicAdd(bar + 1, 1u);
-    } else {
-      const uint64_t t0 = global_timer_ns();
-      uint32_t spins = 0;
-      while (*gen == g) {
-        if (++spins > 1024u) __nanosleep(32);
-        if ((spins & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
-          report(status, DEV_WAIT_TIMEOUT_GRID);
-          ok = 0;
-          break;
-        }
-      }
+// One thread per CTA: arrive at grid barrier number `m.bars + 1` and wait for
+// every CTA (all co-resident: cooperative launch). The arrival is a gpu-scope
+// release, so this CTA's earlier writes (ordered before this thread by the
+// block barrier that precedes the call) are visible to every CTA that passes;
+// the wait polls with relaxed loads and ends with an acquire fence. The count
+// is compared as a wrap-around difference. False when the wait gave up
+// (recorded in the status word).
+__device__ bool grid_sync_thread(DecSmem& m, unsigned* count, int32_t* status) {
+  m.bars += 1;
+  const unsigned target = m.bars * gridDim.x;  // at most 48 barriers of <= 1024 CTAs per launch
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
+  uint64_t t0 = 0;
+  uint32_t spins = 0;
+  while (true) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
+    if (static_cast<int>(v - target) >= 0) break;
+    if (++spins == 64u) t0 = global_timer_ns();
+    if (spins > 64u && (spins & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+      report(status, DEV_WAIT_TIMEOUT_GRID);
+      return false;
     }
-    __threadfence();
-    *ok_s = ok;
   }
-  __syncwarp();  // warp 0 whole again before the block barrier
-  __syncthreads();
-  return *ok_s != 0;
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  return true;
 }
 
+// Grid barrier with every thread of the CTA taking part; the result is the
+// same in every thread.
+__device__ bool grid_barrier(DecSmem& m, const DecArgs& a) {
+  __syncwarp();
+  __syncthreads();
+  if (threadIdx.x == 0) m.ok = grid_sync_thread(m, a.bar, a.status) ? 1 : 0;
+  __syncthreads();
+  return m.ok != 0;
+}
+
+// Eight bf16 values to fp32. A bf16 is the top half of the fp32 with the same
+// value, so the widening is a shift or a mask: integer ALU work at full rate
+// (the conversion instructions run on the quarter-rate pipe that also serves
+// the special functions, and bound this kernel's inner loops).
 __device__ __forceinline__ void bf16x8(const uint4& q, float (&v)[8]) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
-    v[2 * j] = f2.x;
-    v[2 * j + 1] = f2.y;
+    v[2 * j] = __uint_as_float(w[j] << 16);
+    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
   }
 }
 
@@ -159,375 +174,459 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
-// NT: tokens the phase-1 accumulators are sized for (1, 2, 4 or 8; T <= NT).
-// STACK: walks a.n_layers layers of a stack; otherwise exactly one layer (a
-// loop whose trip count the compiler knows keeps the kernel free of register
-// spills; the stack's runtime layer loop costs some).
-template <int NT, bool STACK>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __grid_constant__ DecArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  __nv_bfloat16* act = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // x [T, d], later h [T*k, f]
-  DecSmem& m = *reinterpret_cast<DecSmem*>(smem_raw + kDecActBytes);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = a.T, d = a.d, E = a.E, k = a.k, f = a.f;
-  const int nvd = d / 8, nvf = f / 8;  // 16-byte vectors per row
-  const int gw = blockIdx.x * kDecWarps + warp;
-  const int nw = gridDim.x * kDecWarps;
-  // the layer table in shared memory (indexed by layer below; kernel parameters
-  // are only read at fixed offsets)
+// This CTA's share of the output columns, dealt round-robin (its l-th is
+// CTA + G l; ncols of them), whose down rows (each column's touched experts in
+// turn) form n2 jobs of rows_per_job rows. (The gate/up pairs are dealt by
+// pair_index below.)
+struct Share {
+  int ncols;
+  int rows2, n2;
+};
+
+__device__ Share cta_share(const DecArgs& a, int nt) {
+  Share s;
+  const int G = gridDim.x, c = blockIdx.x;
+  s.ncols = c < a.d ? (a.d - c + G - 1) / G : 0;
+  s.rows2 = s.ncols * nt;
+  s.n2 = (s.rows2 + a.rows_per_job - 1) / a.rows_per_job;
+  return s;
+}
+
+// The gate/up pair of streaming warp w's q-th job.
+__device__ __forceinline__ int pair_index(int SW, int w, int q) {
+  return static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) * (w + SW * q);
+}
+
+// How many jobs streaming warp w has in phase 1.
+__device__ __forceinline__ int pair_jobs(int SW, int w, int P) {
+  const int first = pair_index(SW, w, 0);
+  return first < P ? (P - first + static_cast<int>(gridDim.x) * SW - 1) / (static_cast<int>(gridDim.x) * SW) : 0;
+}
+
+// Output column of this CTA's l-th column.
+__device__ __forceinline__ int cta_col(int l) { return static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) * l; }
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Warp `w`'s job q (its phase-1 pairs w, w + SW, ... then its phase-2 jobs
+// w, w + SW, ...) into `buf`, as 16-byte asynchronous copies by the 32 lanes,
+// then one commit group (also when q is past the warp's last job).
+__device__ __forceinline__ void fetch_job(const DecArgs& a, const DecSmem& m, const DecLayer& Ly, const Share& sh,
+                                          int nt, int w, int lane, int c1, int c2, int q, unsigned char* buf) {
+  const int SW = a.n_stream;
+  if (q < c1) {
+    const int p = pair_index(SW, w, q);
+    const int u = p / a.f, i = p - u * a.f;
+    const __nv_bfloat16* g = Ly.wgu + (static_cast<int64_t>(m.touched[u]) * 2 * a.f + i) * a.d;
+    const __nv_bfloat16* up = g + static_cast<int64_t>(a.f) * a.d;
+    const int nvd = a.d / 8;
+    for (int c = lane; c < 2 * nvd; c += 32)
+      cp_async16(buf + 16 * c, c < nvd ? g + 8 * c : up + 8 * (c - nvd));
+  } else if (q < c1 + c2) {
+    const int r0 = (w + SW * (q - c1)) * a.rows_per_job;
+    const int nr = min(a.rows_per_job, sh.rows2 - r0);
+    const int nvf = a.f / 8;
+    int cl = r0 / nt, u = r0 - cl * nt;  // the row's column (of this CTA's) and touched-expert index
+    for (int rr = 0; rr < nr; ++rr) {
+      const __nv_bfloat16* row = Ly.wd + (static_cast<int64_t>(m.touched[u]) * a.d + cta_col(cl)) * a.f;
+      unsigned char* dst = buf + static_cast<size_t>(rr) * nvf * 16;
+      for (int v = lane; v < nvf; v += 32) cp_async16(dst + 16 * v, row + 8 * v);
+      if (++u == nt) {
+        u = 0;
+        ++cl;
+      }
+    }
+  }
+  cp_async_commit();
+}
+
+// Logit task q: expert q / T, token q % T, as an fp64 sum of the exact
+// products (a bf16 x bf16 product is exact in fp32), lane l taking elements
+// 8l + 256i, then a fixed reduction tree; written to the workspace. One warp.
+__device__ __forceinline__ void logit_task(const DecArgs& a, const DecLayer& Ly, const __nv_bfloat16* act, int q,
+                                           int lane) {
+  const int T = a.T, d = a.d, E = a.E, nvd = d / 8;
+  const int e = q / T, t = q - e * T;
+  const uint4* wrow = reinterpret_cast<const uint4*>(Ly.wr + static_cast<int64_t>(e) * d);
+  const uint4* xrow = reinterpret_cast<const uint4*>(act + static_cast<int64_t>(t) * d);
+  double acc = 0.0;
+  for (int v0 = 0; v0 < nvd; v0 += 32 * 8) {
+    uint4 wq[8];
 #pragma unroll
-  for (int l = 0; l < kDecMaxLayers; ++l)
-    if (tid == l) m.layers[l] = a.layer[l];
+    for (int j = 0; j < 8; ++j) {
+      const int v = v0 + j * 32 + lane;
+      if (v < nvd) wq[j] = __ldg(wrow + v);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int v = v0 + j * 32 + lane;
+      if (v < nvd) {
+        float wv[8], xv[8];
+        bf16x8(wq[j], wv);
+        bf16x8(xrow[v], xv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc += static_cast<double>(xv[i] * wv[i]);
+      }
+    }
+  }
+  acc = warp_sum_d(acc);
+  if (lane == 0) a.logits[t * E + e] = acc + (Ly.bias != nullptr ? static_cast<double>(Ly.bias[e]) : 0.0);
+}
+
+// Phase-1 job: gate/up row pair p (in `buf`) meets every token of the pair's
+// expert; h = SiLU(g) * u in bf16.
+template <int NT>
+__device__ __forceinline__ void pair_job(const DecArgs& a, const DecSmem& m, const __nv_bfloat16* act,
+                                         const unsigned char* buf, int p, int lane) {
+  const int d = a.d, k = a.k, f = a.f, nvd = d / 8;
+  const int u = p / f, i = p - u * f;
+  const int e = m.touched[u];
+  const unsigned tm = m.tokmask[e];
+  const uint4* g4 = reinterpret_cast<const uint4*>(buf);
+  const uint4* u4 = g4 + nvd;
+  const uint4* x4 = reinterpret_cast<const uint4*>(act);
+  float ag[NT], au[NT];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) ag[t] = au[t] = 0.f;
+  for (int v = lane; v < nvd; v += 32) {
+    float gv[8], uv[8];
+    bf16x8(g4[v], gv);
+    bf16x8(u4[v], uv);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      if ((tm >> t) & 1u) {
+        float xv[8];
+        bf16x8(x4[t * nvd + v], xv);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          ag[t] = fmaf(gv[c], xv[c], ag[t]);
+          au[t] = fmaf(uv[c], xv[c], au[t]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    if ((tm >> t) & 1u) {
+      const float g = warp_sum(ag[t]), uu = warp_sum(au[t]);
+      if (lane == 0)
+        a.h[static_cast<int64_t>(t * k + m.slot_of[t][e]) * f + i] = __float2bfloat16_rn(silu_fast(g) * uu);
+    }
+  }
+}
+
+// Phase-2 job g of this CTA (down rows g * rows_per_job ..., in `buf`): each
+// row's dot products with the h rows (shared memory) of its expert's tokens.
+__device__ __forceinline__ void down_job(const DecArgs& a, const DecSmem& m, const Share& sh, int nt,
+                                         const __nv_bfloat16* act, float* ps, const unsigned char* buf, int g,
+                                         int lane) {
+  const int k = a.k, nvf = a.f / 8, TK = a.T * k;
+  const int r0 = g * a.rows_per_job;
+  const int nr = min(a.rows_per_job, sh.rows2 - r0);
+  const uint4* h4 = reinterpret_cast<const uint4*>(act);
+  int cl = r0 / nt, u = r0 - cl * nt;  // the row's column (of this CTA's) and touched-expert index
+  for (int rr = 0; rr < nr; ++rr) {
+    const int e = m.touched[u];
+    const uint4* w4 = reinterpret_cast<const uint4*>(buf) + rr * nvf;
+    unsigned tm = m.tokmask[e];
+    while (tm != 0u) {
+      const int t = __ffs(tm) - 1;
+      tm &= tm - 1u;
+      const int slot = t * k + m.slot_of[t][e];
+      float acc = 0.f;
+      for (int v = lane; v < nvf; v += 32) {
+        float wv[8], hv[8];
+        bf16x8(w4[v], wv);
+        bf16x8(h4[slot * nvf + v], hv);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc = fmaf(wv[c], hv[c], acc);
+      }
+      acc = warp_sum(acc);
+      if (lane == 0) ps[cl * TK + slot] = acc;
+    }
+    if (++u == nt) {
+      u = 0;
+      ++cl;
+    }
+  }
+}
+
+// NT: tokens the phase-1 accumulators are sized for (1, 2, 4 or 8; T <= NT).
+template <int NT>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __grid_constant__ DecArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  DecSmem& m = *reinterpret_cast<DecSmem*>(smem_raw);
+  __nv_bfloat16* act = reinterpret_cast<__nv_bfloat16*>(smem_raw + a.act_off);  // x [T, d], later h [T*k, f]
+  float* ps = reinterpret_cast<float*>(smem_raw + a.ps_off);  // [ncols][T*k] down-row dot products
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = a.T, d = a.d, E = a.E, k = a.k;
+  const int TK = T * k;
+  const int nvd = d / 8, nvf = a.f / 8;  // 16-byte vectors per row
+  const int G = gridDim.x;
+  const int SW = a.n_stream;
+  unsigned char* buf0 = smem_raw + a.buf_off + static_cast<size_t>(2 * warp) * a.job_bytes;
+  unsigned char* buf1 = buf0 + a.job_bytes;
+
+  if (tid == 0) {
+    m.abort = *reinterpret_cast<volatile int32_t*>(a.status) != 0 ? 1 : 0;
+    m.bars = 0;
+  }
+  if (tid < kDecMaxLayers) m.layers[tid] = a.layer[tid];
   __syncthreads();
+  if (m.abort != 0) return;  // a failure is recorded: the counters may be stale
 
-  const int n_layers = STACK ? a.n_layers : 1;
 #pragma unroll 1
-  for (int l = 0; l < n_layers; ++l) {
-  // a layer of a stack reads the residual the previous layer completed
-  if (l > 0 && !grid_barrier(a.bar, gridDim.x, a.status, &m.ok)) return;
-  const DecLayer Ly = m.layers[l];
-  int32_t* const idx_out = a.idx_out != nullptr ? a.idx_out + static_cast<int64_t>(l) * T * k : nullptr;
-  int32_t* const counts = a.counts != nullptr ? a.counts + static_cast<int64_t>(l) * E : nullptr;
-  float* const losses = a.losses != nullptr ? a.losses + 2 * l : nullptr;
+  for (int l = 0; l < a.n_layers; ++l) {
+    const DecLayer& Ly = m.layers[l];
+    // this CTA's logit tasks: task q = warp * G + CTA, expert q / T, token q % T
+    const int q = warp * G + blockIdx.x;
+    const bool has_task = q < T * E;
+    // a layer of a stack reads the residual the previous layer completed
+    if (l > 0 && !grid_barrier(m, a)) return;
+    int32_t* const idx_out = a.idx_out != nullptr ? a.idx_out + static_cast<int64_t>(l) * TK : nullptr;
+    int32_t* const counts = a.counts != nullptr ? a.counts + static_cast<int64_t>(l) * E : nullptr;
+    float* const losses = a.losses != nullptr ? a.losses + 2 * l : nullptr;
 
-  // ---- prologue: the T input rows, bf16, in shared memory
-  if (a.resid != nullptr) {
-    if (warp < T) {  // RMSNorm (unit weight) of token `warp` in fp64, mean of squares in a fixed order
-      const float* r = a.resid + static_cast<int64_t>(warp) * d;
-      double ss = 0.0;
-      for (int i = lane; i < d; i += 32) ss = fma(static_cast<double>(r[i]), static_cast<double>(r[i]), ss);
-      ss = warp_sum_d(ss);
-      if (lane == 0) m.rms[warp] = 1.0 / sqrt(ss / static_cast<double>(d) + a.eps);
+    // ---- prologue: the T input rows, bf16, in shared memory
+    if (a.resid != nullptr) {
+      if (warp < T) {  // RMSNorm (unit weight) of token `warp` in fp64, mean of squares in a fixed order
+        const float* r = a.resid + static_cast<int64_t>(warp) * d;
+        double ss = 0.0;
+        for (int i = lane; i < d; i += 32) {
+          const double v = static_cast<double>(__ldcg(r + i));
+          ss = fma(v, v, ss);
+        }
+        ss = warp_sum_d(ss);
+        if (lane == 0) m.rms[warp] = 1.0 / sqrt(ss / static_cast<double>(d) + a.eps);
+        __syncwarp();
+      }
+      __syncthreads();
+      // the fp64 value rounded to fp32, then to bf16 (as the separate RMSNorm kernel does)
+      for (int t = 0; t < T; ++t)
+        for (int i = tid; i < d; i += kDecThreads)
+          act[t * d + i] = __float2bfloat16_rn(
+              static_cast<float>(static_cast<double>(__ldcg(a.resid + static_cast<int64_t>(t) * d + i)) * m.rms[t]));
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(a.x);
+      uint4* dst = reinterpret_cast<uint4*>(act);
+      for (int i = tid; i < T * nvd; i += kDecThreads) dst[i] = __ldg(src + i);
+    }
+    if (tid < kDecMaxE) m.tokmask[tid] = 0u;
+    if (tid < kDecSlots) m.sel_e[tid] = 0;  // defined even if non-finite logits leave a slot unranked
+    for (int i = tid; i < (d / G + 1) * TK; i += kDecThreads) ps[i] = 0.f;
+    __syncthreads();
+
+    // ---- logits: fp64 sums of the exact products (a bf16 x bf16 product is
+    //      exact in fp32), lane l taking elements 8l + 256i; fixed reduction tree
+    if (has_task) logit_task(a, Ly, act, q, lane);
+    if (!grid_barrier(m, a)) return;
+    for (int i = tid; i < T * E; i += kDecThreads) m.hd[i / E][i % E] = __ldcg(a.logits + i);
+    __syncthreads();
+
+    // ---- routing (every CTA): warp t takes token t; lane l holds experts l, l + 32
+    if (warp < T) {
+      const int t = warp;
+      const int e0 = lane, e1 = lane + 32;
+      const double h0 = e0 < E ? m.hd[t][e0] : -INFINITY;
+      const double h1 = e1 < E ? m.hd[t][e1] : -INFINITY;
+      // rank by (logit descending, index ascending): the experts ranked below k are the choice
+      int r0 = 0, r1 = 0;
+      for (int e = 0; e < E; ++e) {
+        const double v = m.hd[t][e];
+        r0 += (v > h0 || (v == h0 && e < e0)) ? 1 : 0;
+        r1 += (v > h1 || (v == h1 && e < e1)) ? 1 : 0;
+      }
+      if (e0 < E) {
+        m.slot_of[t][e0] = r0 < k ? r0 : -1;
+        if (r0 < k) {
+          m.sel_e[t * k + r0] = e0;
+          atomicOr(&m.tokmask[e0], 1u << t);
+        }
+      }
+      if (e1 < E) {
+        m.slot_of[t][e1] = r1 < k ? r1 : -1;
+        if (r1 < k) {
+          m.sel_e[t * k + r1] = e1;
+          atomicOr(&m.tokmask[e1], 1u << t);
+        }
+      }
+      // softmax over all experts in fp32 from the logits
+      double mx = fmax(h0, h1);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float x0 = e0 < E ? expf(static_cast<float>(h0 - mx)) : 0.f;
+      const float x1 = e1 < E ? expf(static_cast<float>(h1 - mx)) : 0.f;
+      const float sum = warp_sum(x0 + x1);
+      if (e0 < E) m.p[t][e0] = x0 / sum;
+      if (e1 < E) m.p[t][e1] = x1 / sum;
+      if (lane == 0) m.lse[t] = static_cast<float>(mx) + logf(sum);
+      __syncwarp();
+      if (lane == 0) {  // weights in slot order (renormalised: over the k chosen, summed in slot order)
+        float den = 0.f;
+        for (int j = 0; j < k; ++j) den += m.p[t][m.sel_e[t * k + j]];
+        for (int j = 0; j < k; ++j) {
+          const int e = m.sel_e[t * k + j];
+          const float w = a.renorm ? m.p[t][e] / den : m.p[t][e];
+          m.sel_w[t * k + j] = w;
+          if (blockIdx.x == 0) {
+            if (idx_out != nullptr) idx_out[t * k + j] = e;
+            if (a.w_out != nullptr) a.w_out[t * k + j] = w;
+          }
+        }
+      }
       __syncwarp();
     }
     __syncthreads();
-    // the fp64 value rounded to fp32, then to bf16 (as the separate RMSNorm kernel does)
-    for (int i = tid; i < T * d; i += kDecThreads)
-      act[i] = __float2bfloat16_rn(static_cast<float>(static_cast<double>(a.resid[i]) * m.rms[i / d]));
-  } else {
-    const uint4* src = reinterpret_cast<const uint4*>(a.x);
-    uint4* dst = reinterpret_cast<uint4*>(act);
-    for (int i = tid; i < T * nvd; i += kDecThreads) dst[i] = __ldg(src + i);
-  }
-  if (tid < kDecMaxE) m.tokmask[tid] = 0u;
-  if (tid < kDecSlots) m.sel_e[tid] = 0;  // defined even if non-finite logits leave a slot unranked
-  __syncthreads();
-
-  // ---- phase 0 (every CTA, no grid barrier): the T*E router logits. Warp w
-  //      takes experts w, w + 16, ...; each W_r row is read once into registers
-  //      and meets every token. bf16 x bf16 products are exact in fp32 and are
-  //      summed in fp32 here; every CTA sums in the same order, so every CTA
-  //      holds the same values and takes the same decisions.
-  for (int e = warp; e < E; e += kDecWarps) {
-    const uint4* wrow = reinterpret_cast<const uint4*>(Ly.wr + static_cast<int64_t>(e) * d);
-    float acc[NT];
-#pragma unroll
-    for (int q = 0; q < NT; ++q) acc[q] = 0.f;
-    for (int v0 = 0; v0 < nvd; v0 += 32 * 8) {
-      uint4 wq[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int v = v0 + j * 32 + lane;
-        if (v < nvd) wq[j] = __ldg(wrow + v);
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int v = v0 + j * 32 + lane;
-        if (v < nvd) {
-          float wv[8];
-          bf16x8(wq[j], wv);
-#pragma unroll
-          for (int q = 0; q < NT; ++q) {
-            if (q < T) {
-              float xv[8];
-              bf16x8(reinterpret_cast<const uint4*>(act + static_cast<int64_t>(q) * d)[v], xv);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) acc[q] = fmaf(xv[i], wv[i], acc[q]);
-            }
-          }
+    if (warp == 0) {  // the touched experts, ascending; CTA 0: counts and losses
+      int base = 0;
+      double lb = 0.0;
+      for (int c = 0; c < E; c += 32) {
+        const int e = c + lane;
+        const bool on = e < E && m.tokmask[e] != 0u;
+        const unsigned b = __ballot_sync(0xffffffffu, on);
+        if (on) m.touched[base + __popc(b & ((1u << lane) - 1u))] = e;
+        base += __popc(b);
+        if (blockIdx.x == 0 && e < E) {
+          const int ce = __popc(m.tokmask[e]);
+          double pe = 0.0;
+          for (int t = 0; t < T; ++t) pe += m.p[t][e];
+          lb += static_cast<double>(ce) * pe;
+          if (counts != nullptr) counts[e] = ce;
         }
       }
-    }
-#pragma unroll
-    for (int q = 0; q < NT; ++q) {
-      if (q < T) {
-        const float h = warp_sum(acc[q]);
-        if (lane == 0) m.hd[q][e] = static_cast<double>(h) + (Ly.bias != nullptr ? static_cast<double>(Ly.bias[e]) : 0.0);
-      }
-    }
-  }
-  __syncthreads();
-  // The choice must be the exact one: a token whose k+1 largest fp32 logits
-  // hold two values closer than 2e-4 * max(1, |h|) (far above the error of a
-  // 2048-term fp32 sum of exact products) has all E logits recomputed exactly
-  // (fp64 sums of the exact products), lane l taking experts l and l + 32.
-  if (warp < T) {
-    const int t = warp;
-    const int e0 = lane, e1 = lane + 32;
-    const double h0 = e0 < E ? m.hd[t][e0] : -INFINITY, h1 = e1 < E ? m.hd[t][e1] : -INFINITY;
-    int r0 = 0, r1 = 0;
-    for (int e = 0; e < E; ++e) {
-      const double v = m.hd[t][e];
-      r0 += (v > h0 || (v == h0 && e < e0)) ? 1 : 0;
-      r1 += (v > h1 || (v == h1 && e < e1)) ? 1 : 0;
-    }
-    bool near = false;
-    for (int e = 0; e < E; ++e) {
-      const double v = m.hd[t][e];
-      const double g = 2e-4 * fmax(1.0, fabs(v));
-      if (e0 < E && e != e0 && r0 <= k && fabs(v - h0) < g) near = true;
-      if (e1 < E && e != e1 && r1 <= k && fabs(v - h1) < g) near = true;
-    }
-    // (a near value may rank below k + 1 itself: then it is within the gap of
-    // a ranked one, which the loop above finds from that ranked lane)
-    if (__any_sync(0xffffffffu, near)) {
-      const uint4* xrow = reinterpret_cast<const uint4*>(act + static_cast<int64_t>(t) * d);
-      double ex[2] = {0.0, 0.0};
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int e = lane + 32 * u;
-        if (e < E) {
-          const uint4* wrow = reinterpret_cast<const uint4*>(Ly.wr + static_cast<int64_t>(e) * d);
-          double acc = 0.0;
-          for (int v = 0; v < nvd; ++v) {
-            float xv[8], wv[8];
-            bf16x8(xrow[v], xv);
-            bf16x8(__ldg(wrow + v), wv);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc += static_cast<double>(xv[i] * wv[i]);  // exact product
+      if (lane == 0) m.n_touched = base;
+      if (blockIdx.x == 0) {  // E * sum_e (c_e / (T k)) (P_e / T), and the mean of lse^2
+        lb = warp_sum_d(lb);
+        if (lane == 0) {
+          double z = 0.0;
+          for (int t = 0; t < T; ++t) z += static_cast<double>(m.lse[t]) * m.lse[t];
+          const double Td = static_cast<double>(T);
+          const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(z / Td);
+          a.losses_ws[0] = l0;
+          a.losses_ws[1] = l1;
+          if (losses != nullptr) {
+            losses[0] = l0;
+            losses[1] = l1;
           }
-          ex[u] = acc + (Ly.bias != nullptr ? static_cast<double>(Ly.bias[e]) : 0.0);
         }
       }
       __syncwarp();
-      if (e0 < E) m.hd[t][e0] = ex[0];
-      if (e1 < E) m.hd[t][e1] = ex[1];
     }
-    __syncwarp();
-  }
-  __syncthreads();
+    __syncthreads();
+    const int nt = m.n_touched;
+    const Share sh = cta_share(a, nt);
 
-  // ---- phase 0b (every CTA): warp t takes token t; lane l holds experts l, l + 32
-  if (warp < T) {
-    const int t = warp;
-    const int e0 = lane, e1 = lane + 32;
-    const double h0 = e0 < E ? m.hd[t][e0] : -INFINITY;
-    const double h1 = e1 < E ? m.hd[t][e1] : -INFINITY;
-    // rank by (logit descending, index ascending): the experts ranked below k are the choice
-    int r0 = 0, r1 = 0;
-    for (int e = 0; e < E; ++e) {
-      const double v = m.hd[t][e];
-      r0 += (v > h0 || (v == h0 && e < e0)) ? 1 : 0;
-      r1 += (v > h1 || (v == h1 && e < e1)) ? 1 : 0;
-    }
-    if (e0 < E) {
-      m.slot_of[t][e0] = r0 < k ? r0 : -1;
-      if (r0 < k) {
-        m.sel_e[t * k + r0] = e0;
-        atomicOr(&m.tokmask[e0], 1u << t);
+    // this warp's jobs: phase-1 pairs warp, warp + SW, ... then phase-2 jobs likewise
+    const bool streams = warp < SW;
+    const int c1 = streams ? pair_jobs(SW, warp, nt * a.f) : 0;
+    const int c2 = streams && warp < sh.n2 ? (sh.n2 - warp + SW - 1) / SW : 0;
+    if (streams) {
+      fetch_job(a, m, Ly, sh, nt, warp, lane, c1, c2, 0, buf0);
+      fetch_job(a, m, Ly, sh, nt, warp, lane, c1, c2, 1, buf1);
+      // ---- phase 1: the next job's copies in flight while this one is computed
+      for (int qq = 0; qq < c1; ++qq) {
+        unsigned char* b = (qq & 1) ? buf1 : buf0;
+        cp_async_wait<1>();
+        __syncwarp();
+        pair_job<NT>(a, m, act, b, pair_index(SW, warp, qq), lane);
+        __syncwarp();
+        fetch_job(a, m, Ly, sh, nt, warp, lane, c1, c2, qq + 2, b);
       }
     }
-    if (e1 < E) {
-      m.slot_of[t][e1] = r1 < k ? r1 : -1;
-      if (r1 < k) {
-        m.sel_e[t * k + r1] = e1;
-        atomicOr(&m.tokmask[e1], 1u << t);
-      }
+    // every CTA's h is written before any CTA reads it
+    if (!grid_barrier(m, a)) {
+      cp_async_wait<0>();  // no copy in flight when the CTA leaves
+      return;
     }
-    // softmax over all experts in fp32 from the exact logits
-    double mx = fmax(h0, h1);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float x0 = e0 < E ? expf(static_cast<float>(h0 - mx)) : 0.f;
-    const float x1 = e1 < E ? expf(static_cast<float>(h1 - mx)) : 0.f;
-    const float sum = warp_sum(x0 + x1);
-    if (e0 < E) m.p[t][e0] = x0 / sum;
-    if (e1 < E) m.p[t][e1] = x1 / sum;
-    if (lane == 0) m.lse[t] = static_cast<float>(mx) + logf(sum);
-    __syncwarp();
-    if (lane == 0) {  // weights in slot order (renormalised: over the k chosen, summed in slot order)
-      float den = 0.f;
-      for (int j = 0; j < k; ++j) den += m.p[t][m.sel_e[t * k + j]];
-      for (int j = 0; j < k; ++j) {
-        const int e = m.sel_e[t * k + j];
-        const float w = a.renorm ? m.p[t][e] / den : m.p[t][e];
-        m.sel_w[t * k + j] = w;
-        if (blockIdx.x == 0) {
-          if (idx_out != nullptr) idx_out[t * k + j] = e;
-          if (a.w_out != nullptr) a.w_out[t * k + j] = w;
-        }
-      }
+    {  // h of all slots into shared memory (x is dead)
+      const uint4* src = reinterpret_cast<const uint4*>(a.h);
+      uint4* dst = reinterpret_cast<uint4*>(act);
+      for (int i = tid; i < TK * nvf; i += kDecThreads) dst[i] = __ldcg(src + i);
     }
-    __syncwarp();
-  }
-  __syncthreads();
-  if (warp == 0) {  // the touched experts, ascending; CTA 0: counts and losses
-    int base = 0;
-    double lb = 0.0;
-    for (int c = 0; c < E; c += 32) {
-      const int e = c + lane;
-      const bool on = e < E && m.tokmask[e] != 0u;
-      const unsigned b = __ballot_sync(0xffffffffu, on);
-      if (on) m.touched[base + __popc(b & ((1u << lane) - 1u))] = e;
-      base += __popc(b);
-      if (blockIdx.x == 0 && e < E) {
-        const int ce = __popc(m.tokmask[e]);
-        double pe = 0.0;
-        for (int t = 0; t < T; ++t) pe += m.p[t][e];
-        lb += static_cast<double>(ce) * pe;
-        if (counts != nullptr) counts[e] = ce;
-      }
-    }
-    if (lane == 0) m.n_touched = base;
-    if (blockIdx.x == 0) {  // E * sum_e (c_e / (T k)) (P_e / T), and the mean of lse^2
-      lb = warp_sum_d(lb);
-      if (lane == 0) {
-        double z = 0.0;
-        for (int t = 0; t < T; ++t) z += static_cast<double>(m.lse[t]) * m.lse[t];
-        const double Td = static_cast<double>(T);
-        const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(z / Td);
-        a.losses_ws[0] = l0;
-        a.losses_ws[1] = l1;
-        if (losses != nullptr) {
-          losses[0] = l0;
-          losses[1] = l1;
-        }
-      }
-    }
-    __syncwarp();
-  }
-  __syncthreads();
-  const int nt = m.n_touched;
+    __syncthreads();
 
-  // ---- phase 1: gate/up rows of the touched experts, a warp per (expert, row);
-  //      the whole row pair's loads are in flight before any arithmetic
-  for (int item = gw; item < nt * f; item += nw) {
-    const int u = item / f, i = item - u * f;
-    const int e = m.touched[u];
-    const unsigned tmask = m.tokmask[e];
-    const uint4* grow = reinterpret_cast<const uint4*>(Ly.wgu + (static_cast<int64_t>(e) * 2 * f + i) * d);
-    const uint4* urow = grow + static_cast<int64_t>(f) * nvd;
-    float ag[NT], au[NT];
-#pragma unroll
-    for (int q = 0; q < NT; ++q) ag[q] = au[q] = 0.f;
-    for (int v0 = 0; v0 < nvd; v0 += 32 * 8) {
-      uint4 gq[8], uq[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int v = v0 + j * 32 + lane;
-        if (v < nvd) {
-          gq[j] = __ldg(grow + v);
-          uq[j] = __ldg(urow + v);
-        }
+    // ---- phase 2
+    if (streams) {
+      for (int qq = c1; qq < c1 + c2; ++qq) {
+        unsigned char* b = (qq & 1) ? buf1 : buf0;
+        cp_async_wait<1>();
+        __syncwarp();
+        down_job(a, m, sh, nt, act, ps, b, warp + SW * (qq - c1), lane);
+        __syncwarp();
+        fetch_job(a, m, Ly, sh, nt, warp, lane, c1, c2, qq + 2, b);
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int v = v0 + j * 32 + lane;
-        if (v < nvd) {
-          float gv[8], uv[8];
-          bf16x8(gq[j], gv);
-          bf16x8(uq[j], uv);
-#pragma unroll
-          for (int q = 0; q < NT; ++q) {
-            if ((tmask >> q) & 1u) {
-              float xv[8];
-              bf16x8(reinterpret_cast<const uint4*>(act + static_cast<int64_t>(q) * d)[v], xv);
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                ag[q] = fmaf(gv[c], xv[c], ag[q]);
-                au[q] = fmaf(uv[c], xv[c], au[q]);
-              }
-            }
-          }
-        }
-      }
+      cp_async_wait<0>();
     }
-#pragma unroll
-    for (int q = 0; q < NT; ++q) {
-      if ((tmask >> q) & 1u) {
-        const float g = warp_sum(ag[q]), uu = warp_sum(au[q]);
-        if (lane == 0) {
-          const int slot = q * k + m.slot_of[q][e];
-          a.h[static_cast<int64_t>(slot) * f + i] = __float2bfloat16_rn(silu_fast(g) * uu);
-        }
-      }
-    }
-  }
-  if (!grid_barrier(a.bar, gridDim.x, a.status, &m.ok)) return;
-
-  // ---- phase 2: h in shared memory, then a warp per output column
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(a.h);
-    uint4* dst = reinterpret_cast<uint4*>(act);
-    for (int i = tid; i < T * k * nvf; i += kDecThreads) dst[i] = __ldcg(src + i);
-  }
-  __syncthreads();
-  for (int c = gw; c < d; c += nw) {
-    for (int u0 = 0; u0 < nt; u0 += 4) {
-      uint4 wq[4][4];  // four experts' rows, four 16-byte vectors per lane at a time
-      for (int v0 = 0; v0 < nvf; v0 += 32 * 4) {
-#pragma unroll
-        for (int uu = 0; uu < 4; ++uu) {
-          if (u0 + uu < nt) {
-            const uint4* row =
-                reinterpret_cast<const uint4*>(Ly.wd + (static_cast<int64_t>(m.touched[u0 + uu]) * d + c) * f);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int v = v0 + j * 32 + lane;
-              if (v < nvf) wq[uu][j] = __ldg(row + v);
-            }
-          }
-        }
-#pragma unroll
-        for (int uu = 0; uu < 4; ++uu) {
-          if (u0 + uu < nt) {
-            const int e = m.touched[u0 + uu];
-            unsigned tm = m.tokmask[e];
-            while (tm != 0u) {
-              const int t = __ffs(tm) - 1;
-              tm &= tm - 1u;
-              const int slot = t * k + m.slot_of[t][e];
-              const uint4* hrow = reinterpret_cast<const uint4*>(act + static_cast<int64_t>(slot) * f);
-              float acc = 0.f;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int v = v0 + j * 32 + lane;
-                if (v < nvf) {
-                  float wv[8], hv[8];
-                  bf16x8(wq[uu][j], wv);
-                  bf16x8(hrow[v], hv);
-#pragma unroll
-                  for (int cc = 0; cc < 8; ++cc) acc = fmaf(wv[cc], hv[cc], acc);
-                }
-              }
-              acc = warp_sum(acc);
-              if (lane == 0) m.ps[warp][slot] = (v0 == 0 ? 0.f : m.ps[warp][slot]) + acc;
-            }
-          }
-        }
-      }
-    }
-    __syncwarp();
-    if (lane < T) {  // token `lane`: weighted sum over its slots, in slot order
+    __syncthreads();
+    // each (column, token): the weighted sum over the token's slots in slot order
+    for (int it = tid; it < sh.ncols * T; it += kDecThreads) {
+      const int t = it / sh.ncols, cl = it - t * sh.ncols;
       float acc = 0.f;
-      for (int j = 0; j < k; ++j) acc = fmaf(m.sel_w[lane * k + j], m.ps[warp][lane * k + j], acc);
-      const int64_t o = static_cast<int64_t>(lane) * d + c;
+      for (int j = 0; j < k; ++j) acc = fmaf(m.sel_w[t * k + j], ps[cl * TK + t * k + j], acc);
+      const int64_t o = static_cast<int64_t>(t) * d + cta_col(cl);
       if (a.resid != nullptr)
-        a.resid[o] += acc;
+        a.resid[o] = __ldcg(a.resid + o) + acc;
       else
         a.y[o] = __float2bfloat16_rn(acc);
     }
-    __syncwarp();
-  }
+    __syncthreads();
   }  // layers
+
+  // every CTA has passed its last grid barrier: the last one out puts the counters back to zero
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(a.bar + 1, 1u) == static_cast<unsigned>(G) - 1u) {
+      a.bar[0] = 0u;
+      a.bar[1] = 0u;
+    }
+  }
+}
+
+// Shared-memory plan for T tokens on a grid of G CTAs: bookkeeping, the
+// activation rows (x, later h), the per-column dot products, and two job
+// buffers for as many streaming warps (up to 16) as fit.
+struct DecPlan {
+  uint32_t act_off, ps_off, buf_off, job_bytes;
+  int rows_per_job, n_stream;
+  size_t smem;
+};
+
+size_t align128(size_t v) { return (v + 127) / 128 * 128; }
+
+bool decode_plan(const Shape& s, int G, DecPlan* p) {
+  const size_t misc = align128(sizeof(DecSmem));
+  const size_t act = align128(std::max(static_cast<size_t>(s.T) * s.d * 2, static_cast<size_t>(s.T) * s.k * s.f * 2));
+  const size_t ps = align128(static_cast<size_t>(s.d / G + 1) * s.T * s.k * 4);
+  const size_t jb = align128(std::max(static_cast<size_t>(s.d) * 4, static_cast<size_t>(s.f) * 2));
+  if (misc + act + ps + 2 * jb > kDecSmemCap) return false;
+  const size_t sw = std::min<size_t>(kMaxStreamWarps, (kDecSmemCap - misc - act - ps) / (2 * jb));
+  p->act_off = static_cast<uint32_t>(misc);
+  p->ps_off = static_cast<uint32_t>(misc + act);
+  p->buf_off = static_cast<uint32_t>(misc + act + ps);
+  p->job_bytes = static_cast<uint32_t>(jb);
+  p->rows_per_job = static_cast<int>(jb / (static_cast<size_t>(s.f) * 2));
+  p->n_stream = static_cast<int>(sw);
+  p->smem = misc + act + ps + 2 * sw * jb;
+  return true;
 }
 
 }  // namespace
 
 bool decode_supported(const Shape& s) {
-  if (s.fp32 || s.T > kDecMaxT || s.E > kDecMaxE || s.k > kMaxTopK) return false;
-  const size_t x_bytes = static_cast<size_t>(s.T) * s.d * 2, h_bytes = static_cast<size_t>(s.T) * s.k * s.f * 2;
-  return x_bytes <= kDecActBytes && h_bytes <= kDecActBytes;
+  if (s.fp32 || s.T < 1 || s.T > kDecMaxT || s.E > kDecMaxE || s.k > kMaxTopK) return false;
+  if (s.d % 8 != 0 || s.f % 8 != 0) return false;  // 16-byte rows
+  const size_t rows = std::max(static_cast<size_t>(s.T) * s.d, static_cast<size_t>(s.T) * s.k * s.f) * 2;
+  if (rows > 192 * 1024) return false;  // the staged rows (x, later h) in shared memory
+  if (static_cast<size_t>(s.T) * s.E * 8 > static_cast<size_t>(s.P) * s.d * s.esize) return false;  // logits scratch
+  DecPlan p;
+  return decode_plan(s, device_sm_count(), &p);
 }
 
 namespace {
@@ -537,17 +636,18 @@ cudaError_t launch_decode(const Shape& s, const void* x, float* resid, double ep
                           const void* const* w_down, void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
                           float* losses, void* ws, const Workspace& L, cudaStream_t st) {
   // the accumulator count follows the batch: fewer live registers for small T
-  // keep more of each warp's row loads in flight
-  static std::atomic<size_t> set_smem[8][kMaxDevices];
-  const bool stack = n > 1;
-  void (*kern)(DecArgs) = s.T <= 1 ? (stack ? decode_layer_kernel<1, true> : decode_layer_kernel<1, false>)
-                          : s.T <= 2 ? (stack ? decode_layer_kernel<2, true> : decode_layer_kernel<2, false>)
-                          : s.T <= 4 ? (stack ? decode_layer_kernel<4, true> : decode_layer_kernel<4, false>)
-                                     : (stack ? decode_layer_kernel<8, true> : decode_layer_kernel<8, false>);
-  const int which = (s.T <= 1 ? 0 : s.T <= 2 ? 1 : s.T <= 4 ? 2 : 3) + (stack ? 4 : 0);
-  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(kern), kDecSmem, set_smem[which]);
-  if (e != cudaSuccess) return e;
+  static std::atomic<size_t> set_smem[4][kMaxDevices];
+  void (*kern)(DecArgs) = s.T <= 1   ? decode_layer_kernel<1>
+                          : s.T <= 2 ? decode_layer_kernel<2>
+                          : s.T <= 4 ? decode_layer_kernel<4>
+                                     : decode_layer_kernel<8>;
+  const int which = s.T <= 1 ? 0 : s.T <= 2 ? 1 : s.T <= 4 ? 2 : 3;
   if (n < 1 || n > kDecMaxLayers) return cudaErrorInvalidValue;
+  const int G = device_sm_count();
+  DecPlan plan;
+  if (!decode_plan(s, G, &plan)) return cudaErrorInvalidValue;
+  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(kern), kDecSmemCap, set_smem[which]);
+  if (e != cudaSuccess) return e;
   DecArgs a{};
   a.T = static_cast<int>(s.T);
   a.d = s.d;
@@ -567,6 +667,7 @@ cudaError_t launch_decode(const Shape& s, const void* x, float* resid, double ep
   a.resid = resid;
   a.y = static_cast<__nv_bfloat16*>(y);
   a.h = at<__nv_bfloat16>(ws, L.h);
+  a.logits = at<double>(ws, L.x_perm);
   a.idx_out = topk_idx;
   a.w_out = topk_w;
   a.counts = counts;
@@ -574,10 +675,16 @@ cudaError_t launch_decode(const Shape& s, const void* x, float* resid, double ep
   a.losses_ws = at<float>(ws, L.losses);
   a.bar = reinterpret_cast<unsigned*>(at<int32_t>(ws, L.ctrl) + 3);
   a.status = at<int32_t>(ws, L.ctrl);
+  a.act_off = plan.act_off;
+  a.ps_off = plan.ps_off;
+  a.buf_off = plan.buf_off;
+  a.job_bytes = plan.job_bytes;
+  a.rows_per_job = plan.rows_per_job;
+  a.n_stream = plan.n_stream;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(device_sm_count()));
+  cfg.gridDim = dim3(static_cast<unsigned>(G));
   cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = kDecSmem;
+  cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;

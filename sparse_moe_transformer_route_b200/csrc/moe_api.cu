@@ -599,7 +599,7 @@ moe_status moe_get_device_status(void* ws, int32_t* code, cudaStream_t stream) {
   MOE_TRY(cudaStreamSynchronize(stream));
   // the status word and, with it, the completion counters: a launch that gave
   // up part-way may have left a counter behind
-  MOE_TRY(cudaMemsetAsync(ws, 0, 4 * sizeof(int32_t), stream));
+  MOE_TRY(cudaMemsetAsync(ws, 0, 8 * sizeof(int32_t), stream));
   *code = v;
   return v == 0 ? MOE_OK : MOE_ERR_DEVICE_CHECK;
 }

@@ -34,7 +34,7 @@ struct Shape {
 // Byte offsets of every region inside the caller's workspace.
 struct Workspace {
   // control words: [0] status, [1] router ticket, [2] dispatch ticket,
-  // [3] grid-barrier arrivals, [4] grid-barrier generation
+  // [3] grid-barrier arrivals, [4] CTAs past their last grid barrier
   size_t ctrl;
   size_t counts_part, psum_part, zsum_part;  // router per-CTA partials
   size_t counts, losses;                     // router totals
@@ -104,11 +104,11 @@ cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t*
 // is RMSNorm(resid) (unit weight, eps) and the output is added to resid;
 // otherwise x -> y. Forward only (nothing is kept for the backward).
 bool decode_supported(const Shape& s);
-// Batches the layer forward routes to the one-kernel form by itself: up to 6
-// tokens (measured on B200, L2 flushed before each call: T=1 45 against 93 us
-// layered, T=4 97 against 157, T=6 155 against 159; at T=8 they tie, and in
-// CUDA-graph replays the layered path is ahead there, 166 against 176 us).
-constexpr int64_t kDecodeAutoTokens = 6;
+// Batches the layer forward routes to the one-kernel form by itself: up to 4
+// tokens (measured on B200 in CUDA-graph replays, L2 flushed before each: T=1
+// 45 us, T=4 113 us; at T=6 and T=8 the layered tensor-core path is ahead,
+// about 155 against 217 and 307 us).
+constexpr int64_t kDecodeAutoTokens = 4;
 cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, double eps, const void* w_router,
                                 const float* bias, const void* w_gate_up, const void* w_down, void* y,
                                 int32_t* topk_idx, float* topk_w, int32_t* counts, float* losses, void* ws,

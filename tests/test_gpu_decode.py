@@ -72,9 +72,9 @@ def test_olmoe_shapes(olmoe_layer, T):
     _check(sh, x, *olmoe_layer, out)
 
 
-@pytest.mark.parametrize("T", [1, 6, 8])
+@pytest.mark.parametrize("T", [1, 4, 6, 8])
 def test_fused_and_layered_paths_agree(olmoe_layer, T):
-    """moe_forward without save_for_backward runs the one-kernel layer up to 6
+    """moe_forward without save_for_backward runs the one-kernel layer up to 4
     tokens (bit-identical to moe_forward_decode there); with save_for_backward
     it runs the layered kernels. Both choose the same experts; weights and
     outputs agree."""
@@ -83,7 +83,7 @@ def test_fused_and_layered_paths_agree(olmoe_layer, T):
     fused = _decode(sh, x, *olmoe_layer, explicit=True)
     auto = _decode(sh, x, *olmoe_layer, explicit=False)
     assert np.array_equal(auto["idx"], fused["idx"])
-    if T <= 6:
+    if T <= 4:
         assert torch.equal(auto["y"], fused["y"])
     cfg = M.config(T, sh.d_model, sh.n_experts, sh.top_k, sh.d_ff)
     ws = M.workspace(cfg, True)
@@ -112,7 +112,7 @@ def test_shapes_and_options(T, d, E, k, f, bias, renorm):
     inp = S.layer_inputs(sh, seed=T * 31 + E)
     b = S.zipf_router_offset(E) if bias else None
     cfg = M.config(T, d, E, k, f, renorm=renorm)
-    fits = T * d * 2 <= 160 * 1024 and T * k * f * 2 <= 160 * 1024
+    fits = f <= 2 * d and max(T * d, T * k * f) * 2 + 8 * d <= 192 * 1024
     if not fits:  # beyond the kernel's staging: moe_forward_decode refuses, moe_forward runs the layered path
         with pytest.raises(M.MoeError) as e:
             _decode(sh, inp.x, inp.w_router, inp.w_gate_up, inp.w_down, b, renorm)
@@ -165,7 +165,7 @@ def olmoe_stack_weights():
     return layers
 
 
-@pytest.mark.parametrize("T", [1, 6])
+@pytest.mark.parametrize("T", [1, 4])
 def test_sixteen_layer_decode_stack_in_one_launch(olmoe_stack_weights, T):
     """The whole 16-layer stack of decode blocks as one persistent launch: every
     layer on the oracle's residual at its depth, and the one-launch stack equal
