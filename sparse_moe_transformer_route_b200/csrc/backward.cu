@@ -31,7 +31,7 @@ __device__ __forceinline__ void load8(const T_* p, float (&v)[8]) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      const float2 f = bf16x2_to_float2(w[j]);
       v[2 * j] = f.x;
       v[2 * j + 1] = f.y;
     }
@@ -163,8 +163,8 @@ __device__ __forceinline__ void load4(const T_* p, float (&v)[4]) {
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
   } else {
     const uint2 q = *reinterpret_cast<const uint2*>(p);
-    const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
-    const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+    const float2 f0 = bf16x2_to_float2(q.x);
+    const float2 f1 = bf16x2_to_float2(q.y);
     v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
   }
 }

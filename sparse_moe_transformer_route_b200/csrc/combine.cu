@@ -31,7 +31,7 @@ struct Vec8 {
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+        const float2 f = bf16x2_to_float2(w[j]);
         v[2 * j] = f.x;
         v[2 * j + 1] = f.y;
       }
@@ -68,7 +68,7 @@ struct Raw8 {
       const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+        const float2 f = bf16x2_to_float2(w[j]);
         v[2 * j] = f.x;
         v[2 * j + 1] = f.y;
       }

@@ -149,16 +149,15 @@ __device__ bool grid_barrier(DecSmem& m, const DecArgs& a) {
   return m.ok != 0;
 }
 
-// Eight bf16 values to fp32. A bf16 is the top half of the fp32 with the same
-// value, so the widening is a shift or a mask: integer ALU work at full rate
-// (the conversion instructions run on the quarter-rate pipe that also serves
-// the special functions, and bound this kernel's inner loops).
+// Eight bf16 values to fp32 (integer widening: the conversion instructions'
+// pipe bounded this kernel's inner loops).
 __device__ __forceinline__ void bf16x8(const uint4& q, float (&v)[8]) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    v[2 * j] = __uint_as_float(w[j] << 16);
-    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    const float2 f = bf16x2_to_float2(w[j]);
+    v[2 * j] = f.x;
+    v[2 * j + 1] = f.y;
   }
 }
 

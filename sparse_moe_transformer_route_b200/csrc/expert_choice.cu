@@ -118,8 +118,8 @@ __device__ __forceinline__ double exact_logit(const EcArgs& a, int64_t t, int ee
         const uint32_t xa[4] = {xq[j].x, xq[j].y, xq[j].z, xq[j].w}, wa[4] = {wq[j].x, wq[j].y, wq[j].z, wq[j].w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xa[c]));
-          const float2 wf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[c]));
+          const float2 xf = bf16x2_to_float2(xa[c]);
+          const float2 wf = bf16x2_to_float2(wa[c]);
           acc += static_cast<double>(xf.x * wf.x);  // exact products
           acc += static_cast<double>(xf.y * wf.y);
         }

@@ -238,8 +238,7 @@ __device__ __forceinline__ void load16(const T* src, float (&v)[16]) {
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
-        const float2 f = __bfloat1622float2(b);
+        const float2 f = bf16x2_to_float2(w[j]);
         v[8 * i + 2 * j] = f.x;
         v[8 * i + 2 * j + 1] = f.y;
       }

@@ -52,6 +52,12 @@ constexpr int kStageMax = kAload + kMaxE * 128;          // 12 KB
 // ring bytes for S stages, plus the over-read of the last stage's A
 constexpr int ring_bytes(int S) { return S * kStageMax + 16 * 1024; }
 constexpr int kLogitStride = kMaxE + 1;
+// Independent accumulators the K steps are dealt to (K step kb accumulates into
+// chain kb % kChains; the epilogue adds the chains in order). One chain of
+// M=128 x N=E x K=16 UMMAs is a dependent sequence whose latency, not the
+// tensor pipe, bounds it; four chains let the UMMAs overlap.
+constexpr int kChains = 4;
+__host__ __device__ constexpr uint32_t tmem_cols(int NP) { return NP <= 32 ? 32u * kChains : 64u * kChains; }
 constexpr size_t kMiscBytes = 4096;
 constexpr size_t smem_bytes(int S) { return 1024 + static_cast<size_t>(ring_bytes(S)) + kMiscBytes; }
 static_assert(kTile == 32, "one mask word per expert");
@@ -166,8 +172,8 @@ __device__ __forceinline__ double exact_logit_warp(const __nv_bfloat16* xr, cons
         const uint32_t xa[4] = {xv[b].x, xv[b].y, xv[b].z, xv[b].w}, wa[4] = {wv[b].x, wv[b].y, wv[b].z, wv[b].w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xa[c]));
-          const float2 wf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[c]));
+          const float2 xf = bf16x2_to_float2(xa[c]);
+          const float2 wf = bf16x2_to_float2(wa[c]);
           acc = fma(static_cast<double>(xf.x), static_cast<double>(wf.x), acc);
           acc = fma(static_cast<double>(xf.y), static_cast<double>(wf.y), acc);
         }
@@ -226,33 +232,64 @@ __device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& s
   }
   if (a.probs_only) return;  // uniform over the CTA
 
-  // ---- ranks among the fp32 logits and the nearest other logit
-  int rank[4] = {0, 0, 0, 0};
-  float gap[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
-  for (int e2 = 0; e2 < E; ++e2) {
-    const float v = S[r * kLogitStride + e2];
+  // ---- ranks: a bitonic sort of the token's 64 logits by (logit descending,
+  //      expert ascending) across the half-warp, as 64-bit keys (the logit's
+  //      bits made order-preserving, then the complemented expert index);
+  //      thread `sub` holds sorted positions 4 sub .. 4 sub + 3 at the end
+  unsigned long long key[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = sub + 16 * i;
-      if (e2 != e) {
-        rank[i] += (v > h[i] || (v == h[i] && e2 < e)) ? 1 : 0;
-        gap[i] = fminf(gap[i], fabsf(v - h[i]));
+  for (int j = 0; j < 4; ++j) {
+    const int e = 4 * sub + j;
+    uint32_t b = __float_as_uint(e < E ? S[r * kLogitStride + e] : -INFINITY);
+    if (b == 0x80000000u) b = 0u;  // -0 equals +0: the expert index decides
+    const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    key[j] = (static_cast<unsigned long long>(o) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - e);
+  }
+#pragma unroll
+  for (int size = 2; size <= kMaxE; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      unsigned long long other[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        other[j] = stride >= 4 ? __shfl_xor_sync(hm, key[j], stride / 4) : key[j ^ stride];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = 4 * sub + j;
+        const bool lower = (i & stride) == 0, desc = (i & size) == 0;
+        const unsigned long long hi = key[j] > other[j] ? key[j] : other[j];
+        const unsigned long long lo = key[j] > other[j] ? other[j] : key[j];
+        key[j] = (lower == desc) ? hi : lo;
       }
     }
   }
+  float sval[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t o = static_cast<uint32_t>(key[j] >> 32);
+    sval[j] = __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+  }
+  // the sorted neighbours across thread boundaries
+  const float prev_last = __shfl_up_sync(hm, sval[3], 1);
+  const float next_first = __shfl_down_sync(hm, sval[0], 1);
   bool nearv = false;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int e = sub + 16 * i;
+  for (int j = 0; j < 4; ++j) {
+    const int pos = 4 * sub + j;
+    const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key[j]));
     if (e < E) {
-      rk[r * kMaxE + e] = static_cast<uint8_t>(rank[i]);
-      if (rank[i] <= k && gap[i] < near_gap(h[i])) nearv = true;
-      if (rank[i] < kWin) {  // the sorted window of the first k+4 ranks
-        sv[r * kWin + rank[i]] = h[i];
-        se[r * kWin + rank[i]] = e;
+      rk[r * kMaxE + e] = static_cast<uint8_t>(pos);
+      if (pos < kWin) {  // the sorted window of the first k+4 ranks
+        sv[r * kWin + pos] = sval[j];
+        se[r * kWin + pos] = e;
       }
+      const float up = j > 0 ? sval[j - 1] : (sub > 0 ? prev_last : INFINITY);
+      const float dn = j < 3 ? sval[j + 1] : (sub < 15 ? next_first : -INFINITY);
+      const float gap = fminf(up - sval[j], sval[j] - dn);
+      if (pos <= k && gap < near_gap(sval[j])) nearv = true;
     }
   }
+  int rank[4];
   const bool near = valid && __any_sync(hm, nearv);
   if (tid == 0) *sm.qn = 0;
   epi_sync();
@@ -569,7 +606,7 @@ __global__ void __launch_bounds__(kFusedThreads, MINB)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, a.NP <= 32 ? 32u : 64u);
+    tmem_alloc(tmem_holder, tmem_cols(a.NP));
     tmem_relinquish();
   }
   tc_fence_before();
@@ -619,10 +656,11 @@ __global__ void __launch_bounds__(kFusedThreads, MINB)
         tc_fence_after();
         const uint32_t sa = smem_u32(ring + static_cast<size_t>(s) * STAGE);
         const uint32_t sb = sa + kAload;
+        const uint32_t acc = tmem + static_cast<uint32_t>((kb % kChains) * a.NP);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tmem, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024), idesc,
-                    (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16(acc, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024), idesc,
+                    (kb >= kChains || kk > 0) ? 1u : 0u);
         umma_commit(&empty[s]);
       }
       if (ok) umma_commit(acc_full);
@@ -637,15 +675,21 @@ __global__ void __launch_bounds__(kFusedThreads, MINB)
     if (tid == 0) *qn = 0;
     if (!mbar_wait(acc_full, 0)) report(a.status, DEV_WAIT_TIMEOUT_EPILOGUE);
     tc_fence_after();
-    if (warp == 4) {  // TMEM lanes 0..31 hold the 32 tokens' logits
+    if (warp == 4) {  // TMEM lanes 0..31 hold the 32 tokens' logits, one partial per chain
+      const int nch = nk < kChains ? nk : kChains;
       for (int c = 0; c < a.NP; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + c, v);
-        tmem_ld_wait();
+        float hs[16];
+        for (int j = 0; j < nch; ++j) {
+          uint32_t v[16];
+          tmem_ld16(tmem + static_cast<uint32_t>(j * a.NP + c), v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) hs[i] = j == 0 ? __uint_as_float(v[i]) : hs[i] + __uint_as_float(v[i]);
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int e = c + i;
-          float h = __uint_as_float(v[i]);
+          float h = hs[i];
           if (e < E && a.bias != nullptr) h += a.bias[e];
           S[lane * kLogitStride + e] = (e < E) ? h : -INFINITY;
         }
@@ -663,7 +707,7 @@ __global__ void __launch_bounds__(kFusedThreads, MINB)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, a.NP <= 32 ? 32u : 64u);
+    tmem_dealloc(tmem, tmem_cols(a.NP));
   }
 }
 
@@ -710,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, a.NP <= 32 ? 32u : 64u);
+    tmem_alloc(tmem_holder, tmem_cols(a.NP));
     tmem_relinquish();
   }
   tc_fence_before();
@@ -764,10 +808,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t sa = smem_u32(ring + static_cast<size_t>(s) * STAGE);
         const uint32_t sb = sa + kLogitTile * 128;
+        const uint32_t acc = tmem + static_cast<uint32_t>((kb % kChains) * a.NP);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tmem, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024), idesc,
-                    (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16(acc, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024), idesc,
+                    (kb >= kChains || kk > 0) ? 1u : 0u);
         umma_commit(&empty[s]);
         if (++s == kLogitStages) {
           s = 0;
@@ -782,16 +827,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t t = t0 + q * 32 + lane;
     if (!mbar_wait(acc_full, 0)) report(a.status, DEV_WAIT_TIMEOUT_EPILOGUE);
     tc_fence_after();
+    const int nch = nk < kChains ? nk : kChains;
     for (int c = 0; c < a.NP; c += 16) {
-      uint32_t v[16];
-      tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c), v);
-      tmem_ld_wait();
+      float hs[16];
+      for (int j = 0; j < nch; ++j) {
+        uint32_t v[16];
+        tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(j * a.NP + c), v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) hs[i] = j == 0 ? __uint_as_float(v[i]) : hs[i] + __uint_as_float(v[i]);
+      }
       if (t < a.T) {
         float* dst = a.logit_part + (static_cast<int64_t>(ks) * a.T + t) * a.E;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int e = c + i;
-          if (e < a.E) dst[e] = __uint_as_float(v[i]);
+          if (e < a.E) dst[e] = hs[i];
         }
       }
     }
@@ -801,7 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, a.NP <= 32 ? 32u : 64u);
+    tmem_dealloc(tmem, tmem_cols(a.NP));
   }
 }
 

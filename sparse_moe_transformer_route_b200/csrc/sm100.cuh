@@ -311,6 +311,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Two bf16 values (the low half first) widened to fp32. A bf16 is the top
+// half of the fp32 with the same value, so a shift and a mask are exact: plain
+// integer work at full rate, where the conversion instructions run on the
+// quarter-rate pipe that also serves the special functions.
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
 template <typename T>
 __device__ __forceinline__ float to_f32(T v);
 template <>
@@ -319,7 +327,7 @@ __device__ __forceinline__ float to_f32<float>(float v) {
 }
 template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
-  return __bfloat162float(v);
+  return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&v)) << 16);
 }
 
 template <typename T>
