@@ -232,62 +232,57 @@ __device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& s
   }
   if (a.probs_only) return;  // uniform over the CTA
 
-  // ---- ranks: a bitonic sort of the token's 64 logits by (logit descending,
-  //      expert ascending) across the half-warp, as 64-bit keys (the logit's
-  //      bits made order-preserving, then the complemented expert index);
-  //      thread `sub` holds sorted positions 4 sub .. 4 sub + 3 at the end
-  unsigned long long key[4];
+  // ---- the sorted window: the first min(k + 4, E) ranks by (logit
+  //      descending, expert ascending), picked one per round by an arg-max
+  //      over the half-warp; every other expert gets rank 255 (not chosen).
+  //      A NaN logit counts as -inf here.
+  const int win = min(k + 4, E);
+  float cv[4];
+  bool live[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int e = 4 * sub + j;
-    uint32_t b = __float_as_uint(e < E ? S[r * kLogitStride + e] : -INFINITY);
-    if (b == 0x80000000u) b = 0u;  // -0 equals +0: the expert index decides
-    const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    key[j] = (static_cast<unsigned long long>(o) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - e);
+  for (int i = 0; i < 4; ++i) {
+    const int e = sub + 16 * i;
+    cv[i] = (e < E && !isnan(h[i])) ? h[i] : -INFINITY;
+    live[i] = true;
+    if (e < E) rk[r * kMaxE + e] = 255;
   }
+  for (int p = 0; p < win; ++p) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
 #pragma unroll
-  for (int size = 2; size <= kMaxE; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      unsigned long long other[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        other[j] = stride >= 4 ? __shfl_xor_sync(hm, key[j], stride / 4) : key[j ^ stride];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = 4 * sub + j;
-        const bool lower = (i & stride) == 0, desc = (i & size) == 0;
-        const unsigned long long hi = key[j] > other[j] ? key[j] : other[j];
-        const unsigned long long lo = key[j] > other[j] ? other[j] : key[j];
-        key[j] = (lower == desc) ? hi : lo;
+    for (int i = 0; i < 4; ++i) {
+      const int e = sub + 16 * i;
+      if (live[i] && (cv[i] > bv || (cv[i] == bv && e < be))) {
+        bv = cv[i];
+        be = e;
       }
     }
-  }
-  float sval[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t o = static_cast<uint32_t>(key[j] >> 32);
-    sval[j] = __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+    for (int o = 8; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(hm, bv, o);
+      const int oe = __shfl_xor_sync(hm, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 15) == sub) {  // the owner of the picked expert (be < E: win <= E live experts remain)
+      live[be >> 4] = false;
+      rk[r * kMaxE + be] = static_cast<uint8_t>(p);
+    }
+    if (sub == 0) {
+      sv[r * kWin + p] = bv;
+      se[r * kWin + p] = be;
+    }
   }
-  // the sorted neighbours across thread boundaries
-  const float prev_last = __shfl_up_sync(hm, sval[3], 1);
-  const float next_first = __shfl_down_sync(hm, sval[0], 1);
+  __syncwarp(hm);
+  // near neighbours among the first k + 1 ranks (both sides lie in the window)
   bool nearv = false;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int pos = 4 * sub + j;
-    const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key[j]));
-    if (e < E) {
-      rk[r * kMaxE + e] = static_cast<uint8_t>(pos);
-      if (pos < kWin) {  // the sorted window of the first k+4 ranks
-        sv[r * kWin + pos] = sval[j];
-        se[r * kWin + pos] = e;
-      }
-      const float up = j > 0 ? sval[j - 1] : (sub > 0 ? prev_last : INFINITY);
-      const float dn = j < 3 ? sval[j + 1] : (sub < 15 ? next_first : -INFINITY);
-      const float gap = fminf(up - sval[j], sval[j] - dn);
-      if (pos <= k && gap < near_gap(sval[j])) nearv = true;
-    }
+  for (int p = sub; p <= k && p < win; p += 16) {
+    const float v = sv[r * kWin + p];
+    const float up = p > 0 ? sv[r * kWin + p - 1] : INFINITY;
+    const float dn = p + 1 < win ? sv[r * kWin + p + 1] : -INFINITY;
+    if (fminf(up - v, v - dn) < near_gap(v)) nearv = true;
   }
   int rank[4];
   const bool near = valid && __any_sync(hm, nearv);
