@@ -112,31 +112,10 @@ struct DecSmem {
   DecLayer layers[kDecMaxLayers];  // the launch's layer table
 };
 
-// One thread per CTA: arrive at grid barrier number `m.bars + 1` and wait for
-// every CTA (all co-resident: cooperative launch). The arrival is a gpu-scope
-// release, so this CTA's earlier writes (ordered before this thread by the
-// block barrier that precedes the call) are visible to every CTA that passes;
-// the wait polls with relaxed loads and ends with an acquire fence. The count
-// is compared as a wrap-around difference. False when the wait gave up
-// (recorded in the status word).
+// One thread per CTA: grid barrier number `m.bars + 1` (sm100.cuh).
 __device__ bool grid_sync_thread(DecSmem& m, unsigned* count, int32_t* status) {
   m.bars += 1;
-  const unsigned target = m.bars * gridDim.x;  // at most 48 barriers of <= 1024 CTAs per launch
-  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
-  uint64_t t0 = 0;
-  uint32_t spins = 0;
-  while (true) {
-    unsigned v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
-    if (static_cast<int>(v - target) >= 0) break;
-    if (++spins == 64u) t0 = global_timer_ns();
-    if (spins > 64u && (spins & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
-      report(status, DEV_WAIT_TIMEOUT_GRID);
-      return false;
-    }
-  }
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-  return true;
+  return grid_arrive_wait(count, m.bars * gridDim.x, status);  // at most 48 barriers of <= 1024 CTAs
 }
 
 // Grid barrier with every thread of the CTA taking part; the result is the
@@ -579,13 +558,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
   }  // layers
 
   // every CTA has passed its last grid barrier: the last one out puts the counters back to zero
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(a.bar + 1, 1u) == static_cast<unsigned>(G) - 1u) {
-      a.bar[0] = 0u;
-      a.bar[1] = 0u;
-    }
-  }
+  if (tid == 0) grid_exit(a.bar);
 }
 
 // Shared-memory plan for T tokens on a grid of G CTAs: bookkeeping, the

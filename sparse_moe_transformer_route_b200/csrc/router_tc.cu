@@ -185,7 +185,165 @@ __device__ __forceinline__ double exact_logit_warp(const __nv_bfloat16* xr, cons
   return acc;
 }
 
-__device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& sm, int64_t t0, int tid, int lane) {
+// Tile `cta` (tokens cta * 32 ...) of `ntiles`; the last tile to finish scans.
+// A tile's per-chunk partials (counts from the chosen-token masks, the
+// probability sums from P [kTile][kMaxE], the sum of lse^2), then the ticket:
+// the last tile to finish scans the per-chunk counts into chunk bases,
+// offsets and group starts and reduces both losses, in a fixed order.
+__device__ __forceinline__ void router_finish(const RArgs& a, const EpiSmem& sm, const float* P, int cta, int ntiles,
+                                              int tid, int lane) {
+  unsigned char* R = sm.ring;
+  const int E = a.E, k = a.k;
+  if (tid < E) {
+    a.chunk_count[static_cast<size_t>(cta) * E + tid] = __popc(sm.mask[tid]);
+    float ps = 0.f;
+    for (int rr = 0; rr < kTile; ++rr) ps += P[rr * kMaxE + tid];
+    a.psum_part[static_cast<size_t>(cta) * E + tid] = ps;
+  }
+  if (tid == kMaxE) {
+    double z = 0.0;
+    for (int rr = 0; rr < kTile; ++rr) z += static_cast<double>(sm.lse_s[rr]) * sm.lse_s[rr];
+    a.zsum_part[cta] = z;
+  }
+  __threadfence();
+  epi_sync();
+  if (tid == 0) *sm.s_last = (atomicAdd(a.ticket, 1) == ntiles - 1);
+  epi_sync();
+  if (!*sm.s_last) return;
+
+  // ---- the last CTA: scan of the per-chunk counts, losses
+  __threadfence();
+  const int nb = ntiles;
+  int32_t* seg_i = reinterpret_cast<int32_t*>(R + kOffSegI);
+  double* seg_d = reinterpret_cast<double*>(R + kOffSegD);
+  double* zred = reinterpret_cast<double*>(R + kOffZ);
+  int32_t* cnt_s = reinterpret_cast<int32_t*>(R + kOffScan);               // [kScanBlock][E]
+  float* ps_s = reinterpret_cast<float*>(R + kOffScan + kScanBlock * kMaxE * 4);  // [kScanBlock][E]
+  const int e = tid & (kMaxE - 1), g = tid / kMaxE;  // expert, segment
+  constexpr int kSegLen = kScanBlock / kScanSeg;
+  int run = 0;
+  double pe = 0.0;
+  for (int c0 = 0; c0 < nb; c0 += kScanBlock) {
+    const int nc = min(kScanBlock, nb - c0);
+    {  // the block's counts and probability sums, 16-byte loads (c0 * E is a multiple of 4)
+      const int n = nc * E;
+      const int32_t* gc = a.chunk_count + static_cast<size_t>(c0) * E;
+      const float* gp = a.psum_part + static_cast<size_t>(c0) * E;
+      for (int i = tid * 4; i < (n & ~3); i += kEpiThreads * 4) {
+        *reinterpret_cast<int4*>(cnt_s + i) = __ldcg(reinterpret_cast<const int4*>(gc + i));
+        *reinterpret_cast<float4*>(ps_s + i) = __ldcg(reinterpret_cast<const float4*>(gp + i));
+      }
+      for (int i = (n & ~3) + tid; i < n; i += kEpiThreads) {
+        cnt_s[i] = __ldcg(gc + i);
+        ps_s[i] = __ldcg(gp + i);
+      }
+    }
+    epi_sync();
+    int sc = 0;
+    double sp = 0.0;
+    if (e < E) {
+      for (int j = 0; j < kSegLen; ++j) {
+        const int c = g * kSegLen + j;
+        if (c < nc) {
+          sc += cnt_s[c * E + e];
+          sp += static_cast<double>(ps_s[c * E + e]);
+        }
+      }
+    }
+    seg_i[g * kMaxE + e] = sc;
+    seg_d[g * kMaxE + e] = sp;
+    epi_sync();
+    if (e < E) {
+      int base = run;
+      for (int g2 = 0; g2 < g; ++g2) base += seg_i[g2 * kMaxE + e];
+      for (int j = 0; j < kSegLen; ++j) {
+        const int c = g * kSegLen + j;
+        if (c < nc) {
+          a.chunk_base[static_cast<size_t>(c0 + c) * E + e] = base;
+          base += cnt_s[c * E + e];
+        }
+      }
+      for (int g2 = 0; g2 < kScanSeg; ++g2) {
+        run += seg_i[g2 * kMaxE + e];
+        pe += seg_d[g2 * kMaxE + e];
+      }
+    }
+    epi_sync();  // the block's scratch is reused by the next pass
+  }
+  if (g == 0 && e < E) {
+    sm.tot[e] = run;
+    sm.tot_p[e] = pe;
+    a.counts_ws[e] = run;
+    if (a.counts_user != nullptr) a.counts_user[e] = run;
+  }
+  {  // sum of lse^2 partials: contiguous slices in order, then the slices in order
+    const int per = (nb + kEpiThreads - 1) / kEpiThreads;
+    double z = 0.0;
+    for (int c = tid * per; c < min(nb, (tid + 1) * per); ++c) z += __ldcg(&a.zsum_part[c]);
+    zred[tid] = z;
+  }
+  epi_sync();
+  if (tid < 32) {
+    // warp-wide finalisation (E <= 64): lane holds experts lane and lane + 32.
+    // Group starts and offsets are exclusive prefix sums; the two loss sums use a
+    // fixed butterfly order, so every lane ends with the same bits on every run.
+    const int e0 = lane, e1 = lane + 32;
+    const int c0v = e0 < E ? sm.tot[e0] : 0, c1v = e1 < E ? sm.tot[e1] : 0;
+    const int g0v = (c0v + kRowAlign - 1) / kRowAlign * kRowAlign;
+    const int g1v = (c1v + kRowAlign - 1) / kRowAlign * kRowAlign;
+    int ic0 = c0v, ig0 = g0v, ic1 = c1v, ig1 = g1v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u0 = __shfl_up_sync(0xffffffffu, ic0, o), w0 = __shfl_up_sync(0xffffffffu, ig0, o);
+      const int u1 = __shfl_up_sync(0xffffffffu, ic1, o), w1 = __shfl_up_sync(0xffffffffu, ig1, o);
+      if (lane >= o) {
+        ic0 += u0;
+        ig0 += w0;
+        ic1 += u1;
+        ig1 += w1;
+      }
+    }
+    const int tc0 = __shfl_sync(0xffffffffu, ic0, 31), tg0 = __shfl_sync(0xffffffffu, ig0, 31);
+    const int tc1 = __shfl_sync(0xffffffffu, ic1, 31), tg1 = __shfl_sync(0xffffffffu, ig1, 31);
+    if (e0 < E) {
+      a.offsets_ws[e0] = ic0 - c0v;
+      a.gs_ws[e0] = ig0 - g0v;
+    }
+    if (e1 < E) {
+      a.offsets_ws[e1] = tc0 + ic1 - c1v;
+      a.gs_ws[e1] = tg0 + ig1 - g1v;
+    }
+    // load balance: E * sum_e (c_e / (T k)) (P_e / T) = E * sum_e c_e P_e / (T^2 k)
+    double lb = (e0 < E ? static_cast<double>(c0v) * sm.tot_p[e0] : 0.0) +
+                (e1 < E ? static_cast<double>(c1v) * sm.tot_p[e1] : 0.0);
+    double zt = 0.0;
+    for (int j = 0; j < kEpiThreads / 32; ++j) zt += zred[lane * (kEpiThreads / 32) + j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lb += __shfl_xor_sync(0xffffffffu, lb, o);
+      zt += __shfl_xor_sync(0xffffffffu, zt, o);
+    }
+    if (lane == 0) {
+      const int off = tc0 + tc1;
+      a.offsets_ws[E] = off;
+      a.gs_ws[E] = tg0 + tg1;
+      const double Td = static_cast<double>(a.T);
+      const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(zt / Td);
+      a.losses_ws[0] = l0;
+      a.losses_ws[1] = l1;
+      if (a.losses_user != nullptr) {
+        a.losses_user[0] = l0;
+        a.losses_user[1] = l1;
+      }
+      if (static_cast<int64_t>(off) != a.T * k) report(a.status, DEV_COUNT_MISMATCH);
+      *a.ticket = 0;
+    }
+  }
+}
+
+__device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& sm, int cta, int ntiles, int tid,
+                                                int lane) {
+  const int64_t t0 = static_cast<int64_t>(cta) * kTile;
   unsigned char* R = sm.ring;
   float* S = reinterpret_cast<float*>(R + kOffS);
   float* P = reinterpret_cast<float*>(R + kOffP);
@@ -413,152 +571,7 @@ __device__ __forceinline__ void router_epilogue(const RArgs& a, const EpiSmem& s
       if (rank[i] < k) a.local_rank[t * k + rank[i]] = __popc(sm.mask[e] & ((1u << r) - 1u));
     }
   }
-  const int cta = blockIdx.x;
-  if (tid < E) {
-    a.chunk_count[static_cast<size_t>(cta) * E + tid] = __popc(sm.mask[tid]);
-    float ps = 0.f;
-    for (int rr = 0; rr < kTile; ++rr) ps += P[rr * kMaxE + tid];
-    a.psum_part[static_cast<size_t>(cta) * E + tid] = ps;
-  }
-  if (tid == kMaxE) {
-    double z = 0.0;
-    for (int rr = 0; rr < kTile; ++rr) z += static_cast<double>(sm.lse_s[rr]) * sm.lse_s[rr];
-    a.zsum_part[cta] = z;
-  }
-  __threadfence();
-  epi_sync();
-  if (tid == 0) *sm.s_last = (atomicAdd(a.ticket, 1) == static_cast<int>(gridDim.x) - 1);
-  epi_sync();
-  if (!*sm.s_last) return;
-
-  // ---- the last CTA: scan of the per-chunk counts, losses
-  __threadfence();
-  const int nb = gridDim.x;
-  int32_t* seg_i = reinterpret_cast<int32_t*>(R + kOffSegI);
-  double* seg_d = reinterpret_cast<double*>(R + kOffSegD);
-  double* zred = reinterpret_cast<double*>(R + kOffZ);
-  int32_t* cnt_s = reinterpret_cast<int32_t*>(R + kOffScan);               // [kScanBlock][E]
-  float* ps_s = reinterpret_cast<float*>(R + kOffScan + kScanBlock * kMaxE * 4);  // [kScanBlock][E]
-  const int e = tid & (kMaxE - 1), g = tid / kMaxE;  // expert, segment
-  constexpr int kSegLen = kScanBlock / kScanSeg;
-  int run = 0;
-  double pe = 0.0;
-  for (int c0 = 0; c0 < nb; c0 += kScanBlock) {
-    const int nc = min(kScanBlock, nb - c0);
-    {  // the block's counts and probability sums, 16-byte loads (c0 * E is a multiple of 4)
-      const int n = nc * E;
-      const int32_t* gc = a.chunk_count + static_cast<size_t>(c0) * E;
-      const float* gp = a.psum_part + static_cast<size_t>(c0) * E;
-      for (int i = tid * 4; i < (n & ~3); i += kEpiThreads * 4) {
-        *reinterpret_cast<int4*>(cnt_s + i) = __ldcg(reinterpret_cast<const int4*>(gc + i));
-        *reinterpret_cast<float4*>(ps_s + i) = __ldcg(reinterpret_cast<const float4*>(gp + i));
-      }
-      for (int i = (n & ~3) + tid; i < n; i += kEpiThreads) {
-        cnt_s[i] = __ldcg(gc + i);
-        ps_s[i] = __ldcg(gp + i);
-      }
-    }
-    epi_sync();
-    int sc = 0;
-    double sp = 0.0;
-    if (e < E) {
-      for (int j = 0; j < kSegLen; ++j) {
-        const int c = g * kSegLen + j;
-        if (c < nc) {
-          sc += cnt_s[c * E + e];
-          sp += static_cast<double>(ps_s[c * E + e]);
-        }
-      }
-    }
-    seg_i[g * kMaxE + e] = sc;
-    seg_d[g * kMaxE + e] = sp;
-    epi_sync();
-    if (e < E) {
-      int base = run;
-      for (int g2 = 0; g2 < g; ++g2) base += seg_i[g2 * kMaxE + e];
-      for (int j = 0; j < kSegLen; ++j) {
-        const int c = g * kSegLen + j;
-        if (c < nc) {
-          a.chunk_base[static_cast<size_t>(c0 + c) * E + e] = base;
-          base += cnt_s[c * E + e];
-        }
-      }
-      for (int g2 = 0; g2 < kScanSeg; ++g2) {
-        run += seg_i[g2 * kMaxE + e];
-        pe += seg_d[g2 * kMaxE + e];
-      }
-    }
-    epi_sync();  // the block's scratch is reused by the next pass
-  }
-  if (g == 0 && e < E) {
-    sm.tot[e] = run;
-    sm.tot_p[e] = pe;
-    a.counts_ws[e] = run;
-    if (a.counts_user != nullptr) a.counts_user[e] = run;
-  }
-  {  // sum of lse^2 partials: contiguous slices in order, then the slices in order
-    const int per = (nb + kEpiThreads - 1) / kEpiThreads;
-    double z = 0.0;
-    for (int c = tid * per; c < min(nb, (tid + 1) * per); ++c) z += __ldcg(&a.zsum_part[c]);
-    zred[tid] = z;
-  }
-  epi_sync();
-  if (tid < 32) {
-    // warp-wide finalisation (E <= 64): lane holds experts lane and lane + 32.
-    // Group starts and offsets are exclusive prefix sums; the two loss sums use a
-    // fixed butterfly order, so every lane ends with the same bits on every run.
-    const int e0 = lane, e1 = lane + 32;
-    const int c0v = e0 < E ? sm.tot[e0] : 0, c1v = e1 < E ? sm.tot[e1] : 0;
-    const int g0v = (c0v + kRowAlign - 1) / kRowAlign * kRowAlign;
-    const int g1v = (c1v + kRowAlign - 1) / kRowAlign * kRowAlign;
-    int ic0 = c0v, ig0 = g0v, ic1 = c1v, ig1 = g1v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u0 = __shfl_up_sync(0xffffffffu, ic0, o), w0 = __shfl_up_sync(0xffffffffu, ig0, o);
-      const int u1 = __shfl_up_sync(0xffffffffu, ic1, o), w1 = __shfl_up_sync(0xffffffffu, ig1, o);
-      if (lane >= o) {
-        ic0 += u0;
-        ig0 += w0;
-        ic1 += u1;
-        ig1 += w1;
-      }
-    }
-    const int tc0 = __shfl_sync(0xffffffffu, ic0, 31), tg0 = __shfl_sync(0xffffffffu, ig0, 31);
-    const int tc1 = __shfl_sync(0xffffffffu, ic1, 31), tg1 = __shfl_sync(0xffffffffu, ig1, 31);
-    if (e0 < E) {
-      a.offsets_ws[e0] = ic0 - c0v;
-      a.gs_ws[e0] = ig0 - g0v;
-    }
-    if (e1 < E) {
-      a.offsets_ws[e1] = tc0 + ic1 - c1v;
-      a.gs_ws[e1] = tg0 + ig1 - g1v;
-    }
-    // load balance: E * sum_e (c_e / (T k)) (P_e / T) = E * sum_e c_e P_e / (T^2 k)
-    double lb = (e0 < E ? static_cast<double>(c0v) * sm.tot_p[e0] : 0.0) +
-                (e1 < E ? static_cast<double>(c1v) * sm.tot_p[e1] : 0.0);
-    double zt = 0.0;
-    for (int j = 0; j < kEpiThreads / 32; ++j) zt += zred[lane * (kEpiThreads / 32) + j];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      lb += __shfl_xor_sync(0xffffffffu, lb, o);
-      zt += __shfl_xor_sync(0xffffffffu, zt, o);
-    }
-    if (lane == 0) {
-      const int off = tc0 + tc1;
-      a.offsets_ws[E] = off;
-      a.gs_ws[E] = tg0 + tg1;
-      const double Td = static_cast<double>(a.T);
-      const float l0 = static_cast<float>(lb * E / (Td * Td * k)), l1 = static_cast<float>(zt / Td);
-      a.losses_ws[0] = l0;
-      a.losses_ws[1] = l1;
-      if (a.losses_user != nullptr) {
-        a.losses_user[0] = l0;
-        a.losses_user[1] = l1;
-      }
-      if (static_cast<int64_t>(off) != a.T * k) report(a.status, DEV_COUNT_MISMATCH);
-      *a.ticket = 0;
-    }
-  }
+  router_finish(a, sm, P, cta, ntiles, tid, lane);
 }
 
 // STAGES-deep ring, MINB CTAs per SM: one CTA with a 16-deep ring when the
@@ -695,7 +708,7 @@ __global__ void __launch_bounds__(kFusedThreads, MINB)
     epi_sync();
 
     const EpiSmem sm{ring, mask, lse_s, s_last, qn, tot, tot_p};
-    router_epilogue(a, sm, t0, tid, lane);
+    router_epilogue(a, sm, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), tid, lane);
   }
   __syncwarp();
   tc_fence_before();
@@ -851,10 +864,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-__global__ void __launch_bounds__(kEpiThreads, 2) router_epi_kernel(const RArgs a) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* ring = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+// The epilogue of tile `tile` of `ntiles` from logits in the workspace (the
+// K-range partials, summed in a fixed order, plus the offset). `smem` is
+// 1024-aligned with kEpiSmem bytes.
+__device__ __forceinline__ void epi_tile(const RArgs& a, unsigned char* ring, int tile, int ntiles) {
   unsigned char* misc = ring + kEpiRing;
   uint32_t* mask = reinterpret_cast<uint32_t*>(misc);          // [kMaxE]
   float* lse_s = reinterpret_cast<float*>(mask + kMaxE);      // [kTile]
@@ -864,13 +877,9 @@ __global__ void __launch_bounds__(kEpiThreads, 2) router_epi_kernel(const RArgs 
   double* tot_p = reinterpret_cast<double*>(tot + kMaxE);     // [kMaxE]
   float* S = reinterpret_cast<float*>(ring + kOffS);
   const int tid = threadIdx.x, lane = tid & 31;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
-  pdl_trigger();
+  const int64_t t0 = static_cast<int64_t>(tile) * kTile;
   if (tid < kMaxE) mask[tid] = 0u;
   if (tid == 0) *qn = 0;
-  pdl_wait();
-  // this tile's logits: the K-range partials (all loads in flight, then summed
-  // in a fixed order), plus the offset
   for (int i = tid; i < kTile * kMaxE; i += kEpiThreads) {
     const int r = i / kMaxE, e = i - r * kMaxE;
     float h = -INFINITY;
@@ -890,7 +899,16 @@ __global__ void __launch_bounds__(kEpiThreads, 2) router_epi_kernel(const RArgs 
   }
   epi_sync();
   const EpiSmem sm{ring, mask, lse_s, s_last, qn, tot, tot_p};
-  router_epilogue(a, sm, t0, tid, lane);
+  router_epilogue(a, sm, tile, ntiles, tid, lane);
+}
+
+__global__ void __launch_bounds__(kEpiThreads, 2) router_epi_kernel(const RArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* ring = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  pdl_trigger();
+  pdl_wait();
+  epi_tile(a, ring, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x));
 }
 
 }  // namespace

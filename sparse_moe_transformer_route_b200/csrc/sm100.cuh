@@ -52,6 +52,45 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// ---------------------------------------------------------------- grid barrier
+// For cooperative launches (all CTAs co-resident). bar[0] counts arrivals up
+// through a launch (barrier j opens when it reaches j * grid); bar[1] counts
+// the CTAs that are past their last barrier, and the last of them puts both
+// back to zero, so every launch starts from zero.
+
+// One thread per CTA: arrive (a gpu-scope release: this CTA's earlier writes,
+// ordered before this thread by the block barrier in front of the call, are
+// visible to every CTA that passes) and wait until the count reaches `target`
+// (compared as a wrap-around difference), polling with relaxed loads and
+// ending with an acquire fence. False when the wait gave up after about a
+// second (recorded in the status word).
+__device__ __forceinline__ bool grid_arrive_wait(unsigned* count, unsigned target, int32_t* status) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
+  uint64_t t0 = 0;
+  uint32_t spins = 0;
+  while (true) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
+    if (static_cast<int>(v - target) >= 0) break;
+    if (++spins == 64u) t0 = global_timer_ns();
+    if (spins > 64u && (spins & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+      report(status, DEV_WAIT_TIMEOUT_GRID);
+      return false;
+    }
+  }
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  return true;
+}
+
+// One thread per CTA, after the CTA's last barrier of the launch.
+__device__ __forceinline__ void grid_exit(unsigned* bar) {
+  __threadfence();
+  if (atomicAdd(bar + 1, 1u) == gridDim.x - 1u) {
+    bar[0] = 0u;
+    bar[1] = 0u;
+  }
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
