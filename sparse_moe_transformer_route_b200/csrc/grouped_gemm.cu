@@ -767,7 +767,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
     }
     for (int b = 0; b < P::ACC_BUFS; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 2 * 32 * P::EPI_WARPS);  // both CTAs' epilogue threads (the leader's copy)
+      mbar_init(&acc_empty[b], 2 * P::EPI_WARPS);  // both CTAs' epilogue warps (the leader's copy)
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -910,7 +910,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
     uint32_t acc_phase = 0;
     for (int L = cluster; L < n_tiles; L += n_clusters) {
       const PairTile t = decode_pair_tile<P>(a, gs, off, pts, L, rank);
-      if (!mbar_wait(&acc_full[acc], acc_phase)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase))) {  // warp-uniform
         report(a.status, DEV_WAIT_TIMEOUT_EPILOGUE);
         break;
       }
@@ -976,8 +976,12 @@ __global__ void __launch_bounds__(P::THREADS, 1)
           }
         }
       }
+      // the warp's TMEM reads are complete (wait::ld) and fenced; one arrive per
+      // warp releases the accumulator to the leader's MMA issuer (nothing in
+      // this kernel reads the stored rows, so no global ordering is needed)
       tc_fence_before();
-      mbar_arrive_cluster(acc_empty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
       if (++acc == P::ACC_BUFS) {
         acc = 0;
         acc_phase ^= 1u;
