@@ -34,10 +34,12 @@
 //             products with the h rows of the expert's tokens; then each
 //             token's slot-ordered weighted sum is written once (bf16 y, or
 //             added to the residual, whose columns this CTA owns).
-// The streaming warps each own two job buffers in shared memory and fetch
-// their jobs with 16-byte asynchronous copies, the next job's bytes in flight
-// while the current one is computed; so no register holds data in flight, and
-// the copies of a warp's first phase-2 jobs go out before the grid barrier.
+// The streaming warps each own a few job buffers in shared memory, each with
+// an mbarrier; lane 0 fetches a job as bulk copies of whole weight rows (the
+// copy engine, not the load/store units, moves the bytes), the next jobs'
+// bytes in flight while the current one is computed; so no register holds
+// data in flight, and the copies of a warp's first phase-2 jobs go out before
+// the grid barrier.
 // Shares are dealt round-robin by rows (pairs, columns): every SM streams
 // within one row of the same number of bytes, and at any moment the grid
 // reads one contiguous stretch of each weight matrix (per-CTA contiguous
@@ -61,6 +63,8 @@ constexpr int kDecSlots = kDecMaxT * kMaxTopK;  // (token, slot) pairs
 constexpr int kDecMaxLayers = 16;               // layers of a stack per launch
 constexpr size_t kDecSmemCap = 227 * 1024;      // dynamic shared memory of one CTA
 constexpr int kMaxStreamWarps = kDecWarps;     // warps that fetch and compute jobs
+constexpr int kDecBufsPerWarp = 2;             // job buffers of one streaming warp
+constexpr int kDecJobBufs = kMaxStreamWarps * kDecBufsPerWarp;
 
 // One layer's weights.
 struct DecLayer {
@@ -92,7 +96,7 @@ struct DecArgs {
   uint32_t act_off, ps_off, buf_off;
   uint32_t job_bytes;        // one job buffer: a gate/up row pair, or rows_per_job down rows
   int rows_per_job;
-  int n_stream;              // streaming warps (0 .. n_stream-1), two job buffers each
+  int n_stream;              // streaming warps (0 .. n_stream-1), kDecBufsPerWarp job buffers each
 };
 
 struct DecSmem {
@@ -110,6 +114,7 @@ struct DecSmem {
   float p[kDecMaxT][kDecMaxE];
   float lse[kDecMaxT];
   DecLayer layers[kDecMaxLayers];  // the launch's layer table
+  uint64_t jbar[kDecJobBufs];      // completion of each job buffer (streaming warp w: w * kDecBufsPerWarp ...)
 };
 
 // One thread per CTA: grid barrier number `m.bars + 1` (sm100.cuh).
@@ -138,6 +143,33 @@ __device__ __forceinline__ void bf16x8(const uint4& q, float (&v)[8]) {
     v[2 * j] = f.x;
     v[2 * j + 1] = f.y;
   }
+}
+
+// acc + a.lo * x.lo, then + a.hi * x.hi: two fused multiply-adds of bf16
+// operands into fp32 (each the exact product, one rounding), in element order.
+__device__ __forceinline__ float fma2_bf16(uint32_t a, uint32_t x, float acc) {
+  asm("{\n\t.reg .b16 al, ah, xl, xh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {xl, xh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, xl, %0;\n\t"
+      "fma.rn.f32.bf16 %0, ah, xh, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(a), "r"(x));
+  return acc;
+}
+
+// The same for two rows (gate and up) against one x pair.
+__device__ __forceinline__ void fma2_bf16_pair(uint32_t g, uint32_t u, uint32_t x, float& ag, float& au) {
+  asm("{\n\t.reg .b16 gl, gh, ul, uh, xl, xh;\n\t"
+      "mov.b32 {gl, gh}, %2;\n\t"
+      "mov.b32 {ul, uh}, %3;\n\t"
+      "mov.b32 {xl, xh}, %4;\n\t"
+      "fma.rn.f32.bf16 %0, gl, xl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, ul, xl, %1;\n\t"
+      "fma.rn.f32.bf16 %0, gh, xh, %0;\n\t"
+      "fma.rn.f32.bf16 %1, uh, xh, %1;\n\t}"
+      : "+f"(ag), "+f"(au)
+      : "r"(g), "r"(u), "r"(x));
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -184,45 +216,92 @@ __device__ __forceinline__ int pair_jobs(int SW, int w, int P) {
 // Output column of this CTA's l-th column.
 __device__ __forceinline__ int cta_col(int l) { return static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) * l; }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+// A streaming warp's job buffers: job q goes to buffer q % kDecBufsPerWarp, whose
+// mbarrier completes once per job. `ph` holds the parity each buffer's next
+// wait expects, `pend` the buffers with a copy in flight; both live across
+// layers. `live` turns false when a wait gave up (recorded in the status
+// word): the warp then issues and computes nothing more.
+struct JobPipe {
+  uint64_t* bar;       // [kDecBufsPerWarp]
+  unsigned char* buf;  // kDecBufsPerWarp buffers of job_bytes
+  uint32_t job_bytes;
+  uint32_t ph, pend;
+  bool live;
+  __device__ unsigned char* at(int q) const { return buf + static_cast<size_t>(q % kDecBufsPerWarp) * job_bytes; }
+};
 
-// Warp `w`'s job q (its phase-1 pairs w, w + SW, ... then its phase-2 jobs
-// w, w + SW, ...) into `buf`, as 16-byte asynchronous copies by the 32 lanes,
-// then one commit group (also when q is past the warp's last job).
+// Lane 0: warp w's job q (its phase-1 pairs w, w + SW, ... then its phase-2
+// jobs w, w + SW, ...) into `buf` as bulk copies of whole weight rows,
+// completing on the buffer's mbarrier; nothing when q is past the warp's last
+// job. The caller has made the whole warp's reads of the buffer complete.
 __device__ __forceinline__ void fetch_job(const DecArgs& a, const DecSmem& m, const DecLayer& Ly, const Share& sh,
-                                          int nt, int w, int lane, int c1, int c2, int q, unsigned char* buf) {
+                                          int nt, int w, int c1, int c2, int q, unsigned char* buf, uint64_t* bar) {
   const int SW = a.n_stream;
   if (q < c1) {
     const int p = pair_index(SW, w, q);
     const int u = p / a.f, i = p - u * a.f;
     const __nv_bfloat16* g = Ly.wgu + (static_cast<int64_t>(m.touched[u]) * 2 * a.f + i) * a.d;
-    const __nv_bfloat16* up = g + static_cast<int64_t>(a.f) * a.d;
-    const int nvd = a.d / 8;
-    for (int c = lane; c < 2 * nvd; c += 32)
-      cp_async16(buf + 16 * c, c < nvd ? g + 8 * c : up + 8 * (c - nvd));
+    const uint32_t rb = static_cast<uint32_t>(a.d) * 2;
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, 2 * rb);
+    bulk_load(buf, g, rb, bar);
+    bulk_load(buf + rb, g + static_cast<int64_t>(a.f) * a.d, rb, bar);
   } else if (q < c1 + c2) {
     const int r0 = (w + SW * (q - c1)) * a.rows_per_job;
     const int nr = min(a.rows_per_job, sh.rows2 - r0);
-    const int nvf = a.f / 8;
+    const uint32_t rb = static_cast<uint32_t>(a.f) * 2;
     int cl = r0 / nt, u = r0 - cl * nt;  // the row's column (of this CTA's) and touched-expert index
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nr) * rb);
     for (int rr = 0; rr < nr; ++rr) {
       const __nv_bfloat16* row = Ly.wd + (static_cast<int64_t>(m.touched[u]) * a.d + cta_col(cl)) * a.f;
-      unsigned char* dst = buf + static_cast<size_t>(rr) * nvf * 16;
-      for (int v = lane; v < nvf; v += 32) cp_async16(dst + 16 * v, row + 8 * v);
+      bulk_load(buf + static_cast<size_t>(rr) * rb, row, rb, bar);
       if (++u == nt) {
         u = 0;
         ++cl;
       }
     }
   }
-  cp_async_commit();
+}
+
+// The whole warp: issue job q (if it exists) into buffer q % kDecBufsPerWarp.
+__device__ __forceinline__ void issue_job(const DecArgs& a, const DecSmem& m, const DecLayer& Ly, const Share& sh,
+                                          int nt, int w, int lane, int c1, int c2, int q, JobPipe& jp) {
+  if (!jp.live || q >= c1 + c2) return;
+  const int b = q % kDecBufsPerWarp;
+  __syncwarp();
+  if (lane == 0) fetch_job(a, m, Ly, sh, nt, w, c1, c2, q, jp.at(q), jp.bar + b);
+  jp.pend |= 1u << b;
+}
+
+// The whole warp: wait until buffer b's bytes have landed (every lane
+// observes the completion itself). False when the warp is no longer live.
+__device__ __forceinline__ bool await_buf(JobPipe& jp, int b, int32_t* status) {
+  if (!jp.live) return false;
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(jp.bar + b, (jp.ph >> b) & 1u));
+  jp.ph ^= 1u << b;
+  jp.pend &= ~(1u << b);
+  if (!ok) {
+    report(status, DEV_WAIT_TIMEOUT_PRODUCER);
+    jp.live = false;
+  }
+  return ok;
+}
+
+__device__ __forceinline__ bool await_job(JobPipe& jp, int q, int32_t* status) {
+  return await_buf(jp, q % kDecBufsPerWarp, status);
+}
+
+// The whole warp, before the CTA leaves: no copy in flight into its buffers
+// (each wait bounded).
+__device__ __forceinline__ void drain_jobs(JobPipe& jp) {
+  for (int b = 0; b < kDecBufsPerWarp; ++b)
+    if ((jp.pend >> b) & 1u) {
+      mbar_wait(jp.bar + b, (jp.ph >> b) & 1u);
+      jp.ph ^= 1u << b;
+    }
+  jp.pend = 0;
+  __syncwarp();
 }
 
 // Logit task q: expert q / T, token q % T, as an fp64 sum of the exact
@@ -258,77 +337,134 @@ __device__ __forceinline__ void logit_task(const DecArgs& a, const DecLayer& Ly,
   if (lane == 0) a.logits[t * E + e] = acc + (Ly.bias != nullptr ? static_cast<double>(Ly.bias[e]) : 0.0);
 }
 
-// Phase-1 job: gate/up row pair p (in `buf`) meets every token of the pair's
-// expert; h = SiLU(g) * u in bf16.
+// The tokens of a mask in ascending order: tok[j] is its j-th set bit
+// (statically indexed, so the list stays in registers).
 template <int NT>
-__device__ __forceinline__ void pair_job(const DecArgs& a, const DecSmem& m, const __nv_bfloat16* act,
-                                         const unsigned char* buf, int p, int lane) {
-  const int d = a.d, k = a.k, f = a.f, nvd = d / 8;
-  const int u = p / f, i = p - u * f;
-  const int e = m.touched[u];
-  const unsigned tm = m.tokmask[e];
-  const uint4* g4 = reinterpret_cast<const uint4*>(buf);
-  const uint4* u4 = g4 + nvd;
-  const uint4* x4 = reinterpret_cast<const uint4*>(act);
-  float ag[NT], au[NT];
+__device__ __forceinline__ int mask_tokens(unsigned tm, int (&tok)[NT]) {
+  const int n = __popc(tm);
 #pragma unroll
-  for (int t = 0; t < NT; ++t) ag[t] = au[t] = 0.f;
-  for (int v = lane; v < nvd; v += 32) {
-    float gv[8], uv[8];
-    bf16x8(g4[v], gv);
-    bf16x8(u4[v], uv);
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      if ((tm >> t) & 1u) {
-        float xv[8];
-        bf16x8(x4[t * nvd + v], xv);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          ag[t] = fmaf(gv[c], xv[c], ag[t]);
-          au[t] = fmaf(uv[c], xv[c], au[t]);
-        }
-      }
-    }
+  for (int j = 0; j < NT; ++j) {
+    tok[j] = tm != 0u ? __ffs(tm) - 1 : 0;
+    tm &= tm - 1u;
   }
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    if ((tm >> t) & 1u) {
-      const float g = warp_sum(ag[t]), uu = warp_sum(au[t]);
-      if (lane == 0)
-        a.h[static_cast<int64_t>(t * k + m.slot_of[t][e]) * f + i] = __float2bfloat16_rn(silu_fast(g) * uu);
-    }
+  return n;
+}
+
+// Calls body.template run<n>() for the runtime count n in [1, NT], so the
+// per-token accumulators are sized to the tokens present rather than to NT
+// (predicated-off tokens would still take issue slots).
+template <int N, int NT, class Body>
+__device__ __forceinline__ void with_count(int n, Body& body) {
+  if constexpr (N <= NT) {
+    if (n == N)
+      body.template run<N>();
+    else
+      with_count<N + 1, NT>(n, body);
   }
 }
 
+// Phase-1 job: gate/up row pair p (in `buf`) meets the n tokens of the pair's
+// expert; h = SiLU(g) * u in bf16.
+template <int NT>
+struct PairBody {
+  const DecArgs& a;
+  const DecSmem& m;
+  const uint4* g4;
+  const uint4* x4;
+  const int (&tok)[NT];
+  int e, i, lane;
+  template <int N>
+  __device__ __forceinline__ void run() {
+    const int nvd = a.d / 8;
+    const uint4* u4 = g4 + nvd;
+    float ag[N], au[N];
+#pragma unroll
+    for (int j = 0; j < N; ++j) ag[j] = au[j] = 0.f;
+    for (int v = lane; v < nvd; v += 32) {
+      const uint4 gq = g4[v], uq = u4[v];
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const uint4 xq = x4[tok[j] * nvd + v];
+        fma2_bf16_pair(gq.x, uq.x, xq.x, ag[j], au[j]);
+        fma2_bf16_pair(gq.y, uq.y, xq.y, ag[j], au[j]);
+        fma2_bf16_pair(gq.z, uq.z, xq.z, ag[j], au[j]);
+        fma2_bf16_pair(gq.w, uq.w, xq.w, ag[j], au[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const float g = warp_sum(ag[j]), uu = warp_sum(au[j]);
+      if (lane == 0) {
+        const int t = tok[j];
+        a.h[static_cast<int64_t>(t * a.k + m.slot_of[t][e]) * a.f + i] = __float2bfloat16_rn(silu_fast(g) * uu);
+      }
+    }
+  }
+};
+
+template <int NT>
+__device__ __forceinline__ void pair_job(const DecArgs& a, const DecSmem& m, const __nv_bfloat16* act,
+                                         const unsigned char* buf, int p, int lane) {
+  const int u = p / a.f, i = p - u * a.f;
+  const int e = m.touched[u];
+  int tok[NT];
+  const int n = mask_tokens<NT>(m.tokmask[e], tok);
+  PairBody<NT> body{a, m, reinterpret_cast<const uint4*>(buf), reinterpret_cast<const uint4*>(act), tok, e, i, lane};
+  with_count<1, NT>(n, body);
+}
+
+// One down row (in shared memory) against the h rows of its expert's n
+// tokens (slots slot[j]): the row is widened once for all of them.
+template <int NT>
+struct DownBody {
+  const uint4* w4;
+  const uint4* h4;
+  const int (&slot)[NT];
+  float* ps;  // this row's column: ps[slot]
+  int nvf, lane;
+  template <int N>
+  __device__ __forceinline__ void run() {
+    float acc[N];
+#pragma unroll
+    for (int j = 0; j < N; ++j) acc[j] = 0.f;
+    for (int v = lane; v < nvf; v += 32) {
+      const uint4 wq = w4[v];
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const uint4 hq = h4[slot[j] * nvf + v];
+        acc[j] = fma2_bf16(wq.x, hq.x, acc[j]);
+        acc[j] = fma2_bf16(wq.y, hq.y, acc[j]);
+        acc[j] = fma2_bf16(wq.z, hq.z, acc[j]);
+        acc[j] = fma2_bf16(wq.w, hq.w, acc[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const float r = warp_sum(acc[j]);
+      if (lane == 0) ps[slot[j]] = r;
+    }
+  }
+};
+
 // Phase-2 job g of this CTA (down rows g * rows_per_job ..., in `buf`): each
 // row's dot products with the h rows (shared memory) of its expert's tokens.
+template <int NT>
 __device__ __forceinline__ void down_job(const DecArgs& a, const DecSmem& m, const Share& sh, int nt,
                                          const __nv_bfloat16* act, float* ps, const unsigned char* buf, int g,
                                          int lane) {
   const int k = a.k, nvf = a.f / 8, TK = a.T * k;
   const int r0 = g * a.rows_per_job;
   const int nr = min(a.rows_per_job, sh.rows2 - r0);
-  const uint4* h4 = reinterpret_cast<const uint4*>(act);
   int cl = r0 / nt, u = r0 - cl * nt;  // the row's column (of this CTA's) and touched-expert index
   for (int rr = 0; rr < nr; ++rr) {
     const int e = m.touched[u];
-    const uint4* w4 = reinterpret_cast<const uint4*>(buf) + rr * nvf;
-    unsigned tm = m.tokmask[e];
-    while (tm != 0u) {
-      const int t = __ffs(tm) - 1;
-      tm &= tm - 1u;
-      const int slot = t * k + m.slot_of[t][e];
-      float acc = 0.f;
-      for (int v = lane; v < nvf; v += 32) {
-        float wv[8], hv[8];
-        bf16x8(w4[v], wv);
-        bf16x8(h4[slot * nvf + v], hv);
+    int slot[NT];
+    const int n = mask_tokens<NT>(m.tokmask[e], slot);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc = fmaf(wv[c], hv[c], acc);
-      }
-      acc = warp_sum(acc);
-      if (lane == 0) ps[cl * TK + slot] = acc;
-    }
+    for (int j = 0; j < NT; ++j) slot[j] = slot[j] * k + max(m.slot_of[slot[j]][e], 0);
+    DownBody<NT> body{reinterpret_cast<const uint4*>(buf) + rr * nvf, reinterpret_cast<const uint4*>(act), slot,
+                      ps + cl * TK, nvf, lane};
+    with_count<1, NT>(n, body);
     if (++u == nt) {
       u = 0;
       ++cl;
@@ -349,16 +485,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
   const int nvd = d / 8, nvf = a.f / 8;  // 16-byte vectors per row
   const int G = gridDim.x;
   const int SW = a.n_stream;
-  unsigned char* buf0 = smem_raw + a.buf_off + static_cast<size_t>(2 * warp) * a.job_bytes;
-  unsigned char* buf1 = buf0 + a.job_bytes;
 
   if (tid == 0) {
     m.abort = *reinterpret_cast<volatile int32_t*>(a.status) != 0 ? 1 : 0;
     m.bars = 0;
   }
   if (tid < kDecMaxLayers) m.layers[tid] = a.layer[tid];
+  if (tid < kDecJobBufs) mbar_init(&m.jbar[tid], 1);
+  fence_mbar_init();
   __syncthreads();
   if (m.abort != 0) return;  // a failure is recorded: the counters may be stale
+  JobPipe jp{m.jbar + warp * kDecBufsPerWarp,
+             smem_raw + a.buf_off + static_cast<size_t>(warp) * kDecBufsPerWarp * a.job_bytes, a.job_bytes, 0u, 0u,
+             warp < SW};
 
 #pragma unroll 1
   for (int l = 0; l < a.n_layers; ++l) {
@@ -414,12 +553,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
       const int e0 = lane, e1 = lane + 32;
       const double h0 = e0 < E ? m.hd[t][e0] : -INFINITY;
       const double h1 = e1 < E ? m.hd[t][e1] : -INFINITY;
-      // rank by (logit descending, index ascending): the experts ranked below k are the choice
+      // rank by (logit descending, index ascending): the experts ranked below k
+      // are the choice (unrolled and branch-free: a broadcast read and four
+      // compares per expert)
       int r0 = 0, r1 = 0;
-      for (int e = 0; e < E; ++e) {
-        const double v = m.hd[t][e];
-        r0 += (v > h0 || (v == h0 && e < e0)) ? 1 : 0;
-        r1 += (v > h1 || (v == h1 && e < e1)) ? 1 : 0;
+#pragma unroll
+      for (int e = 0; e < kDecMaxE; ++e) {
+        if (e < E) {
+          const double v = m.hd[t][e];
+          r0 += static_cast<int>(v > h0) | (static_cast<int>(v == h0) & static_cast<int>(e < e0));
+          r1 += static_cast<int>(v > h1) | (static_cast<int>(v == h1) & static_cast<int>(e < e1));
+        }
       }
       if (e0 < E) {
         m.slot_of[t][e0] = r0 < k ? r0 : -1;
@@ -446,17 +590,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
       if (e1 < E) m.p[t][e1] = x1 / sum;
       if (lane == 0) m.lse[t] = static_cast<float>(mx) + logf(sum);
       __syncwarp();
-      if (lane == 0) {  // weights in slot order (renormalised: over the k chosen, summed in slot order)
-        float den = 0.f;
-        for (int j = 0; j < k; ++j) den += m.p[t][m.sel_e[t * k + j]];
-        for (int j = 0; j < k; ++j) {
-          const int e = m.sel_e[t * k + j];
-          const float w = a.renorm ? m.p[t][e] / den : m.p[t][e];
-          m.sel_w[t * k + j] = w;
-          if (blockIdx.x == 0) {
-            if (idx_out != nullptr) idx_out[t * k + j] = e;
-            if (a.w_out != nullptr) a.w_out[t * k + j] = w;
-          }
+      // weights, lane j taking slot j (renormalised: over the k chosen, summed in slot order)
+      const int ej = lane < k ? m.sel_e[t * k + lane] : 0;
+      const float pj = lane < k ? m.p[t][ej] : 0.f;
+      float den = 0.f;
+      if (a.renorm)
+        for (int j = 0; j < k; ++j) den += __shfl_sync(0xffffffffu, pj, j);
+      if (lane < k) {
+        const float w = a.renorm ? pj / den : pj;
+        m.sel_w[t * k + lane] = w;
+        if (blockIdx.x == 0) {
+          if (idx_out != nullptr) idx_out[t * k + lane] = ej;
+          if (a.w_out != nullptr) a.w_out[t * k + lane] = w;
         }
       }
       __syncwarp();
@@ -506,21 +651,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
     const int c1 = streams ? pair_jobs(SW, warp, nt * a.f) : 0;
     const int c2 = streams && warp < sh.n2 ? (sh.n2 - warp + SW - 1) / SW : 0;
     if (streams) {
-      fetch_job(a, m, Ly, sh, nt, warp, lane, c1, c2, 0, buf0);
-      fetch_job(a, m, Ly, sh, nt, warp, lane, c1, c2, 1, buf1);
-      // ---- phase 1: the next job's copies in flight while this one is computed
+      for (int qq = 0; qq < kDecBufsPerWarp; ++qq) issue_job(a, m, Ly, sh, nt, warp, lane, c1, c2, qq, jp);
+      // ---- phase 1: the next jobs' copies in flight while this one is computed
       for (int qq = 0; qq < c1; ++qq) {
-        unsigned char* b = (qq & 1) ? buf1 : buf0;
-        cp_async_wait<1>();
-        __syncwarp();
-        pair_job<NT>(a, m, act, b, pair_index(SW, warp, qq), lane);
-        __syncwarp();
-        fetch_job(a, m, Ly, sh, nt, warp, lane, c1, c2, qq + 2, b);
+        if (await_job(jp, qq, a.status)) pair_job<NT>(a, m, act, jp.at(qq), pair_index(SW, warp, qq), lane);
+        issue_job(a, m, Ly, sh, nt, warp, lane, c1, c2, qq + kDecBufsPerWarp, jp);
       }
     }
     // every CTA's h is written before any CTA reads it
     if (!grid_barrier(m, a)) {
-      cp_async_wait<0>();  // no copy in flight when the CTA leaves
+      drain_jobs(jp);  // no copy in flight when the CTA leaves
       return;
     }
     {  // h of all slots into shared memory (x is dead)
@@ -533,14 +673,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
     // ---- phase 2
     if (streams) {
       for (int qq = c1; qq < c1 + c2; ++qq) {
-        unsigned char* b = (qq & 1) ? buf1 : buf0;
-        cp_async_wait<1>();
-        __syncwarp();
-        down_job(a, m, sh, nt, act, ps, b, warp + SW * (qq - c1), lane);
-        __syncwarp();
-        fetch_job(a, m, Ly, sh, nt, warp, lane, c1, c2, qq + 2, b);
+        if (await_job(jp, qq, a.status)) down_job<NT>(a, m, sh, nt, act, ps, jp.at(qq), warp + SW * (qq - c1), lane);
+        issue_job(a, m, Ly, sh, nt, warp, lane, c1, c2, qq + kDecBufsPerWarp, jp);
       }
-      cp_async_wait<0>();
+      drain_jobs(jp);
     }
     __syncthreads();
     // each (column, token): the weighted sum over the token's slots in slot order
@@ -562,8 +698,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
 }
 
 // Shared-memory plan for T tokens on a grid of G CTAs: bookkeeping, the
-// activation rows (x, later h), the per-column dot products, and two job
-// buffers for as many streaming warps (up to 16) as fit.
+// activation rows (x, later h), the per-column dot products, and
+// kDecBufsPerWarp job buffers for as many streaming warps (up to 16) as fit.
 struct DecPlan {
   uint32_t act_off, ps_off, buf_off, job_bytes;
   int rows_per_job, n_stream;
@@ -577,15 +713,16 @@ bool decode_plan(const Shape& s, int G, DecPlan* p) {
   const size_t act = align128(std::max(static_cast<size_t>(s.T) * s.d * 2, static_cast<size_t>(s.T) * s.k * s.f * 2));
   const size_t ps = align128(static_cast<size_t>(s.d / G + 1) * s.T * s.k * 4);
   const size_t jb = align128(std::max(static_cast<size_t>(s.d) * 4, static_cast<size_t>(s.f) * 2));
-  if (misc + act + ps + 2 * jb > kDecSmemCap) return false;
-  const size_t sw = std::min<size_t>(kMaxStreamWarps, (kDecSmemCap - misc - act - ps) / (2 * jb));
+  const size_t nb = kDecBufsPerWarp;
+  if (misc + act + ps + nb * jb > kDecSmemCap) return false;
+  const size_t sw = std::min<size_t>(kMaxStreamWarps, (kDecSmemCap - misc - act - ps) / (nb * jb));
   p->act_off = static_cast<uint32_t>(misc);
   p->ps_off = static_cast<uint32_t>(misc + act);
   p->buf_off = static_cast<uint32_t>(misc + act + ps);
   p->job_bytes = static_cast<uint32_t>(jb);
   p->rows_per_job = static_cast<int>(jb / (static_cast<size_t>(s.f) * 2));
   p->n_stream = static_cast<int>(sw);
-  p->smem = misc + act + ps + 2 * sw * jb;
+  p->smem = misc + act + ps + nb * sw * jb;
   return true;
 }
 
