@@ -49,6 +49,8 @@
 // every wait gives up after about a second, records a status and lets the
 // kernel finish; a launch that finds the status word set does nothing
 // (moe_get_device_status clears it and the counters).
+#include <climits>
+
 #include "moe_internal.h"
 #include "sm100.cuh"
 
@@ -109,8 +111,10 @@ struct DecSmem {
   int ok;                          // result of the last grid barrier
   int abort;                       // a failure is recorded: do nothing
   unsigned bars;                   // grid barriers passed in this launch
-  double rms[kDecMaxT];            // 1 / sqrt(mean square + eps) of each input row
+  double wss[kDecWarps];           // each warp's sum of squares (of its input row)
+  double rinv[kDecMaxT];           // 1 / sqrt(mean square + eps) of each input row
   double hd[kDecMaxT][kDecMaxE];   // logits (+ offset)
+  long long key[kDecMaxT][kDecMaxE];  // the logits as ordered integers (order_key)
   float p[kDecMaxT][kDecMaxE];
   float lse[kDecMaxT];
   DecLayer layers[kDecMaxLayers];  // the launch's layer table
@@ -143,6 +147,18 @@ __device__ __forceinline__ void bf16x8(const uint4& q, float (&v)[8]) {
     v[2 * j] = f.x;
     v[2 * j + 1] = f.y;
   }
+}
+
+// A double as a signed integer in the same order (-0 taken as +0), so that
+// comparisons run on the integer pipe (FP64 runs at a small fraction of the
+// FP32 rate on this part). A NaN becomes `nan_key`: the smallest integer for a
+// value compared against (it beats nothing), the largest for the value being
+// ranked (nothing beats it), as every comparison with NaN is false.
+__device__ __forceinline__ long long order_key(double x, long long nan_key) {
+  long long b = __double_as_longlong(x);
+  if ((b & 0x7FFFFFFFFFFFFFFFll) == 0) b = 0;
+  const long long k = b ^ ((b >> 63) & 0x7FFFFFFFFFFFFFFFll);
+  return (b & 0x7FFFFFFFFFFFFFFFll) > 0x7FF0000000000000ll ? nan_key : k;
 }
 
 // acc + a.lo * x.lo, then + a.hi * x.hi: two fused multiply-adds of bf16
@@ -472,6 +488,54 @@ __device__ __forceinline__ void down_job(const DecArgs& a, const DecSmem& m, con
   }
 }
 
+// The block's RMSNorm (unit weight) of the fp32 residual rows into the bf16
+// layer input `act`, all rows at once: 512 / T (rounded down to a power of
+// two, at least 64) threads per row. In fp64: each thread's squares in
+// element order, a butterfly within each warp, the row's warps in order; one
+// reciprocal root per row and a product per element, rounded to fp32, then to
+// bf16 (as the separate RMSNorm kernel rounds). The row is read twice, from
+// L2, so that no register holds it across the block barrier.
+__device__ __forceinline__ void stage_rmsnorm(const DecArgs& a, DecSmem& m, __nv_bfloat16* act) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = a.T, d = a.d, nv = d / 4;
+  const int tpr = T <= 1 ? kDecThreads : T <= 2 ? kDecThreads / 2 : T <= 4 ? kDecThreads / 4 : kDecThreads / 8;
+  const int row = tid / tpr, p = tid - row * tpr;
+  const bool live = row < T;
+  const float4* r = reinterpret_cast<const float4*>(a.resid + static_cast<int64_t>(row) * d);
+  double ss = 0.0;
+  if (live) {
+#pragma unroll 4
+    for (int i = p; i < nv; i += tpr) {
+      const float4 q = __ldcg(r + i);
+      ss = fma(static_cast<double>(q.x), static_cast<double>(q.x), ss);
+      ss = fma(static_cast<double>(q.y), static_cast<double>(q.y), ss);
+      ss = fma(static_cast<double>(q.z), static_cast<double>(q.z), ss);
+      ss = fma(static_cast<double>(q.w), static_cast<double>(q.w), ss);
+    }
+  }
+  ss = warp_sum_d(ss);  // a warp lies within one row
+  if (lane == 0) m.wss[warp] = ss;
+  __syncthreads();
+  if (tid < T) {
+    const int wpr = tpr / 32;
+    double sum = 0.0;
+    for (int w = tid * wpr; w < (tid + 1) * wpr; ++w) sum += m.wss[w];
+    m.rinv[tid] = 1.0 / sqrt(sum / static_cast<double>(d) + a.eps);
+  }
+  __syncthreads();
+  if (live) {
+    const double inv = m.rinv[row];
+#pragma unroll 4
+    for (int i = p; i < nv; i += tpr) {
+      const float4 q = __ldcg(r + i);
+      uint2 o;
+      o.x = pack_bf16x2(static_cast<float>(static_cast<double>(q.x) * inv), static_cast<float>(static_cast<double>(q.y) * inv));
+      o.y = pack_bf16x2(static_cast<float>(static_cast<double>(q.z) * inv), static_cast<float>(static_cast<double>(q.w) * inv));
+      *reinterpret_cast<uint2*>(act + static_cast<int64_t>(row) * d + 4 * i) = o;
+    }
+  }
+}
+
 // NT: tokens the phase-1 accumulators are sized for (1, 2, 4 or 8; T <= NT).
 template <int NT>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __grid_constant__ DecArgs a) {
@@ -513,23 +577,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
 
     // ---- prologue: the T input rows, bf16, in shared memory
     if (a.resid != nullptr) {
-      if (warp < T) {  // RMSNorm (unit weight) of token `warp` in fp64, mean of squares in a fixed order
-        const float* r = a.resid + static_cast<int64_t>(warp) * d;
-        double ss = 0.0;
-        for (int i = lane; i < d; i += 32) {
-          const double v = static_cast<double>(__ldcg(r + i));
-          ss = fma(v, v, ss);
-        }
-        ss = warp_sum_d(ss);
-        if (lane == 0) m.rms[warp] = 1.0 / sqrt(ss / static_cast<double>(d) + a.eps);
-        __syncwarp();
-      }
-      __syncthreads();
-      // the fp64 value rounded to fp32, then to bf16 (as the separate RMSNorm kernel does)
-      for (int t = 0; t < T; ++t)
-        for (int i = tid; i < d; i += kDecThreads)
-          act[t * d + i] = __float2bfloat16_rn(
-              static_cast<float>(static_cast<double>(__ldcg(a.resid + static_cast<int64_t>(t) * d + i)) * m.rms[t]));
+      stage_rmsnorm(a, m, act);
     } else {
       const uint4* src = reinterpret_cast<const uint4*>(a.x);
       uint4* dst = reinterpret_cast<uint4*>(act);
@@ -544,7 +592,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
     //      exact in fp32), lane l taking elements 8l + 256i; fixed reduction tree
     if (has_task) logit_task(a, Ly, act, q, lane);
     if (!grid_barrier(m, a)) return;
-    for (int i = tid; i < T * E; i += kDecThreads) m.hd[i / E][i % E] = __ldcg(a.logits + i);
+    for (int i = tid; i < T * E; i += kDecThreads) {
+      const double h = __ldcg(a.logits + i);
+      m.hd[i / E][i % E] = h;
+      m.key[i / E][i % E] = order_key(h, LLONG_MIN);
+    }
     __syncthreads();
 
     // ---- routing (every CTA): warp t takes token t; lane l holds experts l, l + 32
@@ -554,16 +606,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
       const double h0 = e0 < E ? m.hd[t][e0] : -INFINITY;
       const double h1 = e1 < E ? m.hd[t][e1] : -INFINITY;
       // rank by (logit descending, index ascending): the experts ranked below k
-      // are the choice (unrolled and branch-free: a broadcast read and four
-      // compares per expert)
+      // are the choice (branch-free integer compares of the keys; a short
+      // loop, as once-per-layer code runs from a cold instruction cache)
+      const long long k0 = order_key(h0, LLONG_MAX), k1 = order_key(h1, LLONG_MAX);
       int r0 = 0, r1 = 0;
-#pragma unroll
-      for (int e = 0; e < kDecMaxE; ++e) {
-        if (e < E) {
-          const double v = m.hd[t][e];
-          r0 += static_cast<int>(v > h0) | (static_cast<int>(v == h0) & static_cast<int>(e < e0));
-          r1 += static_cast<int>(v > h1) | (static_cast<int>(v == h1) & static_cast<int>(e < e1));
-        }
+#pragma unroll 4
+      for (int e = 0; e < E; ++e) {
+        const long long v = m.key[t][e];
+        r0 += static_cast<int>(v > k0) | (static_cast<int>(v == k0) & static_cast<int>(e < e0));
+        r1 += static_cast<int>(v > k1) | (static_cast<int>(v == k1) & static_cast<int>(e < e1));
       }
       if (e0 < E) {
         m.slot_of[t][e0] = r0 < k ? r0 : -1;
@@ -662,6 +713,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(const __gr
     if (!grid_barrier(m, a)) {
       drain_jobs(jp);  // no copy in flight when the CTA leaves
       return;
+    }
+    // the next layer's router rows of this warp's logit task, asked into L2
+    // now so that its logits do not wait on DRAM
+    if (lane == 0 && l + 1 < a.n_layers) {
+      const int q1 = warp * G + static_cast<int>(blockIdx.x);
+      if (q1 < T * E)
+        bulk_prefetch_l2(m.layers[l + 1].wr + static_cast<int64_t>(q1 / T) * d, static_cast<uint32_t>(d) * 2);
     }
     {  // h of all slots into shared memory (x is dead)
       const uint4* src = reinterpret_cast<const uint4*>(a.h);

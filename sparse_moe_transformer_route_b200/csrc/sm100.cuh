@@ -161,6 +161,13 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// Asks for `bytes` (a multiple of 16, 16-byte aligned) of global memory to be
+// brought into L2; nothing waits for it.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
+
 // Orders this thread's earlier generic-proxy accesses to shared memory before
 // its later async-proxy ones (a bulk copy into a buffer just read).
 __device__ __forceinline__ void fence_proxy_async_smem() {
