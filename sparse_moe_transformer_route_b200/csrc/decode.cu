@@ -790,7 +790,8 @@ bool decode_supported(const Shape& s) {
   if (s.fp32 || s.T < 1 || s.T > kDecMaxT || s.E > kDecMaxE || s.k > kMaxTopK) return false;
   if (s.d % 8 != 0 || s.f % 8 != 0) return false;  // 16-byte rows
   const size_t rows = std::max(static_cast<size_t>(s.T) * s.d, static_cast<size_t>(s.T) * s.k * s.f) * 2;
-  if (rows > 192 * 1024) return false;  // the staged rows (x, later h) in shared memory
+  // the staged rows (x, later h) and at least two job buffers in shared memory
+  if (rows + static_cast<size_t>(s.d) * 8 > 192 * 1024) return false;
   if (static_cast<size_t>(s.T) * s.E * 8 > static_cast<size_t>(s.P) * s.d * s.esize) return false;  // logits scratch
   DecPlan p;
   return decode_plan(s, device_sm_count(), &p);

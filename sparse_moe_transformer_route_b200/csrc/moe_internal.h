@@ -106,8 +106,8 @@ cudaError_t launch_combine_ec(const Shape& s, const void* o_perm, const int32_t*
 bool decode_supported(const Shape& s);
 // Batches the layer forward routes to the one-kernel form by itself: up to 4
 // tokens (measured on B200 in CUDA-graph replays, L2 flushed before each: T=1
-// 45 us, T=4 113 us; at T=6 and T=8 the layered tensor-core path is ahead,
-// about 155 against 217 and 307 us).
+// 45 us, T=4 102 us; at T=8 the layered tensor-core path is ahead, about 152
+// against 197 us).
 constexpr int64_t kDecodeAutoTokens = 4;
 cudaError_t launch_decode_layer(const Shape& s, const void* x, float* resid, double eps, const void* w_router,
                                 const float* bias, const void* w_gate_up, const void* w_down, void* y,
